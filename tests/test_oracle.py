@@ -1,0 +1,436 @@
+"""Pins for the CPU oracle, against facts fixed by the pages and by mathematics
+(closed forms, library routines on special cases, brute force on tiny inputs),
+never against the oracle itself.  No GPU."""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle
+from block_sparse_attention_pa_b200 import synth
+
+
+def bf16(a):
+    return torch.as_tensor(np.asarray(a, np.float32)).to(torch.bfloat16)
+
+
+def bits(t):
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def bf16_value(b):
+    return float(np.array([int(b) << 16], np.uint32).view(np.float32)[0])
+
+
+# ----------------------------------------------------------- bf16 rounding
+def test_bf16_rne_exact_and_midpoints():
+    """Every finite bf16 value maps to itself; the exact midpoint of two
+    neighbours goes to the one with an even last mantissa bit; points just off
+    the midpoint go to the nearer neighbour (IEEE roundTiesToEven)."""
+    f = oracle.f64_to_bf16_bits
+    for b in list(range(0x0000, 0x7F7F, 7)) + [0x0001, 0x007F, 0x0080, 0x3F80, 0x7F7E]:
+        v, w = bf16_value(b), bf16_value(b + 1)
+        assert f(v) == b and f(-v) == (b | 0x8000)
+        mid = (v + w) / 2.0
+        even = b if b % 2 == 0 else b + 1
+        assert f(mid) == even
+        assert f(-mid) == (even | 0x8000)
+        assert f(mid - (w - v) * 2.0 ** -20) == b
+        assert f(mid + (w - v) * 2.0 ** -20) == b + 1
+    # beyond the largest finite bf16 by half a spacing -> inf
+    big = bf16_value(0x7F7F)
+    assert f(big + (big - bf16_value(0x7F7E)) / 2) == 0x7F80
+    assert f(0.0) == 0 and f(-0.0) == 0x8000
+
+
+def test_bf16_rne_matches_torch_from_float32():
+    """On float32 inputs (exact in fp64) the oracle's rounding agrees with
+    torch's float32 -> bfloat16 conversion (round to nearest even)."""
+    rng = np.random.default_rng(0)
+    x = np.concatenate([rng.standard_normal(3000).astype(np.float32) * 10.0 ** rng.integers(-30, 30, 3000),
+                        rng.standard_normal(1000).astype(np.float32)]).astype(np.float32)
+    ref = bits(torch.from_numpy(x).to(torch.bfloat16))
+    got = np.array([oracle.f64_to_bf16_bits(float(v)) for v in x], np.uint16)
+    np.testing.assert_array_equal(got, ref)
+
+
+# ------------------------------------------------------------------- pool
+def test_pool_closed_form():
+    """H=4 heads with constant values 1,2,3,4; Hkv=2 KV heads with 10, 20.
+    G=1: Qp=2.5, Kp=mean(10,10,20,20)=15.  G=2: Qp=(1.5, 3.5), Kp=(10, 20)."""
+    N, d = 128, 8
+    q = torch.empty(1, N, 4, d)
+    for h in range(4):
+        q[:, :, h] = h + 1
+    k = torch.empty(1, N, 2, d)
+    k[:, :, 0], k[:, :, 1] = 10.0, 20.0
+    q, k = q.bfloat16(), k.bfloat16()
+    qp, kp, qpb, kpb = oracle.pool(q, k, 1)
+    assert np.all(qp == 2.5) and np.all(kp == 15.0)
+    qp, kp, qpb, kpb = oracle.pool(q, k, 2)
+    assert np.all(qp[0, 0] == 1.5) and np.all(qp[0, 1] == 3.5)
+    assert np.all(kp[0, 0] == 10.0) and np.all(kp[0, 1] == 20.0)
+    assert torch.equal(qpb.float(), torch.from_numpy(qp).float())
+
+
+def test_pool_one_head_per_group_is_identity():
+    """G = H: each proxy is its own head, bit for bit (Q), and the KV head of that
+    q head (K)."""
+    w = synth.small_workload(seqlen=256, heads=4, kv_heads=2, head_dim=64, groups=4)
+    x = synth.make_inputs(w)
+    q, k = x["q"], x["k"]
+    _, _, qpb, kpb = oracle.pool(q, k, 4)
+    for h in range(4):
+        assert torch.equal(qpb[0, h], q[0, :, h])
+        assert torch.equal(kpb[0, h], k[0, :, h * 2 // 4])
+
+
+def test_pool_matches_numpy_mean_and_head_permutation():
+    w = synth.small_workload(seqlen=256, heads=8, kv_heads=4, head_dim=64, groups=2)
+    x = synth.make_inputs(w)
+    q, k = x["q"], x["k"]
+    qp, kp, qpb, kpb = oracle.pool(q, k, 2)
+    qn = q.double().numpy()
+    kn = k.double().numpy()
+    for g in range(2):
+        heads = list(range(4 * g, 4 * g + 4))
+        np.testing.assert_allclose(qp[0, g], qn[0][:, heads].mean(axis=1), rtol=1e-15, atol=0)
+        kvs = [h * 4 // 8 for h in heads]
+        np.testing.assert_allclose(kp[0, g], kn[0][:, kvs].mean(axis=1), rtol=1e-15, atol=0)
+    # permuting the heads inside each group leaves the proxies unchanged
+    perm = [3, 1, 0, 2, 7, 6, 4, 5]
+    qp2, _, qpb2, _ = oracle.pool(q[:, :, perm].contiguous(), k, 2)
+    assert np.array_equal(qp, qp2) and torch.equal(qpb, qpb2)
+
+
+def test_pool_strided_input_equals_contiguous():
+    w = synth.small_workload(seqlen=256, heads=4, kv_heads=2, head_dim=64)
+    x = synth.make_inputs(w)
+    packed = torch.cat([x["q"], x["k"], x["v"]], dim=2)  # [B, N, H+2Hkv, d]
+    q, k = packed[:, :, :4], packed[:, :, 4:6]
+    assert not q.is_contiguous()
+    a = oracle.pool(q, k, 1)
+    b = oracle.pool(x["q"], x["k"], 1)
+    assert torch.equal(a[2], b[2]) and torch.equal(a[3], b[3])
+
+
+# ----------------------------------------------------------------- scores
+def brute_block_max(qh, kh, scale):
+    """Per-head causal block maxima of scale * q k^T by numpy (fp64)."""
+    N = qh.shape[0]
+    nb = N // 128
+    s = (qh @ kh.T) * scale
+    s[np.triu_indices(N, 1)] = -np.inf
+    out = []
+    for qb in range(nb):
+        for kb in range(qb + 1):
+            out.append(s[qb * 128:(qb + 1) * 128, kb * 128:(kb + 1) * 128].max())
+    return np.array(out)
+
+
+def test_scores_one_head_per_group_equal_per_head_scores():
+    """Check (b): MHA with G = H, so each proxy is one head; the proxy block
+    scores equal each head's own causal block maxima."""
+    w = synth.small_workload(seqlen=384, heads=3, kv_heads=3, head_dim=64, groups=3)
+    x = synth.make_inputs(w)
+    q, k = x["q"], x["k"]
+    _, _, qpb, kpb = oracle.pool(q, k, 3)
+    sc = oracle.block_scores(qpb, kpb)
+    for h in range(3):
+        ref = brute_block_max(q[0, :, h].double().numpy(), k[0, :, h].double().numpy(), 1 / 8.0)
+        np.testing.assert_allclose(sc[0, h], ref, rtol=1e-13, atol=1e-13)
+
+
+def test_scores_planted_pair_and_causal_mask():
+    """All-zero proxies except one query row i and key rows j: the tile holding
+    (i, j) scores a*b/sqrt(d); a larger product placed above the diagonal
+    (j > i, same block) must not count; every other tile scores 0."""
+    N, d = 512, 64
+    qp = torch.zeros(1, 1, N, d)
+    kp = torch.zeros(1, 1, N, d)
+    qp[0, 0, 300, 5] = 2.0          # row 300 -> qb 2
+    kp[0, 0, 140, 5] = 3.0          # key 140 -> kb 1: score 6/8 at (2, 1)
+    kp[0, 0, 310, 5] = 16.0         # key 310 > 300 in the diagonal tile: masked
+    sc = oracle.block_scores(qp.bfloat16(), kp.bfloat16())[0, 0]
+    tri = lambda qb: qb * (qb + 1) // 2
+    assert sc[tri(2) + 1] == pytest.approx(6.0 / 8.0)
+    assert sc[tri(2) + 2] == 0.0
+    # row 310 > key 310? no: row 311+ sees key 310 only if qp is nonzero there; it is zero
+    mask = np.ones_like(sc, bool)
+    mask[tri(2) + 1] = False
+    assert np.all(sc[mask] == 0.0)
+    # negative products: max keeps the largest (least negative) valid entry
+    qp2 = torch.zeros(1, 1, 256, d)
+    qp2[0, 0, :, 0] = -1.0
+    kp2 = torch.zeros(1, 1, 256, d)
+    kp2[0, 0, :, 0] = torch.linspace(1, 2, 256)
+    sc2 = oracle.block_scores(qp2.bfloat16(), kp2.bfloat16())[0, 0]
+    kv = kp2.bfloat16().double()[0, 0, :, 0].numpy()
+    assert sc2[0] == pytest.approx(-kv[0] / 8)       # tile (0,0): smallest key
+    assert sc2[1] == pytest.approx(-kv[0] / 8)       # tile (1,0)
+    assert sc2[2] == pytest.approx(-kv[128] / 8)     # tile (1,1)
+
+
+def test_score_tiles_equal_full_scores():
+    w = synth.small_workload(seqlen=384, heads=4, kv_heads=2, head_dim=64, groups=2)
+    x = synth.make_inputs(w)
+    _, _, qpb, kpb = oracle.pool(x["q"], x["k"], 2)
+    sc = oracle.block_scores(qpb, kpb)
+    tiles = [(0, 1, 2, 0), (0, 0, 1, 1), (0, 1, 0, 0)]
+    got = oracle.block_score_tiles(qpb, kpb, tiles)
+    tri = lambda qb: qb * (qb + 1) // 2
+    for (b, g, qb, kb), v in zip(tiles, got):
+        assert v == sc[b, g, tri(qb) + kb]
+
+
+# ------------------------------------------------------------------- mass
+def test_mass_rows_sum_to_one_and_match_scipy_softmax():
+    """Check (d) and a library pin: mass from scipy.special.softmax rows."""
+    w = synth.small_workload(seqlen=384, heads=4, kv_heads=2, head_dim=64)
+    x = synth.make_inputs(w)
+    q, k = x["q"], x["k"]
+    mass, dev = oracle.head_mass(q, k, with_rowsum=True)
+    assert np.all(dev < 1e-12)
+    np.testing.assert_allclose(mass.sum(-1), 1.0, atol=1e-12)
+    N = 384
+    for h in range(4):
+        qh = q[0, N - 128:, h].double().numpy()
+        kh = k[0, :, h * 2 // 4].double().numpy()
+        z = qh @ kh.T / 8.0
+        rows = np.arange(N - 128, N)
+        z[np.arange(N)[None, :] > rows[:, None]] = -np.inf
+        p = scipy.special.softmax(z, axis=1)
+        ref = p.reshape(128, 3, 128).sum(-1).mean(0)
+        np.testing.assert_allclose(mass[0, h], ref, rtol=1e-12, atol=1e-15)
+
+
+def test_mass_single_block_is_one():
+    w = synth.small_workload(seqlen=128, heads=2, kv_heads=1, head_dim=64)
+    x = synth.make_inputs(w)
+    mass = oracle.head_mass(x["q"], x["k"])
+    np.testing.assert_allclose(mass, 1.0, atol=1e-13)
+
+
+# ------------------------------------------------------------------- rank
+def brute_rank_row(row, qb):
+    """The unique order of blocks 1..qb-1 in which every neighbour pair is
+    (higher score first) or (equal score, lower index first), found by
+    enumerating permutations."""
+    rest = list(range(1, qb))
+    for perm in itertools.permutations(rest):
+        ok = all(row[a] > row[b] or (row[a] == row[b] and a < b) for a, b in zip(perm, perm[1:]))
+        if ok:
+            return [0, qb] + list(perm)
+    raise AssertionError
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_rank_brute_force_with_ties(seed):
+    nb = 8
+    rng = np.random.default_rng(seed)
+    T = nb * (nb + 1) // 2
+    scores = rng.integers(0, 4, size=(1, 2, T)).astype(np.float64) * 0.5 - 0.7  # many ties
+    r = oracle.rank(scores, nb)
+    for g in range(2):
+        for qb in range(nb):
+            row = scores[0, g, qb * (qb + 1) // 2: qb * (qb + 1) // 2 + qb + 1]
+            got = list(r[0, g, qb * (qb + 1) // 2: qb * (qb + 1) // 2 + qb + 1])
+            exp = [0] if qb == 0 else brute_rank_row(row, qb)
+            assert got == exp
+
+
+def test_rank_treats_float32_scores_exactly():
+    """Scores that differ only in the last float32 bit keep their order."""
+    nb = 4
+    a = np.float32(1.0)
+    b = np.nextafter(a, np.float32(2.0))
+    s = np.zeros((1, 1, 10), np.float32)
+    s[0, 0, 6:10] = [0.0, a, b, 5.0]  # row qb=3: blocks 0..3
+    r = oracle.rank(s, nb)
+    assert list(r[0, 0, 6:10]) == [0, 3, 2, 1]
+
+
+# ----------------------------------------------------------------- budget
+def fx(m):
+    return int(np.rint(m * 2.0 ** 40))
+
+
+def brute_budget(list_last, mass_h, gamma, nb):
+    F = 1 if nb == 1 else 2
+    g = fx(gamma)
+    for k in range(F, nb + 1):
+        if sum(fx(mass_h[b]) for b in list_last[:k]) >= g:
+            return k
+    return nb
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_budget_brute_force_and_invariants(seed):
+    rng = np.random.default_rng(seed)
+    nb, H, G = 9, 4, 2
+    T = nb * (nb + 1) // 2
+    scores = rng.standard_normal((1, G, T))
+    r = oracle.rank(scores, nb)
+    mass = rng.dirichlet(np.ones(nb) * 0.3, size=(1, H))
+    for gamma in [0.05, 0.5, 0.8, 0.95, 0.999, 1.0]:
+        bud, cnt = oracle.budget(r, mass, H, G, nb, oracle.DYNAMIC, gamma)
+        for h in range(H):
+            g = h * G // H
+            last = list(r[0, g, T - nb:])
+            k = brute_budget(last, mass[0, h], gamma, nb)
+            assert bud[0, h] == k
+            # invariants: prefix reaches gamma; one block fewer does not (unless at |F|)
+            pre = lambda n: sum(fx(mass[0, h][b]) for b in last[:n])
+            if k < nb or pre(nb) >= fx(gamma):
+                assert pre(k) >= fx(gamma)
+            if k > 2:
+                assert pre(k - 1) < fx(gamma)
+            assert cnt[0, h, nb - 1] == k
+            for qb in range(nb):
+                exp = min(max(-(-k * (qb + 1) // nb), 1 if qb == 0 else 2), qb + 1)
+                assert cnt[0, h, qb] == exp
+
+
+def test_budget_nested_in_gamma():
+    rng = np.random.default_rng(5)
+    nb, H = 16, 2
+    T = nb * (nb + 1) // 2
+    r = oracle.rank(rng.standard_normal((1, 1, T)), nb)
+    mass = rng.dirichlet(np.ones(nb), size=(1, H))
+    prev = None
+    for gamma in np.linspace(0.01, 1.0, 25):
+        bud, cnt = oracle.budget(r, mass, H, 1, nb, oracle.DYNAMIC, float(gamma))
+        if prev is not None:
+            assert np.all(cnt >= prev)
+        prev = cnt
+
+
+def test_budget_is_find_blocks_when_ranking_follows_mass():
+    """XAttention's find_blocks: the smallest block set whose mass reaches the
+    threshold.  When the shared ranking orders blocks by this head's own mass,
+    the oracle's prefix rule gives the size of the smallest such set among all
+    subsets that contain the forced sink and diagonal blocks (brute force over
+    all subsets)."""
+    rng = np.random.default_rng(11)
+    nb = 8
+    T = nb * (nb + 1) // 2
+    for trial in range(6):
+        m = rng.dirichlet(np.ones(nb) * 0.5)
+        scores = np.zeros((1, 1, T))
+        scores[0, 0, T - nb:] = m  # last row ranked by the head's mass
+        r = oracle.rank(scores, nb)
+        for gamma in [0.3, 0.6, 0.9]:
+            bud, _ = oracle.budget(r, m[None, None], 1, 1, nb, oracle.DYNAMIC, gamma)
+            best = nb
+            others = list(range(1, nb - 1))
+            for size in range(0, nb - 1):
+                for sub in itertools.combinations(others, size):
+                    s = [0, nb - 1] + list(sub)
+                    if sum(fx(m[b]) for b in s) >= fx(gamma):
+                        best = min(best, len(s))
+            assert bud[0, 0] == best
+
+
+def test_fixed_and_all_counts_closed_form():
+    nb, H = 10, 3
+    T = nb * (nb + 1) // 2
+    r = oracle.rank(np.zeros((1, 1, T)), nb)
+    bud, cnt = oracle.budget(r, None, H, 1, nb, oracle.FIXED_FRACTION, frac_permille=250)
+    for qb in range(nb):
+        assert cnt[0, 0, qb] == min(max(math.ceil(250 * (qb + 1) / 1000), 1 if qb == 0 else 2), qb + 1)
+    assert bud[0, 0] == 3
+    bud, cnt = oracle.budget(r, None, H, 1, nb, oracle.ALL)
+    assert np.all(cnt[0] == np.arange(1, nb + 1)) and np.all(bud == nb)
+
+
+# -------------------------------------------------------------- attention
+def sdpa_reference(q, k, v, mask=None):
+    """torch scaled_dot_product_attention in fp64 on [B, N, H, d] tensors (GQA
+    by repeating KV heads); causal unless an explicit boolean mask [N, N] or
+    [H, N, N] is given."""
+    B, N, H, d = q.shape
+    rep = H // k.shape[2]
+    qq = q.double().permute(0, 2, 1, 3)
+    kk = k.double().repeat_interleave(rep, dim=2).permute(0, 2, 1, 3)
+    vv = v.double().repeat_interleave(rep, dim=2).permute(0, 2, 1, 3)
+    if mask is None:
+        o = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, is_causal=True)
+    else:
+        o = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, attn_mask=mask)
+    return o.permute(0, 2, 1, 3)
+
+
+def test_dense_matches_torch_sdpa():
+    w = synth.small_workload(seqlen=256, heads=4, kv_heads=2, head_dim=64)
+    x = synth.make_inputs(w)
+    q, k, v = x["q"], x["k"], x["v"]
+    rows = [(0, h, i) for h in range(4) for i in [0, 1, 127, 128, 200, 255]]
+    o, lse = oracle.dense_attn(q, k, v, rows)
+    ref = sdpa_reference(q, k, v)
+    for (b, h, i), oo in zip(rows, o):
+        np.testing.assert_allclose(oo, ref[b, i, h].numpy(), rtol=1e-12, atol=1e-12)
+    # lse against torch.logsumexp
+    for (b, h, i), l in zip(rows, lse):
+        z = (q[b, i, h].double() @ k[b, :i + 1, h * 2 // 4].double().T) / 8.0
+        assert l == pytest.approx(torch.logsumexp(z, 0).item(), abs=1e-12)
+
+
+def test_sparse_all_equals_dense():
+    """Check (a): with the budget covering every causal block, block-sparse
+    attention is dense causal softmax attention."""
+    w = synth.small_workload(seqlen=384, heads=4, kv_heads=2, head_dim=64)
+    x = synth.make_inputs(w)
+    q, k, v = x["q"], x["k"], x["v"]
+    m = oracle.prefill_masks(q, k, 1, mode=oracle.ALL)
+    items = [(0, h, qb) for h in range(4) for qb in range(3)]
+    o, lse = oracle.sparse_attn(q, k, v, m["rank"], m["cnt"], 1, items)
+    rows = [(0, h, qb * 128 + i) for (_, h, qb) in items for i in range(128)]
+    od, lsed = oracle.dense_attn(q, k, v, rows)
+    np.testing.assert_allclose(o.reshape(-1, 64), od, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse.reshape(-1), lsed, rtol=0, atol=1e-12)
+
+
+def test_sparse_matches_sdpa_with_block_mask():
+    """Block-sparse attention equals torch SDPA (fp64) under the explicit
+    token mask built from the selected blocks and causality."""
+    w = synth.small_workload(seqlen=512, heads=4, kv_heads=2, head_dim=64, groups=2)
+    x = synth.make_inputs(w)
+    q, k, v = x["q"], x["k"], x["v"]
+    m = oracle.prefill_masks(q, k, 2, mode=oracle.FIXED_FRACTION, frac_permille=500)
+    nb = 4
+    mask = torch.zeros(4, 512, 512, dtype=torch.bool)
+    for h in range(4):
+        g = h * 2 // 4
+        for qb in range(nb):
+            sel = m["rank"][0, g, qb * (qb + 1) // 2: qb * (qb + 1) // 2 + m["cnt"][0, h, qb]]
+            for kb in sel:
+                mask[h, qb * 128:(qb + 1) * 128, kb * 128:(kb + 1) * 128] = True
+    mask &= torch.ones(512, 512, dtype=torch.bool).tril()[None]
+    ref = sdpa_reference(q, k, v, mask=mask[None])
+    items = [(0, h, qb) for h in range(4) for qb in range(nb)]
+    o, _ = oracle.sparse_attn(q, k, v, m["rank"], m["cnt"], 2, items)
+    for (b, h, qb), oo in zip(items, o):
+        np.testing.assert_allclose(oo, ref[0, qb * 128:(qb + 1) * 128, h].numpy(), rtol=1e-12, atol=1e-12)
+    # a head that keeps fewer blocks really attends to fewer keys
+    assert (m["cnt"][0, :, 3] < 4).all()
+
+
+def test_attention_head_dim_one_textbook_softmax():
+    """d = 1, N = 128: O_i = sum_j softmax(q_i k_j)_j v_j over j <= i, written
+    with numpy exp."""
+    N = 128
+    rng = np.random.default_rng(3)
+    q = bf16(rng.standard_normal((1, N, 1, 1)))
+    k = bf16(rng.standard_normal((1, N, 1, 1)))
+    v = bf16(rng.standard_normal((1, N, 1, 1)))
+    m = oracle.prefill_masks(q, k, 1, mode=oracle.ALL)
+    o, _ = oracle.sparse_attn(q, k, v, m["rank"], m["cnt"], 1, [(0, 0, 0)])
+    qd, kd, vd = (t.double().numpy().reshape(N) for t in (q, k, v))
+    for i in range(N):
+        z = qd[i] * kd[:i + 1]
+        p = np.exp(z - z.max())
+        p /= p.sum()
+        assert o[0, i, 0] == pytest.approx(float(p @ vd[:i + 1]), abs=1e-13)
