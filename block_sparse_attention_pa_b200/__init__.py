@@ -1,0 +1,245 @@
+"""Python binding of libpa.so: ProxyAttn-style block-sparse prefill attention
+on B200 (sm_100a).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels of
+``libpa.so`` behind its C ABI (``include/pa.h``).  PyTorch provides device
+memory and the current stream.  There is no CPU fallback: if the library is
+missing or a tensor is not on a CUDA device, the call raises.
+
+Functions mirror the C entry points:
+  pool_heads, block_scores, build_mask, block_sparse_attn, prefill,
+  workspace_size, device_status.
+Tensors use the [B, N, heads, d] layout (any strides with d contiguous).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libpa.so")
+
+DYNAMIC, FIXED_FRACTION, ALL = 0, 1, 2
+
+STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_ERR_WORKSPACE",
+          4: "PA_ERR_CUDA", 5: "PA_ERR_TIMEOUT", 6: "PA_ERR_DEVICE_BOUNDS", 7: "PA_ERR_DEVICE_NONFINITE"}
+
+# Every entry point declared in include/pa.h.
+ENTRY_POINTS = ("pa_workspace_size", "pa_pool_heads", "pa_block_scores", "pa_build_mask",
+                "pa_block_sparse_attn", "pa_prefill", "pa_get_device_status", "pa_status_string",
+                "pa_last_error", "pa_abi_version")
+
+
+class PaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{STATUS.get(code, code)}: {msg}")
+        self.code = code
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("seqlen", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("num_groups", ctypes.c_int32)]
+
+
+class Strides(ctypes.Structure):
+    _fields_ = [("b", ctypes.c_int64), ("s", ctypes.c_int64), ("h", ctypes.c_int64)]
+
+
+class Budget(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int32), ("gamma", ctypes.c_float), ("frac_permille", ctypes.c_int32)]
+
+
+class MaskBufs(ctypes.Structure):
+    _fields_ = [("rank", ctypes.c_void_p), ("cnt", ctypes.c_void_p), ("budget", ctypes.c_void_p),
+                ("mass", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libpa.so; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m block_sparse_attention_pa_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, P = ctypes.c_void_p, ctypes.POINTER
+        st = Strides
+        L.pa_workspace_size.restype = ctypes.c_size_t
+        L.pa_workspace_size.argtypes = [P(Shape), P(Budget)]
+        L.pa_pool_heads.argtypes = [P(Shape), vp, st, vp, st, vp, vp, vp]
+        L.pa_block_scores.argtypes = [P(Shape), vp, vp, vp, vp]
+        L.pa_build_mask.argtypes = [P(Shape), P(Budget), vp, vp, st, vp, st, P(MaskBufs), vp, ctypes.c_size_t, vp]
+        L.pa_block_sparse_attn.argtypes = [P(Shape), vp, st, vp, st, vp, st, vp, vp, ctypes.c_float, vp, st, vp, vp]
+        L.pa_prefill.argtypes = [P(Shape), P(Budget), vp, st, vp, st, vp, st, vp, st, P(MaskBufs), vp,
+                                 ctypes.c_size_t, vp]
+        L.pa_get_device_status.argtypes = [vp, ctypes.c_int]
+        L.pa_status_string.restype = ctypes.c_char_p
+        L.pa_status_string.argtypes = [ctypes.c_int]
+        L.pa_last_error.restype = ctypes.c_char_p
+        L.pa_abi_version.restype = ctypes.c_int32
+        for name in ("pa_pool_heads", "pa_block_scores", "pa_build_mask", "pa_block_sparse_attn", "pa_prefill",
+                     "pa_get_device_status"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(code: int):
+    if code != 0:
+        msg = lib().pa_last_error().decode() or lib().pa_status_string(code).decode()
+        raise PaError(code, msg)
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _strides(t: torch.Tensor) -> Strides:
+    return Strides(t.stride(0), t.stride(1), t.stride(2))
+
+
+def _cuda_bf16(t: torch.Tensor, name: str):
+    if not (isinstance(t, torch.Tensor) and t.is_cuda):
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if t.dtype != torch.bfloat16 or t.dim() != 4 or t.stride(3) != 1:
+        raise ValueError(f"{name} must be bf16 [B, N, heads, d] with a contiguous last dimension")
+
+
+def make_shape(q: torch.Tensor, k: torch.Tensor, num_groups: int) -> Shape:
+    B, N, H, d = q.shape
+    return Shape(B, N, H, k.shape[2], d, 128, num_groups)
+
+
+def make_budget(mode: int = DYNAMIC, gamma: float = 0.95, frac_permille: int = 0) -> Budget:
+    return Budget(mode, gamma, frac_permille)
+
+
+def workspace_size(shape: Shape, budget: Budget) -> int:
+    return int(lib().pa_workspace_size(ctypes.byref(shape), ctypes.byref(budget)))
+
+
+@dataclass
+class Mask:
+    """Device mask buffers (see pa_mask in include/pa.h)."""
+    rank: torch.Tensor     # int32 [B, G, T]
+    cnt: torch.Tensor      # int32 [B, H, nb]
+    budget: torch.Tensor   # int32 [B, H]
+    mass: torch.Tensor | None  # float32 [B, H, nb] (dynamic mode)
+
+    @staticmethod
+    def empty(shape: Shape, device, with_mass: bool) -> "Mask":
+        nb = shape.seqlen // 128
+        T = nb * (nb + 1) // 2
+        i32 = dict(device=device, dtype=torch.int32)
+        return Mask(torch.empty(shape.batch, shape.num_groups, T, **i32),
+                    torch.empty(shape.batch, shape.num_q_heads, nb, **i32),
+                    torch.empty(shape.batch, shape.num_q_heads, **i32),
+                    torch.empty(shape.batch, shape.num_q_heads, nb, device=device, dtype=torch.float32)
+                    if with_mass else None)
+
+    def bufs(self) -> MaskBufs:
+        return MaskBufs(self.rank.data_ptr(), self.cnt.data_ptr(), self.budget.data_ptr(),
+                        self.mass.data_ptr() if self.mass is not None else None)
+
+
+def pool_heads(q: torch.Tensor, k: torch.Tensor, num_groups: int):
+    """pa_pool_heads -> (q_proxy, k_proxy), bf16 [B, G, N, d]."""
+    _cuda_bf16(q, "q")
+    _cuda_bf16(k, "k")
+    shape = make_shape(q, k, num_groups)
+    B, N, H, d = q.shape
+    qp = torch.empty(B, num_groups, N, d, device=q.device, dtype=torch.bfloat16)
+    kp = torch.empty_like(qp)
+    _check(lib().pa_pool_heads(ctypes.byref(shape), q.data_ptr(), _strides(q), k.data_ptr(), _strides(k),
+                               qp.data_ptr(), kp.data_ptr(), _stream(q.device)))
+    return qp, kp
+
+
+def block_scores(q_proxy: torch.Tensor, k_proxy: torch.Tensor, num_q_heads: int = 1, num_kv_heads: int = 1):
+    """pa_block_scores -> fp32 [B, G, T]."""
+    for t, n in ((q_proxy, "q_proxy"), (k_proxy, "k_proxy")):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and t.dim() == 4):
+            raise ValueError(f"{n} must be a contiguous bf16 CUDA tensor [B, G, N, d]")
+    B, G, N, d = q_proxy.shape
+    H = max(num_q_heads, G)
+    shape = Shape(B, N, H, min(num_kv_heads, H), d, 128, G)
+    nb = N // 128
+    scores = torch.empty(B, G, nb * (nb + 1) // 2, device=q_proxy.device, dtype=torch.float32)
+    _check(lib().pa_block_scores(ctypes.byref(shape), q_proxy.data_ptr(), k_proxy.data_ptr(), scores.data_ptr(),
+                                 _stream(q_proxy.device)))
+    return scores
+
+
+def build_mask(scores: torch.Tensor, q: torch.Tensor, k: torch.Tensor, num_groups: int, mode: int = DYNAMIC,
+               gamma: float = 0.95, frac_permille: int = 0, workspace: torch.Tensor | None = None) -> Mask:
+    """pa_build_mask -> Mask."""
+    _cuda_bf16(q, "q")
+    _cuda_bf16(k, "k")
+    shape = make_shape(q, k, num_groups)
+    budget = make_budget(mode, gamma, frac_permille)
+    mask = Mask.empty(shape, q.device, mode == DYNAMIC)
+    if workspace is None:
+        workspace = torch.empty(max(workspace_size(shape, budget), 256), device=q.device, dtype=torch.uint8)
+    bufs = mask.bufs()
+    _check(lib().pa_build_mask(ctypes.byref(shape), ctypes.byref(budget), scores.data_ptr(), q.data_ptr(),
+                               _strides(q), k.data_ptr(), _strides(k), ctypes.byref(bufs), workspace.data_ptr(),
+                               workspace.numel(), _stream(q.device)))
+    return mask
+
+
+def block_sparse_attn(q, k, v, rank, cnt, num_groups: int, softmax_scale: float | None = None,
+                      out: torch.Tensor | None = None, return_lse: bool = False):
+    """pa_block_sparse_attn -> o (bf16 [B, N, H, d]) [, lse fp32 [B, H, N]]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _cuda_bf16(t, n)
+    shape = make_shape(q, k, num_groups)
+    B, N, H, d = q.shape
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
+    o = torch.empty_like(q, memory_format=torch.contiguous_format) if out is None else out
+    lse = torch.empty(B, H, N, device=q.device, dtype=torch.float32) if return_lse else None
+    _check(lib().pa_block_sparse_attn(ctypes.byref(shape), q.data_ptr(), _strides(q), k.data_ptr(), _strides(k),
+                                      v.data_ptr(), _strides(v), rank.data_ptr(), cnt.data_ptr(), scale,
+                                      o.data_ptr(), _strides(o), lse.data_ptr() if lse is not None else None,
+                                      _stream(q.device)))
+    return (o, lse) if return_lse else o
+
+
+class Prefill:
+    """A reusable pa_prefill call: workspace and mask buffers allocated once."""
+
+    def __init__(self, q, k, v, num_groups: int, mode: int = DYNAMIC, gamma: float = 0.95, frac_permille: int = 0):
+        for t, n in ((q, "q"), (k, "k"), (v, "v")):
+            _cuda_bf16(t, n)
+        self.shape = make_shape(q, k, num_groups)
+        self.budget = make_budget(mode, gamma, frac_permille)
+        self.mask = Mask.empty(self.shape, q.device, mode == DYNAMIC)
+        self.ws = torch.empty(workspace_size(self.shape, self.budget), device=q.device, dtype=torch.uint8)
+        self._bufs = self.mask.bufs()
+
+    def __call__(self, q, k, v, out):
+        _check(lib().pa_prefill(ctypes.byref(self.shape), ctypes.byref(self.budget), q.data_ptr(), _strides(q),
+                                k.data_ptr(), _strides(k), v.data_ptr(), _strides(v), out.data_ptr(),
+                                _strides(out), ctypes.byref(self._bufs), self.ws.data_ptr(), self.ws.numel(),
+                                _stream(q.device)))
+        return out
+
+
+def prefill(q, k, v, num_groups: int, mode: int = DYNAMIC, gamma: float = 0.95, frac_permille: int = 0):
+    """pa_prefill -> (o, Mask)."""
+    call = Prefill(q, k, v, num_groups, mode, gamma, frac_permille)
+    o = torch.empty_like(q, memory_format=torch.contiguous_format)
+    call(q, k, v, o)
+    return o, call.mask
+
+
+def device_status(clear: bool = True, device=None) -> int:
+    """pa_get_device_status: syncs the current stream; 0 if no kernel recorded a problem."""
+    return int(lib().pa_get_device_status(_stream(device), 1 if clear else 0))

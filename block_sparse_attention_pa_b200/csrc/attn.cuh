@@ -1,0 +1,335 @@
+// attn.cuh -- causal block-sparse FlashAttention on tcgen05 (ProxyAttn blog:
+// the block-sparse mask "fed to FlashAttention", end of "4. ProxyAttn
+// method"; the attention formula of "2. Background").
+//
+// One CTA computes one query block (128 rows) of one or two heads that share
+// a KV head and a proxy group.  The two heads share the group's ranked list;
+// head t visits its first cnt_t entries, so a K/V tile is loaded once for
+// both heads while both still need it.
+//
+// Warp roles (320 threads, one CTA per SM, all 512 TMEM columns):
+//   warp 0     TMA producer: the two Q tiles once, then K and V tiles of the
+//              listed blocks into a ring (128-byte swizzle).
+//   warp 1     TMEM owner and single-thread tcgen05.mma issuer:
+//                S_t = Q_t K^T   (M=128, N=128, K=16 steps; A, B K-major smem)
+//                O_t += P_t V    (M=128, N=d,   A = P_t read from TMEM,
+//                                 B = V, MN-major smem)
+//              in ping-pong order  PV_0(i), QK_0(i+1), PV_1(i), QK_1(i+1), so
+//              the tensor core computes one head's products while the other
+//              head's softmax runs.
+//   warps 2-5  softmax of head 0, warps 6-9 softmax of head 1: one thread per
+//              query row (TMEM lane).  Two passes over S in TMEM (row max,
+//              then exp2/row sum/bf16 pack of P written back over S), online
+//              softmax with the running max raised only when it grows by more
+//              than 2^8 (then O is rescaled in TMEM), final O/l and LSE.
+// TMEM columns: S_0 [0,128)  S_1 [128,256)  O_0 [256,384)  O_1 [384,512);
+// P_t (bf16 pairs) overwrites the first 64 columns of S_t.
+#pragma once
+#include "sm100.cuh"
+
+namespace pa {
+
+constexpr int kMaxHeads = 128;
+
+struct AttnParams {
+    int B, N, H, Hkv, G, nb;
+    int num_units;             // head units per (b, qb)
+    const int32_t *rank;       // [B][G][T]
+    const int32_t *cnt;        // [B][H][nb]
+    float scale_log2;          // softmax_scale * log2(e)
+    __nv_bfloat16 *o;
+    int64_t osb, oss, osh;
+    float *lse;                // [B][H][N] or nullptr
+    uint64_t timeout_ns;
+    int16_t unit_h0[kMaxHeads];
+    int16_t unit_h1[kMaxHeads];  // -1: the unit has one head
+};
+
+template <int D>
+struct AttnSmem {
+    static constexpr int TB = 128 * D * 2;
+    static constexpr int KS = (D == 128) ? 2 : 4;
+    static constexpr int BYTES = (2 + 2 * KS) * TB + 1024 + 512;
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+    using SM = AttnSmem<D>;
+    constexpr int TB = SM::TB;
+    constexpr int KS = SM::KS;
+    constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false, false);
+    constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = smem;                      // [2][TB]
+    uint8_t *sK = smem + 2 * TB;             // [KS][TB]
+    uint8_t *sV = smem + (2 + KS) * TB;      // [KS][TB]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (2 + 2 * KS) * TB);
+    uint64_t *q_full = bars;                 // 1
+    uint64_t *s_full = bars + 1;             // 2
+    uint64_t *p_full = bars + 3;             // 2
+    uint64_t *o_done = bars + 5;             // 2
+    uint64_t *drain = bars + 7;              // 1
+    uint64_t *k_full = bars + 8;             // KS
+    uint64_t *k_empty = bars + 8 + KS;       // KS
+    uint64_t *v_full = bars + 8 + 2 * KS;    // KS
+    uint64_t *v_empty = bars + 8 + 3 * KS;   // KS
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8 + 4 * KS);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    // ------------------------------------------------------------ work item
+    const int P = p.num_units;
+    const int unit = static_cast<int>(blockIdx.x % P);
+    const int bq = static_cast<int>(blockIdx.x / P);
+    const int b = bq % p.B;
+    const int qb = p.nb - 1 - bq / p.B;  // heaviest query blocks first
+    const int h0 = p.unit_h0[unit];
+    const int h1 = p.unit_h1[unit];
+    const int g = static_cast<int>(static_cast<long long>(h0) * p.G / p.H);
+    const int kvh = static_cast<int>(static_cast<long long>(h0) * p.Hkv / p.H);
+    const long long T = static_cast<long long>(p.nb) * (p.nb + 1) / 2;
+    const int32_t *list = p.rank + (static_cast<long long>(b) * p.G + g) * T +
+                          static_cast<long long>(qb) * (qb + 1) / 2;
+    int craw[2];
+    craw[0] = p.cnt[(static_cast<long long>(b) * p.H + h0) * p.nb + qb];
+    craw[1] = (h1 >= 0) ? p.cnt[(static_cast<long long>(b) * p.H + h1) * p.nb + qb] : 0;
+    int c[2];
+    for (int t = 0; t < 2; ++t) c[t] = min(max(craw[t], 0), qb + 1);
+    const int n = max(c[0], c[1]);
+    const int ntiles = (h1 >= 0) ? 2 : 1;
+
+    const uint32_t warp = warp_id(), lane = lane_id();
+    if (threadIdx.x == 0) {
+        if (c[0] != craw[0] || (h1 >= 0 && c[1] != craw[1])) flag_status(kStBounds);
+        mbar_init(q_full, 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&s_full[t], 1);
+            mbar_init(&p_full[t], 128);
+            mbar_init(&o_done[t], 1);
+        }
+        mbar_init(drain, 1);
+        for (int s = 0; s < KS; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const WaitCtl wc{abort_flag, p.timeout_ns};
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            mbar_arrive_expect_tx(q_full, ntiles * TB);
+#pragma unroll
+            for (int cc = 0; cc < D / 64; ++cc) {
+                tma_load_4d(sQ + cc * 16384, &tmQ, q_full, cc * 64, h0, qb * 128, b);
+                if (h1 >= 0) tma_load_4d(sQ + TB + cc * 16384, &tmQ, q_full, cc * 64, h1, qb * 128, b);
+            }
+            int issued = 0;
+            for (int i = 0; i < n; ++i) {
+                int kb = list[i];
+                if (kb < 0 || kb > qb) {
+                    flag_status(kStBounds);
+                    kb = qb;  // the softmax masks this tile out entirely
+                }
+                const int s = i % KS;
+                const uint32_t ph = ((i / KS) - 1) & 1;
+                if (i >= KS && !mbar_wait(&k_empty[s], ph, wc)) break;
+                mbar_arrive_expect_tx(&k_full[s], TB);
+#pragma unroll
+                for (int cc = 0; cc < D / 64; ++cc)
+                    tma_load_4d(sK + s * TB + cc * 16384, &tmK, &k_full[s], cc * 64, kvh, kb * 128, b);
+                if (i >= KS && !mbar_wait(&v_empty[s], ph, wc)) {
+                    issued = -(i + 1);  // K of tile i issued, V not
+                    break;
+                }
+                mbar_arrive_expect_tx(&v_full[s], TB);
+#pragma unroll
+                for (int cc = 0; cc < D / 64; ++cc)
+                    tma_load_4d(sV + s * TB + cc * 16384, &tmV, &v_full[s], cc * 64, kvh, kb * 128, b);
+                issued = i + 1;
+            }
+            // teardown: let every copy in flight land before the CTA exits
+            mbar_wait_drain(q_full, 0, p.timeout_ns);
+            const int nk = issued >= 0 ? issued : -issued;
+            const int nv = issued >= 0 ? issued : -issued - 1;
+            for (int i = max(nk - KS, 0); i < nk; ++i) mbar_wait_drain(&k_full[i % KS], (i / KS) & 1, p.timeout_ns);
+            for (int i = max(nv - KS, 0); i < nv; ++i) mbar_wait_drain(&v_full[i % KS], (i / KS) & 1, p.timeout_ns);
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0 && n > 0) {
+            const uint32_t qa[2] = {smem_u32(sQ), smem_u32(sQ + TB)};
+            auto issue_qk = [&](int t, int s) {
+                const uint32_t kbase = smem_u32(sK + s * TB);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    umma_ss(tmem + t * 128, sdesc_sw128(qa[t] + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024),
+                            IDESC_QK, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&s_full[t]);
+            };
+            auto issue_pv = [&](int t, int s, bool accumulate) {
+                const uint32_t vbase = smem_u32(sV + s * TB);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)  // 128 keys, 16 per step
+                    umma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, sdesc_sw128(vbase + kk * 2048, 16384, 1024),
+                            IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
+                umma_commit(&o_done[t]);
+            };
+            bool ok = mbar_wait(q_full, 0, wc) && mbar_wait(&k_full[0], 0, wc);
+            if (ok) {
+                tc_fence_after();
+                for (int t = 0; t < 2; ++t)
+                    if (c[t] > 0) issue_qk(t, 0);
+                umma_commit(&k_empty[0]);
+            }
+            for (int i = 0; i < n && ok; ++i) {
+                const int s = i % KS;
+                const int s1 = (i + 1) % KS;
+                const bool has_next = i + 1 < n;
+                if (!mbar_wait(&v_full[s], (i / KS) & 1, wc)) break;
+                if (has_next && !mbar_wait(&k_full[s1], ((i + 1) / KS) & 1, wc)) break;
+                tc_fence_after();
+                for (int t = 0; t < 2; ++t) {
+                    if (i < c[t]) {
+                        if (!mbar_wait(&p_full[t], i & 1, wc)) { ok = false; break; }
+                        tc_fence_after();
+                        issue_pv(t, s, i > 0);
+                    }
+                    if (i + 1 < c[t]) issue_qk(t, s1);
+                }
+                if (!ok) break;
+                umma_commit(&v_empty[s]);
+                if (has_next) umma_commit(&k_empty[s1]);
+            }
+        }
+        if (lane == 0) {
+            umma_commit(drain);
+            mbar_wait_drain(drain, 0, p.timeout_ns);
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------- softmax
+        const int t = (warp >= 6) ? 1 : 0;
+        const int ct = c[t];
+        const int h = t ? h1 : h0;
+        const int q4 = static_cast<int>(warp & 3);
+        const int row = q4 * 32 + static_cast<int>(lane);
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+        const uint32_t s_addr = lane_base + t * 128;
+        const uint32_t o_addr = lane_base + 256 + t * 128;
+        float m = -INFINITY, l = 0.0f;
+        bool ok = true;
+        uint32_t r[32];
+        for (int i = 0; i < ct; ++i) {
+            if (!warp_wait(&s_full[t], i & 1, wc)) { ok = false; break; }
+            tc_fence_after();
+            const int kb = list[i];
+            const bool valid = (kb >= 0 && kb <= qb);
+            const bool diag = (kb == qb);
+            // pass 1: row max of this tile
+            float mt = -INFINITY;
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                tmem_ld32(s_addr + ch * 32, r);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (valid && (!diag || ch * 32 + j <= row)) mt = fmaxf(mt, __uint_as_float(r[j]));
+            }
+            mt *= p.scale_log2;
+            const float m_new = fmaxf(m, mt);
+            if (i > 0) {
+                const bool need = m_new > m + 8.0f;
+                if (__any_sync(0xffffffffu, need)) {
+                    const float alpha = (m == -INFINITY) ? 0.0f : ex2(m - m_new);
+                    if (!warp_wait(&o_done[t], (i - 1) & 1, wc)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int ch = 0; ch < D / 32; ++ch) {
+                        tmem_ld32(o_addr + ch * 32, r);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
+                        tmem_st32(o_addr + ch * 32, r);
+                    }
+                    tmem_st_wait();
+                    l *= alpha;
+                    m = m_new;
+                }
+            } else {
+                m = m_new;
+            }
+            const float mref = (m == -INFINITY) ? 0.0f : m;
+            // pass 2: P = exp2(x - m) as bf16 pairs over the S columns, row sum
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                tmem_ld32(s_addr + ch * 32, r);
+                uint32_t pk[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int c0 = ch * 32 + 2 * j;
+                    const bool ok0 = valid && (!diag || c0 <= row);
+                    const bool ok1 = valid && (!diag || c0 + 1 <= row);
+                    const float e0 = ok0 ? ex2(fmaf(__uint_as_float(r[2 * j]), p.scale_log2, -mref)) : 0.0f;
+                    const float e1 = ok1 ? ex2(fmaf(__uint_as_float(r[2 * j + 1]), p.scale_log2, -mref)) : 0.0f;
+                    l += e0 + e1;
+                    pk[j] = pack_bf16x2(e0, e1);
+                }
+                tmem_st16(s_addr + ch * 16, pk);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&p_full[t]);
+        }
+        // epilogue: O / l -> bf16 -> global; LSE
+        if (ct > 0 && ok && warp_wait(&o_done[t], (ct - 1) & 1, wc)) {
+            tc_fence_after();
+            const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
+            __nv_bfloat16 *orow = p.o + b * p.osb + static_cast<int64_t>(qb * 128 + row) * p.oss + h * p.osh;
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ++ch) {
+                tmem_ld32(o_addr + ch * 32, r);
+                uint32_t w[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    w[j] = pack_bf16x2(__uint_as_float(r[2 * j]) * inv, __uint_as_float(r[2 * j + 1]) * inv);
+                uint4 *dst = reinterpret_cast<uint4 *>(orow + ch * 32);
+                dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                dst[2] = make_uint4(w[8], w[9], w[10], w[11]);
+                dst[3] = make_uint4(w[12], w[13], w[14], w[15]);
+            }
+            if (p.lse)
+                p.lse[(static_cast<long long>(b) * p.H + h) * p.N + qb * 128 + row] =
+                    (m + log2f(l)) * 0.69314718055994531f;
+        }
+    }
+
+    // -------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace pa

@@ -1,0 +1,229 @@
+// mask.cuh -- from block scores and last-block partial softmax statistics to
+// the block-sparse mask (ProxyAttn blog, "4. ProxyAttn method": Step 1 "Block
+// Ranking" and Step 2 "dynamic budget"; the threshold rule is XAttention's
+// find_blocks, XAttention blog 2.2).
+//
+//   mass_combine_kernel  exact softmax normalisation across all KV blocks of
+//                        each last-block row, then mass[kb] = mean over rows
+//   rank_kernel          per (b, g, qb): [0, qb, then blocks 1..qb-1 by
+//                        (score desc, index asc)] via a bitonic sort of
+//                        64-bit keys in shared memory
+//   budget_kernel        per (b, h): fixed-point prefix scan of the head's
+//                        masses along the last row's list -> k_h, then the
+//                        per-row counts
+#pragma once
+#include "sm100.cuh"
+
+namespace pa {
+
+// ------------------------------------------------------------ mass combine
+// partial: [B*H][nb][128] (m, l) with m the log2-domain row max of a tile and
+// l the sum of exp2(x - m) over its valid entries.
+__global__ void __launch_bounds__(256) mass_combine_kernel(const float2 *__restrict__ partial,
+                                                           float *__restrict__ mass, int nb) {
+    __shared__ float sM[2][128], sL[2][128];
+    const long long bh = blockIdx.x;
+    const float2 *part = partial + bh * nb * 128;
+    const int tid = threadIdx.x;
+    const int r = tid & 127, half = tid >> 7;
+    float M = -INFINITY, L = 0.0f;
+    for (int kb = half; kb < nb; kb += 2) {
+        const float2 v = part[static_cast<long long>(kb) * 128 + r];
+        if (v.x > M) {
+            L = L * exp2f(M - v.x) + v.y;
+            M = v.x;
+        } else {
+            L += v.y * exp2f(v.x - M);
+        }
+    }
+    sM[half][r] = M;
+    sL[half][r] = L;
+    __syncthreads();
+    if (tid < 128) {
+        const float M0 = sM[0][r], M1 = sM[1][r];
+        const float Mx = fmaxf(M0, M1);
+        const float Lx = (M0 == -INFINITY ? 0.0f : sL[0][r] * exp2f(M0 - Mx)) +
+                         (M1 == -INFINITY ? 0.0f : sL[1][r] * exp2f(M1 - Mx));
+        sM[0][r] = Mx;
+        sL[0][r] = 1.0f / Lx;
+    }
+    __syncthreads();
+    const int warp = tid >> 5, lane = tid & 31;
+    float Mr[4], Ir[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        Mr[j] = sM[0][lane + 32 * j];
+        Ir[j] = sL[0][lane + 32 * j];
+    }
+    for (int kb = warp; kb < nb; kb += 8) {
+        float s = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 v = part[static_cast<long long>(kb) * 128 + lane + 32 * j];
+            s += v.y * exp2f(v.x - Mr[j]) * Ir[j];
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) mass[bh * nb + kb] = s * (1.0f / 128.0f);
+    }
+}
+
+// ------------------------------------------------------------------- rank
+__device__ __forceinline__ uint32_t score_desc_key(float f) {
+    const uint32_t u = __float_as_uint(f + 0.0f);  // -0 and +0 compare equal
+    const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return ~ord;  // larger score -> smaller key
+}
+
+// One CTA per (b, g, qb); dynamic smem holds P = pow2 >= qb-1 keys.
+__global__ void __launch_bounds__(256) rank_kernel(const float *__restrict__ scores, int32_t *__restrict__ rank,
+                                                   int nb) {
+    extern __shared__ unsigned long long keys[];
+    const long long bg = blockIdx.x / nb;
+    const int qb = nb - 1 - static_cast<int>(blockIdx.x % nb);  // long rows first
+    const long long T = static_cast<long long>(nb) * (nb + 1) / 2;
+    const long long row0 = bg * T + static_cast<long long>(qb) * (qb + 1) / 2;
+    const float *srow = scores + row0;
+    int32_t *out = rank + row0;
+    const int n = qb >= 2 ? qb - 1 : 0;
+    int P = 1;
+    while (P < n) P <<= 1;
+    for (int i = threadIdx.x; i < P; i += blockDim.x) {
+        unsigned long long key = ~0ull;
+        if (i < n) {
+            float s = srow[i + 1];
+            if (!isfinite(s)) {
+                flag_status(kStNonFinite);
+                s = -INFINITY;
+            }
+            key = (static_cast<unsigned long long>(score_desc_key(s)) << 32) | static_cast<uint32_t>(i + 1);
+        }
+        keys[i] = key;
+    }
+    __syncthreads();
+    for (int k = 2; k <= P; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = threadIdx.x; i < P; i += blockDim.x) {
+                const int ixj = i ^ j;
+                if (ixj > i) {
+                    const unsigned long long a = keys[i], c = keys[ixj];
+                    const bool up = (i & k) == 0;
+                    if ((a > c) == up) {
+                        keys[i] = c;
+                        keys[ixj] = a;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    if (threadIdx.x == 0) {
+        out[0] = 0;
+        if (qb > 0) out[1] = qb;
+    }
+    for (int i = threadIdx.x; i < n; i += blockDim.x) out[2 + i] = static_cast<int32_t>(keys[i] & 0xFFFFFFFFu);
+}
+
+// ----------------------------------------------------------------- budget
+struct BudgetParams {
+    int B, H, G, nb;
+    int mode;            // 0 dynamic, 1 fixed fraction, 2 all
+    float gamma;
+    int frac_permille;
+    const int32_t *rank;
+    const float *mass;   // [B][H][nb]
+    int32_t *cnt;        // [B][H][nb]
+    int32_t *budget;     // [B][H]
+};
+
+__device__ __forceinline__ int forced_blocks(int qb) { return qb == 0 ? 1 : 2; }
+
+// One CTA of 1024 threads per (b, h); nb <= 4096 -> at most 4 list entries per thread.
+__global__ void __launch_bounds__(1024) budget_kernel(BudgetParams p) {
+    __shared__ long long warp_sums[32];
+    __shared__ int kmin;
+    const int bh = blockIdx.x;
+    const int b = bh / p.H, h = bh % p.H;
+    const int nb = p.nb;
+    int k = nb;
+    if (p.mode == 0) {
+        const int g = static_cast<int>(static_cast<long long>(h) * p.G / p.H);
+        const long long T = static_cast<long long>(nb) * (nb + 1) / 2;
+        const int32_t *last = p.rank + (static_cast<long long>(b) * p.G + g) * T +
+                              static_cast<long long>(nb - 1) * nb / 2;
+        const float *m = p.mass + static_cast<long long>(bh) * nb;
+        const long long gfx = __double2ll_rn(static_cast<double>(p.gamma) * 1099511627776.0);
+        const int F = forced_blocks(nb - 1);
+        const int per = (nb + blockDim.x - 1) / blockDim.x;
+        const int t0 = threadIdx.x * per;
+        long long v[4];
+        long long local = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v[j] = 0;
+            const int t = t0 + j;
+            if (j < per && t < nb) {
+                int kb = last[t];
+                if (kb < 0 || kb >= nb) {
+                    flag_status(kStBounds);
+                    kb = 0;
+                }
+                const float mk = m[kb];
+                if (!isfinite(mk)) flag_status(kStNonFinite);
+                v[j] = __float2ll_rn(mk * 1099511627776.0f);  // exact scaling by 2^40
+                local += v[j];
+            }
+        }
+        // block-wide exclusive scan of the per-thread sums
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+        long long incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) warp_sums[warp] = incl;
+        if (threadIdx.x == 0) kmin = nb;
+        __syncthreads();
+        if (warp == 0) {
+            long long ws = (lane < static_cast<int>(blockDim.x >> 5)) ? warp_sums[lane] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const long long y = __shfl_up_sync(0xffffffffu, ws, o);
+                if (lane >= o) ws += y;
+            }
+            warp_sums[lane] = ws;  // inclusive over warps
+        }
+        __syncthreads();
+        long long run = (incl - local) + (warp > 0 ? warp_sums[warp - 1] : 0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int t = t0 + j;
+            if (j < per && t < nb) {
+                run += v[j];
+                if (t + 1 >= F && run >= gfx) {
+                    atomicMin(&kmin, t + 1);
+                    break;
+                }
+            }
+        }
+        __syncthreads();
+        k = kmin;
+    }
+    int32_t *c = p.cnt + static_cast<long long>(bh) * nb;
+    for (int qb = threadIdx.x; qb < nb; qb += blockDim.x) {
+        long long want;
+        if (p.mode == 0)
+            want = (static_cast<long long>(k) * (qb + 1) + nb - 1) / nb;
+        else if (p.mode == 1)
+            want = (static_cast<long long>(p.frac_permille) * (qb + 1) + 999) / 1000;
+        else
+            want = qb + 1;
+        const long long lo = forced_blocks(qb), hi = qb + 1;
+        const int val = static_cast<int>(want < lo ? lo : (want > hi ? hi : want));
+        c[qb] = val;
+        if (qb == nb - 1) p.budget[bh] = val;
+    }
+}
+
+}  // namespace pa

@@ -1,0 +1,488 @@
+// pa_api.cu -- the C ABI of libpa.so (declared in include/pa.h): argument
+// validation, TMA descriptor construction, workspace carving and kernel
+// launches.  Every step of the method runs in the kernels of this library;
+// the host code only checks arguments and launches.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "pa.h"
+#include "attn.cuh"
+#include "mask.cuh"
+#include "pool.cuh"
+#include "tile_gemm.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+pa_status fail(pa_status s, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+pa_status ok() {
+    g_last_error.clear();
+    return PA_OK;
+}
+
+#define PA_CUDA(call)                                                                       \
+    do {                                                                                    \
+        cudaError_t e_ = (call);                                                            \
+        if (e_ != cudaSuccess) return fail(PA_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+    } while (0)
+
+constexpr int kBlk = 128;
+constexpr int kMaxNb = 4096;
+constexpr int kScoreChunk = 16;  // tiles per score/mass work unit
+
+uint64_t wait_timeout_ns() {
+    static uint64_t v = [] {
+        const char *e = getenv("PA_WAIT_TIMEOUT_MS");
+        double ms = e ? atof(e) : 2000.0;
+        if (!(ms > 0.0)) ms = 2000.0;
+        return static_cast<uint64_t>(ms * 1e6);
+    }();
+    return v;
+}
+
+// ------------------------------------------------------------- validation
+pa_status check_shape(const pa_shape *s) {
+    if (!s) return fail(PA_ERR_INVALID_ARG, "shape is NULL");
+    if (s->batch < 1 || s->seqlen < 1 || s->num_q_heads < 1 || s->num_kv_heads < 1 || s->num_groups < 1)
+        return fail(PA_ERR_INVALID_ARG, "shape fields must be positive");
+    if (s->block != kBlk) return fail(PA_ERR_UNSUPPORTED, "block must be 128 (got %d)", s->block);
+    if (s->head_dim != 64 && s->head_dim != 128)
+        return fail(PA_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", s->head_dim);
+    if (s->seqlen % kBlk) return fail(PA_ERR_UNSUPPORTED, "seqlen %d is not a multiple of 128", s->seqlen);
+    if (s->seqlen / kBlk > kMaxNb) return fail(PA_ERR_UNSUPPORTED, "seqlen %d exceeds %d", s->seqlen, kMaxNb * kBlk);
+    if (s->num_q_heads > pa::kMaxHeads) return fail(PA_ERR_UNSUPPORTED, "more than %d q heads", pa::kMaxHeads);
+    if (s->num_q_heads % s->num_kv_heads)
+        return fail(PA_ERR_UNSUPPORTED, "num_q_heads %d not a multiple of num_kv_heads %d", s->num_q_heads,
+                    s->num_kv_heads);
+    if (s->num_q_heads % s->num_groups)
+        return fail(PA_ERR_UNSUPPORTED, "num_q_heads %d not a multiple of num_groups %d", s->num_q_heads,
+                    s->num_groups);
+    return PA_OK;
+}
+
+pa_status check_budget(const pa_budget *bu) {
+    if (!bu) return fail(PA_ERR_INVALID_ARG, "budget is NULL");
+    if (bu->mode == PA_BUDGET_DYNAMIC) {
+        if (!(bu->gamma > 0.0f && bu->gamma <= 1.0f))
+            return fail(PA_ERR_INVALID_ARG, "gamma must be in (0, 1] (got %g)", static_cast<double>(bu->gamma));
+    } else if (bu->mode == PA_BUDGET_FIXED_FRACTION) {
+        if (bu->frac_permille < 1 || bu->frac_permille > 1000)
+            return fail(PA_ERR_INVALID_ARG, "frac_permille must be in 1..1000 (got %d)", bu->frac_permille);
+    } else if (bu->mode != PA_BUDGET_ALL) {
+        return fail(PA_ERR_INVALID_ARG, "unknown budget mode %d", bu->mode);
+    }
+    return PA_OK;
+}
+
+pa_status check_ptr(const void *p, const char *name, size_t align = 16) {
+    if (!p) return fail(PA_ERR_INVALID_ARG, "%s is NULL", name);
+    if (reinterpret_cast<uintptr_t>(p) % align)
+        return fail(PA_ERR_INVALID_ARG, "%s is not %zu-byte aligned", name, align);
+    return PA_OK;
+}
+
+pa_status check_tensor(const void *p, pa_strides st, const char *name) {
+    pa_status s = check_ptr(p, name);
+    if (s) return s;
+    if (st.b < 0 || st.s <= 0 || st.h <= 0 || st.b % 8 || st.s % 8 || st.h % 8)
+        return fail(PA_ERR_INVALID_ARG, "%s strides (%lld, %lld, %lld) must be positive multiples of 8 elements", name,
+                    static_cast<long long>(st.b), static_cast<long long>(st.s), static_cast<long long>(st.h));
+    return PA_OK;
+}
+
+// ------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// A bf16 tensor of 4 dims (innermost first) with byte strides of dims 1..3,
+// box 64 x b1 x b2 x 1, 128-byte swizzle.
+pa_status make_map(CUtensorMap *m, const void *base, const cuuint64_t dims[4], const cuuint64_t strides[3],
+                   cuuint32_t box1, cuuint32_t box2, const char *name) {
+    auto fn = encode_fn();
+    if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    const cuuint32_t box[4] = {64, box1, box2, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed: %d", name, static_cast<int>(r));
+    return PA_OK;
+}
+
+// [B][N][heads][d] with element strides -> dims (d, heads, N, B), box 64x1x128x1
+pa_status map_bnhd(CUtensorMap *m, const void *base, int B, int N, int heads, int d, pa_strides st,
+                   const char *name) {
+    const int64_t sb = (B == 1) ? st.s * N : st.b;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
+                                static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(st.h) * 2, static_cast<cuuint64_t>(st.s) * 2,
+                                   static_cast<cuuint64_t>(sb) * 2};
+    return make_map(m, base, dims, strides, 1, 128, name);
+}
+
+// contiguous [B][G][N][d] proxies -> dims (d, N, G, B), box 64x128x1x1
+pa_status map_proxy(CUtensorMap *m, const void *base, int B, int G, int N, int d, const char *name) {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                                static_cast<cuuint64_t>(G), static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2,
+                                   static_cast<cuuint64_t>(G) * N * d * 2};
+    return make_map(m, base, dims, strides, 128, 1, name);
+}
+
+int num_sms() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+// ------------------------------------------------------------- workspace
+struct WsLayout {
+    size_t qp, kp, scores, partial, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+WsLayout ws_layout(const pa_shape *s, const pa_budget *bu) {
+    const size_t B = s->batch, G = s->num_groups, N = s->seqlen, d = s->head_dim, H = s->num_q_heads;
+    const size_t nb = N / kBlk, T = nb * (nb + 1) / 2;
+    WsLayout w;
+    w.partial = 0;
+    const size_t part = (bu && bu->mode == PA_BUDGET_DYNAMIC) ? align256(B * H * nb * 128 * sizeof(float2)) : 0;
+    w.qp = part;
+    w.kp = w.qp + align256(B * G * N * d * 2);
+    w.scores = w.kp + align256(B * G * N * d * 2);
+    w.total = w.scores + align256(B * G * T * sizeof(float));
+    return w;
+}
+
+size_t mask_ws_bytes(const pa_shape *s, const pa_budget *bu) {
+    return ws_layout(s, bu).qp;  // the partial-softmax statistics come first
+}
+
+// ------------------------------------------------------------- launches
+pa_status launch_pool(const pa_shape *s, const void *q, pa_strides qs, const void *k, pa_strides ks, void *qp,
+                      void *kp, cudaStream_t st) {
+    pa::PoolParams p;
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.k = static_cast<const __nv_bfloat16 *>(k);
+    p.qp = static_cast<__nv_bfloat16 *>(qp);
+    p.kp = static_cast<__nv_bfloat16 *>(kp);
+    p.qsb = qs.b; p.qss = qs.s; p.qsh = qs.h;
+    p.ksb = ks.b; p.kss = ks.s; p.ksh = ks.h;
+    p.B = s->batch; p.N = s->seqlen; p.H = s->num_q_heads; p.Hkv = s->num_kv_heads;
+    p.G = s->num_groups; p.d = s->head_dim;
+    const long long threads = static_cast<long long>(p.B) * p.N * p.G * (p.d / 8);
+    const unsigned grid = static_cast<unsigned>((threads + 255) / 256);
+    if (p.d == 128) pa::pool_heads_kernel<128><<<grid, 256, 0, st>>>(p);
+    else pa::pool_heads_kernel<64><<<grid, 256, 0, st>>>(p);
+    PA_CUDA(cudaGetLastError());
+    return PA_OK;
+}
+
+template <int D, int MODE>
+pa_status launch_tile_gemm_t(const CUtensorMap &a, const CUtensorMap &b, const pa::TileParams &p, cudaStream_t st) {
+    auto kern = pa::tile_gemm_kernel<D, MODE>;
+    const int smem = pa::TileSmem<D>::BYTES;
+    PA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    const long long grid = std::min<long long>(p.num_units, num_sms());
+    if (grid <= 0) return PA_OK;
+    kern<<<static_cast<unsigned>(grid), 192, smem, st>>>(a, b, p);
+    PA_CUDA(cudaGetLastError());
+    return PA_OK;
+}
+
+pa_status launch_scores(const pa_shape *s, const void *qp, const void *kp, float *scores, cudaStream_t st) {
+    const int B = s->batch, G = s->num_groups, N = s->seqlen, d = s->head_dim, nb = N / kBlk;
+    CUtensorMap ma, mb;
+    pa_status r = map_proxy(&ma, qp, B, G, N, d, "q_proxy");
+    if (r) return r;
+    if ((r = map_proxy(&mb, kp, B, G, N, d, "k_proxy"))) return r;
+    pa::TileParams p{};
+    p.B = B; p.nb = nb; p.NH = G; p.H = s->num_q_heads; p.Hkv = s->num_kv_heads;
+    p.chunk = kScoreChunk;
+    long long per = 0;
+    for (int qb = 0; qb < nb; ++qb) per += (qb + kScoreChunk) / kScoreChunk;
+    p.units_per_bh = per;
+    p.num_units = per * B * G;
+    p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+    p.scores = scores;
+    p.partial = nullptr;
+    p.timeout_ns = wait_timeout_ns();
+    return d == 128 ? launch_tile_gemm_t<128, pa::MODE_SCORES>(ma, mb, p, st)
+                    : launch_tile_gemm_t<64, pa::MODE_SCORES>(ma, mb, p, st);
+}
+
+pa_status launch_mass(const pa_shape *s, const void *q, pa_strides qs, const void *k, pa_strides ks, float2 *partial,
+                      float *mass, cudaStream_t st) {
+    const int B = s->batch, H = s->num_q_heads, Hkv = s->num_kv_heads, N = s->seqlen, d = s->head_dim;
+    const int nb = N / kBlk;
+    CUtensorMap ma, mb;
+    pa_status r = map_bnhd(&ma, q, B, N, H, d, qs, "q");
+    if (r) return r;
+    if ((r = map_bnhd(&mb, k, B, N, Hkv, d, ks, "k"))) return r;
+    pa::TileParams p{};
+    p.B = B; p.nb = nb; p.NH = H; p.H = H; p.Hkv = Hkv;
+    p.chunk = kScoreChunk;
+    p.units_per_bh = (nb + kScoreChunk - 1) / kScoreChunk;
+    p.num_units = p.units_per_bh * B * H;
+    p.scale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
+    p.scores = nullptr;
+    p.partial = partial;
+    p.timeout_ns = wait_timeout_ns();
+    r = d == 128 ? launch_tile_gemm_t<128, pa::MODE_MASS>(ma, mb, p, st)
+                 : launch_tile_gemm_t<64, pa::MODE_MASS>(ma, mb, p, st);
+    if (r) return r;
+    pa::mass_combine_kernel<<<B * H, 256, 0, st>>>(partial, mass, nb);
+    PA_CUDA(cudaGetLastError());
+    return PA_OK;
+}
+
+pa_status launch_rank(const pa_shape *s, const float *scores, int32_t *rank, cudaStream_t st) {
+    const int nb = s->seqlen / kBlk;
+    int P = 1;
+    while (P < nb - 1) P <<= 1;
+    const int smem = P * 8;
+    PA_CUDA(cudaFuncSetAttribute(pa::rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, std::max(smem, 1)));
+    const long long grid = static_cast<long long>(s->batch) * s->num_groups * nb;
+    pa::rank_kernel<<<static_cast<unsigned>(grid), 256, smem, st>>>(scores, rank, nb);
+    PA_CUDA(cudaGetLastError());
+    return PA_OK;
+}
+
+pa_status launch_budget(const pa_shape *s, const pa_budget *bu, const int32_t *rank, const float *mass, int32_t *cnt,
+                        int32_t *budget, cudaStream_t st) {
+    pa::BudgetParams p;
+    p.B = s->batch; p.H = s->num_q_heads; p.G = s->num_groups; p.nb = s->seqlen / kBlk;
+    p.mode = bu->mode; p.gamma = bu->gamma; p.frac_permille = bu->frac_permille;
+    p.rank = rank; p.mass = mass; p.cnt = cnt; p.budget = budget;
+    pa::budget_kernel<<<s->batch * s->num_q_heads, 1024, 0, st>>>(p);
+    PA_CUDA(cudaGetLastError());
+    return PA_OK;
+}
+
+// Head units of the attention kernel: pairs of consecutive q heads that share
+// both their KV head and their proxy group (so they share one ranked list and
+// one K/V stream); a head left over forms a unit alone.
+int build_units(const pa_shape *s, int16_t *h0, int16_t *h1) {
+    const int H = s->num_q_heads, Hkv = s->num_kv_heads, G = s->num_groups;
+    int n = 0;
+    int h = 0;
+    while (h < H) {
+        const int kv = static_cast<int>(static_cast<long long>(h) * Hkv / H);
+        const int g = static_cast<int>(static_cast<long long>(h) * G / H);
+        const bool pair = h + 1 < H && static_cast<int>(static_cast<long long>(h + 1) * Hkv / H) == kv &&
+                          static_cast<int>(static_cast<long long>(h + 1) * G / H) == g;
+        h0[n] = static_cast<int16_t>(h);
+        h1[n] = static_cast<int16_t>(pair ? h + 1 : -1);
+        ++n;
+        h += pair ? 2 : 1;
+    }
+    return n;
+}
+
+template <int D>
+pa_status launch_attn_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const pa::AttnParams &p,
+                        cudaStream_t st) {
+    auto kern = pa::attn_kernel<D>;
+    const int smem = pa::AttnSmem<D>::BYTES;
+    PA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    const long long grid = static_cast<long long>(p.num_units) * p.B * p.nb;
+    kern<<<static_cast<unsigned>(grid), 320, smem, st>>>(mq, mk, mv, p);
+    PA_CUDA(cudaGetLastError());
+    return PA_OK;
+}
+
+pa_status launch_attn(const pa_shape *s, const void *q, pa_strides qs, const void *k, pa_strides ks, const void *v,
+                      pa_strides vs, const int32_t *rank, const int32_t *cnt, float scale, void *o, pa_strides os,
+                      float *lse, cudaStream_t st) {
+    const int B = s->batch, H = s->num_q_heads, Hkv = s->num_kv_heads, N = s->seqlen, d = s->head_dim;
+    CUtensorMap mq, mk, mv;
+    pa_status r = map_bnhd(&mq, q, B, N, H, d, qs, "q");
+    if (r) return r;
+    if ((r = map_bnhd(&mk, k, B, N, Hkv, d, ks, "k"))) return r;
+    if ((r = map_bnhd(&mv, v, B, N, Hkv, d, vs, "v"))) return r;
+    pa::AttnParams p{};
+    p.B = B; p.N = N; p.H = H; p.Hkv = Hkv; p.G = s->num_groups; p.nb = N / kBlk;
+    p.num_units = build_units(s, p.unit_h0, p.unit_h1);
+    p.rank = rank; p.cnt = cnt;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.o = static_cast<__nv_bfloat16 *>(o);
+    p.osb = os.b; p.oss = os.s; p.osh = os.h;
+    p.lse = lse;
+    p.timeout_ns = wait_timeout_ns();
+    return d == 128 ? launch_attn_t<128>(mq, mk, mv, p, st) : launch_attn_t<64>(mq, mk, mv, p, st);
+}
+
+pa_status check_mask(const pa_mask *m, const pa_budget *bu, bool need_rank_cnt) {
+    if (!m) return fail(PA_ERR_INVALID_ARG, "mask is NULL");
+    pa_status r;
+    if (need_rank_cnt) {
+        if ((r = check_ptr(m->rank, "mask.rank", 4))) return r;
+        if ((r = check_ptr(m->cnt, "mask.cnt", 4))) return r;
+    }
+    if ((r = check_ptr(m->budget, "mask.budget", 4))) return r;
+    if (bu->mode == PA_BUDGET_DYNAMIC && (r = check_ptr(m->mass, "mask.mass", 4))) return r;
+    return PA_OK;
+}
+
+}  // namespace
+
+// ===================================================================== C ABI
+extern "C" {
+
+int32_t pa_abi_version(void) { return PA_ABI_VERSION; }
+
+const char *pa_last_error(void) { return g_last_error.c_str(); }
+
+const char *pa_status_string(pa_status s) {
+    switch (s) {
+        case PA_OK: return "ok";
+        case PA_ERR_INVALID_ARG: return "invalid argument";
+        case PA_ERR_UNSUPPORTED: return "unsupported shape";
+        case PA_ERR_WORKSPACE: return "workspace too small";
+        case PA_ERR_CUDA: return "CUDA error";
+        case PA_ERR_TIMEOUT: return "device wait timed out";
+        case PA_ERR_DEVICE_BOUNDS: return "block index out of range on device";
+        case PA_ERR_DEVICE_NONFINITE: return "non-finite block score or mass on device";
+    }
+    return "unknown status";
+}
+
+size_t pa_workspace_size(const pa_shape *shape, const pa_budget *budget) {
+    if (check_shape(shape) || check_budget(budget)) return 0;
+    return ws_layout(shape, budget).total;
+}
+
+pa_status pa_pool_heads(const pa_shape *shape, const void *q, pa_strides qs, const void *k, pa_strides ks,
+                        void *q_proxy, void *k_proxy, pa_stream_t stream) {
+    pa_status r;
+    if ((r = check_shape(shape))) return r;
+    if ((r = check_tensor(q, qs, "q")) || (r = check_tensor(k, ks, "k"))) return r;
+    if ((r = check_ptr(q_proxy, "q_proxy")) || (r = check_ptr(k_proxy, "k_proxy"))) return r;
+    if ((r = launch_pool(shape, q, qs, k, ks, q_proxy, k_proxy, reinterpret_cast<cudaStream_t>(stream)))) return r;
+    return ok();
+}
+
+pa_status pa_block_scores(const pa_shape *shape, const void *q_proxy, const void *k_proxy, float *scores,
+                          pa_stream_t stream) {
+    pa_status r;
+    if ((r = check_shape(shape))) return r;
+    if ((r = check_ptr(q_proxy, "q_proxy")) || (r = check_ptr(k_proxy, "k_proxy"))) return r;
+    if ((r = check_ptr(scores, "scores", 4))) return r;
+    if ((r = launch_scores(shape, q_proxy, k_proxy, scores, reinterpret_cast<cudaStream_t>(stream)))) return r;
+    return ok();
+}
+
+pa_status pa_build_mask(const pa_shape *shape, const pa_budget *budget, const float *scores, const void *q,
+                        pa_strides qs, const void *k, pa_strides ks, const pa_mask *out, void *ws, size_t ws_bytes,
+                        pa_stream_t stream) {
+    pa_status r;
+    if ((r = check_shape(shape)) || (r = check_budget(budget))) return r;
+    if ((r = check_ptr(scores, "scores", 4))) return r;
+    if ((r = check_mask(out, budget, true))) return r;
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (budget->mode == PA_BUDGET_DYNAMIC) {
+        if ((r = check_tensor(q, qs, "q")) || (r = check_tensor(k, ks, "k"))) return r;
+        const size_t need = mask_ws_bytes(shape, budget);
+        if (!ws || ws_bytes < need)
+            return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, need);
+        if ((r = check_ptr(ws, "workspace", 256))) return r;
+        if ((r = launch_mass(shape, q, qs, k, ks, static_cast<float2 *>(ws), out->mass, st))) return r;
+    }
+    if ((r = launch_rank(shape, scores, out->rank, st))) return r;
+    if ((r = launch_budget(shape, budget, out->rank, out->mass, out->cnt, out->budget, st))) return r;
+    return ok();
+}
+
+pa_status pa_block_sparse_attn(const pa_shape *shape, const void *q, pa_strides qs, const void *k, pa_strides ks,
+                               const void *v, pa_strides vs, const int32_t *rank, const int32_t *cnt,
+                               float softmax_scale, void *o, pa_strides os, float *lse, pa_stream_t stream) {
+    pa_status r;
+    if ((r = check_shape(shape))) return r;
+    if ((r = check_tensor(q, qs, "q")) || (r = check_tensor(k, ks, "k")) || (r = check_tensor(v, vs, "v")) ||
+        (r = check_tensor(o, os, "o")))
+        return r;
+    if ((r = check_ptr(rank, "rank", 4)) || (r = check_ptr(cnt, "cnt", 4))) return r;
+    if (lse && (r = check_ptr(lse, "lse", 4))) return r;
+    if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale))
+        return fail(PA_ERR_INVALID_ARG, "softmax_scale must be positive and finite");
+    if ((r = launch_attn(shape, q, qs, k, ks, v, vs, rank, cnt, softmax_scale, o, os, lse,
+                         reinterpret_cast<cudaStream_t>(stream))))
+        return r;
+    return ok();
+}
+
+pa_status pa_prefill(const pa_shape *shape, const pa_budget *budget, const void *q, pa_strides qs, const void *k,
+                     pa_strides ks, const void *v, pa_strides vs, void *o, pa_strides os, const pa_mask *mask_out,
+                     void *ws, size_t ws_bytes, pa_stream_t stream) {
+    pa_status r;
+    if ((r = check_shape(shape)) || (r = check_budget(budget))) return r;
+    if ((r = check_tensor(q, qs, "q")) || (r = check_tensor(k, ks, "k")) || (r = check_tensor(v, vs, "v")) ||
+        (r = check_tensor(o, os, "o")))
+        return r;
+    if ((r = check_mask(mask_out, budget, true))) return r;
+    const WsLayout w = ws_layout(shape, budget);
+    if (!ws || ws_bytes < w.total)
+        return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, w.total);
+    if ((r = check_ptr(ws, "workspace", 256))) return r;
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    void *qp = base + w.qp;
+    void *kp = base + w.kp;
+    float *scores = reinterpret_cast<float *>(base + w.scores);
+    if ((r = launch_pool(shape, q, qs, k, ks, qp, kp, st))) return r;
+    if ((r = launch_scores(shape, qp, kp, scores, st))) return r;
+    if (budget->mode == PA_BUDGET_DYNAMIC &&
+        (r = launch_mass(shape, q, qs, k, ks, reinterpret_cast<float2 *>(base + w.partial), mask_out->mass, st)))
+        return r;
+    if ((r = launch_rank(shape, scores, mask_out->rank, st))) return r;
+    if ((r = launch_budget(shape, budget, mask_out->rank, mask_out->mass, mask_out->cnt, mask_out->budget, st)))
+        return r;
+    const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(shape->head_dim)));
+    if ((r = launch_attn(shape, q, qs, k, ks, v, vs, mask_out->rank, mask_out->cnt, scale, o, os, nullptr, st)))
+        return r;
+    return ok();
+}
+
+pa_status pa_get_device_status(pa_stream_t stream, int clear) {
+    PA_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+    unsigned v = 0;
+    PA_CUDA(cudaMemcpyFromSymbol(&v, pa::g_status, sizeof v));
+    if (clear) {
+        const unsigned zero = 0;
+        PA_CUDA(cudaMemcpyToSymbol(pa::g_status, &zero, sizeof zero));
+    }
+    g_last_error.clear();
+    return static_cast<pa_status>(v);
+}
+
+}  // extern "C"

@@ -1,0 +1,96 @@
+// pool.cuh -- head pooling (ProxyAttn blog, "4. ProxyAttn method", Step 1
+// "Head Pooling"): the proxy of group g is the mean of the group's q heads,
+// and of the KV heads those q heads read.
+//
+// HBM-bound: every byte of q and k is read once and the proxies are written
+// once.  One thread owns 8 consecutive head-dim elements (one 16-byte vector)
+// of one (batch, token, group); a warp therefore reads whole 128-byte lines of
+// each head row.  Sums run in fp64 over ascending heads and the quotient is
+// rounded once to bf16, so the result equals the exact-mean definition bit for
+// bit whenever the sum of the group's bf16 values is exact in fp64 (always,
+// unless the values span more than ~2^40 in magnitude).
+#pragma once
+#include "sm100.cuh"
+
+namespace pa {
+
+struct PoolParams {
+    const __nv_bfloat16 *q;
+    const __nv_bfloat16 *k;
+    __nv_bfloat16 *qp;
+    __nv_bfloat16 *kp;
+    int64_t qsb, qss, qsh, ksb, kss, ksh;
+    int B, N, H, Hkv, G, d;
+};
+
+__device__ __forceinline__ void add_bf16x8(double (&acc)[8], const uint4 &v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        acc[2 * i] += static_cast<double>(__uint_as_float(w[i] << 16));
+        acc[2 * i + 1] += static_cast<double>(__uint_as_float(w[i] & 0xFFFF0000u));
+    }
+}
+
+__device__ __forceinline__ uint4 mean_to_bf16x8(const double (&acc)[8], int n) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat16 lo = __double2bfloat16(acc[2 * i] / n);
+        const __nv_bfloat16 hi = __double2bfloat16(acc[2 * i + 1] / n);
+        w[i] = static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
+               (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) pool_heads_kernel(PoolParams p) {
+    constexpr int TPR = D / 8;  // threads per (token, group) row
+    const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t rows = static_cast<int64_t>(p.B) * p.N * p.G;
+    const int64_t row = gid / TPR;
+    if (row >= rows) return;
+    const int c = static_cast<int>(gid % TPR) * 8;
+    const int g = static_cast<int>(row % p.G);
+    const int64_t bi = row / p.G;  // b * N + i
+    const int i = static_cast<int>(bi % p.N);
+    const int b = static_cast<int>(bi / p.N);
+
+    const int hpg = p.H / p.G;
+    const int h0 = g * hpg;
+    const __nv_bfloat16 *qrow = p.q + b * p.qsb + i * p.qss + c;
+    const __nv_bfloat16 *krow = p.k + b * p.ksb + i * p.kss + c;
+
+    double aq[8], ak[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) aq[j] = ak[j] = 0.0;
+
+    int last_kv = -1;
+    uint4 kv_raw = make_uint4(0, 0, 0, 0);
+    for (int t0 = 0; t0 < hpg; t0 += 8) {
+        const int n = min(8, hpg - t0);
+        uint4 qv[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+            if (t < n) qv[t] = __ldg(reinterpret_cast<const uint4 *>(qrow + (h0 + t0 + t) * p.qsh));
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            if (t < n) {
+                const int h = h0 + t0 + t;
+                add_bf16x8(aq, qv[t]);
+                const int kvh = static_cast<int>(static_cast<int64_t>(h) * p.Hkv / p.H);
+                if (kvh != last_kv) {
+                    kv_raw = __ldg(reinterpret_cast<const uint4 *>(krow + kvh * p.ksh));
+                    last_kv = kvh;
+                }
+                add_bf16x8(ak, kv_raw);
+            }
+        }
+    }
+    const int64_t o = ((static_cast<int64_t>(b) * p.G + g) * p.N + i) * D + c;
+    *reinterpret_cast<uint4 *>(p.qp + o) = mean_to_bf16x8(aq, hpg);
+    *reinterpret_cast<uint4 *>(p.kp + o) = mean_to_bf16x8(ak, hpg);
+}
+
+}  // namespace pa

@@ -1,0 +1,303 @@
+// tile_gemm.cuh -- 128x128 QK^T tiles on the tcgen05 tensor core, reduced in
+// the epilogue so that no token-level score reaches memory.
+//
+//   MODE_SCORES  (ProxyAttn blog, "4. ProxyAttn method", Step 1 "Score
+//                Estimation": the QK product of the proxy heads fused with
+//                block-level max pooling).  For every causal tile (qb, kb<=qb)
+//                of every proxy group: score = max over the tile's valid
+//                entries of (q_p . k_p)/sqrt(d).
+//   MODE_MASS    (Step 2, budget from the last query block).  For every head,
+//                the last query block against every key block: per row, the
+//                max m and sum l of exp2 of the log2-scaled logits over the
+//                tile (the inputs of an exact softmax combine).
+//
+// Persistent, warp-specialised CTA (one per SM, 192 threads):
+//   warp 0     TMA producer: the unit's A tile (double-buffered) and a ring of
+//              B tiles, 128 rows x d, 128-byte swizzle.
+//   warp 1     allocates 256 TMEM columns (two fp32 128x128 accumulators) and
+//              issues tcgen05.mma (M=128, N=128, K=16) from one thread.
+//   warps 2-5  epilogue: each thread owns one accumulator row (TMEM lane),
+//              reads it with tcgen05.ld and reduces it.
+// A unit is a run of up to `chunk` consecutive tiles sharing one A tile.
+#pragma once
+#include "sm100.cuh"
+
+namespace pa {
+
+enum { MODE_SCORES = 0, MODE_MASS = 1 };
+
+struct TileParams {
+    int B, nb, NH;         // NH: proxy groups (scores) or q heads (mass)
+    int H, Hkv;            // mass: q head -> KV head
+    int chunk;             // tiles per unit
+    long long units_per_bh;
+    long long num_units;
+    float scale;           // scores: 1/sqrt(d); mass: scale*log2(e)
+    float *scores;         // [B][G][T]
+    float2 *partial;       // [B][H][nb][128] (m, l)
+    uint64_t timeout_ns;
+};
+
+struct Unit {
+    int b, bh_head, qb, kb0, kb1;  // tiles kb0 .. kb1-1
+};
+
+// Scores: within one (b, g) the rows qb = C*a + t (t < C) own a+1 units each,
+// so the units before row C*a number C*a(a+1)/2.
+__device__ __forceinline__ Unit decode_unit(const TileParams &p, long long u, int mode) {
+    Unit r;
+    const long long bh = u / p.units_per_bh;
+    long long w = u - bh * p.units_per_bh;
+    r.b = static_cast<int>(bh / p.NH);
+    r.bh_head = static_cast<int>(bh % p.NH);
+    const int C = p.chunk;
+    if (mode == MODE_SCORES) {
+        long long a = static_cast<long long>((sqrt(1.0 + 8.0 * static_cast<double>(w) / C) - 1.0) * 0.5);
+        while (a > 0 && static_cast<long long>(C) * a * (a + 1) / 2 > w) --a;
+        while (static_cast<long long>(C) * (a + 1) * (a + 2) / 2 <= w) ++a;
+        const long long rem = w - static_cast<long long>(C) * a * (a + 1) / 2;
+        const int t = static_cast<int>(rem / (a + 1));
+        const int c = static_cast<int>(rem % (a + 1));
+        r.qb = static_cast<int>(C * a + t);
+        r.kb0 = c * C;
+        r.kb1 = min(r.kb0 + C, r.qb + 1);
+    } else {
+        r.qb = p.nb - 1;
+        r.kb0 = static_cast<int>(w) * C;
+        r.kb1 = min(r.kb0 + C, p.nb);
+    }
+    return r;
+}
+
+// Order-preserving float <-> uint32 map (for an integer atomicMax on scores).
+__device__ __forceinline__ uint32_t f2ord(float f) {
+    const uint32_t u = __float_as_uint(f + 0.0f);  // -0 -> +0
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float ord2f(uint32_t o) {
+    return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
+}
+
+template <int D>
+struct TileSmem {
+    static constexpr int TILE_BYTES = 128 * D * 2;
+    static constexpr int STAGES = (D == 128) ? 4 : 8;
+    static constexpr int BYTES = (2 + STAGES) * TILE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
+};
+
+template <int D, int MODE>
+__global__ void __launch_bounds__(192, 1)
+    tile_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     TileParams p) {
+    using S = TileSmem<D>;
+    constexpr int TB = S::TILE_BYTES;
+    constexpr int NST = S::STAGES;
+    constexpr int KSTEPS = D / 16;
+    constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, false, false);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;                       // [2][TB]
+    uint8_t *sB = smem + 2 * TB;              // [NST][TB]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (2 + NST) * TB);
+    uint64_t *a_full = bars;                  // 2
+    uint64_t *a_empty = bars + 2;             // 2
+    uint64_t *acc_full = bars + 4;            // 2
+    uint64_t *acc_empty = bars + 6;           // 2
+    uint64_t *b_full = bars + 8;              // NST
+    uint64_t *b_empty = bars + 8 + NST;       // NST
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8 + 2 * NST);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    uint32_t *red_max = tmem_slot + 2;        // [4]
+    uint32_t *red_cnt = tmem_slot + 6;        // [4]
+    uint64_t *drain = reinterpret_cast<uint64_t *>(tmem_slot + 10);  // 8-byte aligned: bars + 8 + 2*NST + 5
+
+    const uint32_t warp = warp_id(), lane = lane_id();
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&a_full[i], 1);
+            mbar_init(&a_empty[i], 1);
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 128);
+        }
+        for (int i = 0; i < NST; ++i) {
+            mbar_init(&b_full[i], 1);
+            mbar_init(&b_empty[i], 1);
+        }
+        for (int i = 0; i < 4; ++i) red_max[i] = red_cnt[i] = 0;
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const WaitCtl wc{abort_flag, p.timeout_ns};
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            long long tile = 0;
+            int local = 0;
+            for (long long u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
+                const Unit un = decode_unit(p, u, MODE);
+                const int a = local & 1;
+                if (local >= 2 && !mbar_wait(&a_empty[a], ((local >> 1) - 1) & 1, wc)) break;
+                ++local;
+                mbar_arrive_expect_tx(&a_full[a], TB);
+#pragma unroll
+                for (int cc = 0; cc < D / 64; ++cc) {
+                    if (MODE == MODE_SCORES)
+                        tma_load_4d(sA + a * TB + cc * 16384, &tmA, &a_full[a], cc * 64, un.qb * 128, un.bh_head, un.b);
+                    else
+                        tma_load_4d(sA + a * TB + cc * 16384, &tmA, &a_full[a], cc * 64, un.bh_head, un.qb * 128, un.b);
+                }
+                const int kvh = (MODE == MODE_MASS)
+                                    ? static_cast<int>(static_cast<long long>(un.bh_head) * p.Hkv / p.H) : 0;
+                bool ok = true;
+                for (int kb = un.kb0; kb < un.kb1; ++kb, ++tile) {
+                    const int s = static_cast<int>(tile % NST);
+                    const long long n = tile / NST;
+                    if (tile >= NST && !mbar_wait(&b_empty[s], (n - 1) & 1, wc)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&b_full[s], TB);
+#pragma unroll
+                    for (int cc = 0; cc < D / 64; ++cc) {
+                        if (MODE == MODE_SCORES)
+                            tma_load_4d(sB + s * TB + cc * 16384, &tmB, &b_full[s], cc * 64, kb * 128, un.bh_head, un.b);
+                        else
+                            tma_load_4d(sB + s * TB + cc * 16384, &tmB, &b_full[s], cc * 64, kvh, kb * 128, un.b);
+                    }
+                }
+                if (!ok) break;
+            }
+            // Let in-flight copies land before the CTA can exit.
+            for (long long t = (tile > NST ? tile - NST : 0); t < tile; ++t)
+                mbar_wait_drain(&b_full[t % NST], (t / NST) & 1, p.timeout_ns);
+            for (int l = (local > 2 ? local - 2 : 0); l < local; ++l)
+                mbar_wait_drain(&a_full[l & 1], (l >> 1) & 1, p.timeout_ns);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            long long tile = 0;
+            int local = 0;
+            bool ok = true;
+            for (long long u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++local) {
+                const Unit un = decode_unit(p, u, MODE);
+                const int a = local & 1;
+                if (!mbar_wait(&a_full[a], (local >> 1) & 1, wc)) break;
+                tc_fence_after();
+                const uint32_t a_base = smem_u32(sA + a * TB);
+                for (int kb = un.kb0; kb < un.kb1; ++kb, ++tile) {
+                    const int s = static_cast<int>(tile % NST);
+                    if (!mbar_wait(&b_full[s], (tile / NST) & 1, wc)) { ok = false; break; }
+                    const int acc = static_cast<int>(tile & 1);
+                    if (tile >= 2 && !mbar_wait(&acc_empty[acc], ((tile >> 1) - 1) & 1, wc)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t b_base = smem_u32(sB + s * TB);
+#pragma unroll
+                    for (int kk = 0; kk < KSTEPS; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                        umma_ss(tmem + acc * 128, sdesc_sw128(a_base + off, 16, 1024),
+                                sdesc_sw128(b_base + off, 16, 1024), IDESC, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&b_empty[s]);
+                    umma_commit(&acc_full[acc]);
+                }
+                if (ok) umma_commit(&a_empty[a]);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------ epilogue
+        const int q4 = static_cast<int>(warp & 3);
+        const int row = q4 * 32 + static_cast<int>(lane);
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+        long long tile = 0;
+        bool ok = true;
+        for (long long u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+            const Unit un = decode_unit(p, u, MODE);
+            for (int kb = un.kb0; kb < un.kb1; ++kb, ++tile) {
+                const int acc = static_cast<int>(tile & 1);
+                if (!warp_wait(&acc_full[acc], (tile >> 1) & 1, wc)) { ok = false; break; }
+                tc_fence_after();
+                const bool diag = (kb == un.qb);
+                const uint32_t taddr = lane_base + acc * 128;
+                float mx = -INFINITY;
+                uint32_t r[32];
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    tmem_ld32(taddr + ch * 32, r);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float v = __uint_as_float(r[j]);
+                        if (!diag || ch * 32 + j <= row) mx = fmaxf(mx, v);
+                    }
+                }
+                if (MODE == MODE_SCORES) {
+                    tc_fence_before();
+                    mbar_arrive(&acc_empty[acc]);
+                    float w = mx * p.scale;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) w = fmaxf(w, __shfl_xor_sync(0xffffffffu, w, o));
+                    if (lane == 0) {
+                        const int slot = static_cast<int>(tile & 3);
+                        atomicMax(&red_max[slot], f2ord(w));
+                        __threadfence_block();
+                        if (atomicAdd(&red_cnt[slot], 1u) == 3u) {
+                            const uint32_t best = atomicExch(&red_max[slot], 0u);
+                            atomicExch(&red_cnt[slot], 0u);
+                            const long long T = static_cast<long long>(p.nb) * (p.nb + 1) / 2;
+                            const long long idx = (static_cast<long long>(un.b) * p.NH + un.bh_head) * T +
+                                                  static_cast<long long>(un.qb) * (un.qb + 1) / 2 + kb;
+                            p.scores[idx] = ord2f(best);
+                        }
+                    }
+                } else {
+                    // log2-domain row max and sum of exp2 over the valid entries
+                    const float m = mx * p.scale;
+                    float l = 0.0f;
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        tmem_ld32(taddr + ch * 32, r);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const float e = ex2(fmaf(__uint_as_float(r[j]), p.scale, -m));
+                            if (!diag || ch * 32 + j <= row) l += e;
+                        }
+                    }
+                    tc_fence_before();
+                    mbar_arrive(&acc_empty[acc]);
+                    const long long idx =
+                        ((static_cast<long long>(un.b) * p.H + un.bh_head) * p.nb + kb) * 128 + row;
+                    p.partial[idx] = make_float2(m, l);
+                }
+            }
+        }
+    }
+
+    // ---------------------------------------------------------- teardown
+    if (warp == 1) {
+        // every MMA (and commit) this CTA issued has completed before TMEM is released
+        if (lane == 0) {
+            umma_commit(drain);
+            mbar_wait_drain(drain, 0, p.timeout_ns);
+        }
+        __syncwarp();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 256);
+}
+
+}  // namespace pa

@@ -1,0 +1,212 @@
+/*
+ * pa.h -- C ABI of libpa.so: ProxyAttn-style block-sparse prefill attention
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The method (ProxyAttn blog, HIT; "4. ProxyAttn method"):
+ *   Step 1  head pooling -> token-level proxy scores max-pooled to 128x128
+ *           blocks -> ranking of the KV blocks of every query block;
+ *   Step 2  a per-head budget estimated from the last query block, combined
+ *           with the shared ranking into a block-sparse mask that drives a
+ *           FlashAttention-style kernel.
+ * Each call below is one of those steps; pa_prefill chains them.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Tensors.  q is [B][N][H][d], k and v are [B][N][Hkv][d], o is [B][N][H][d],
+ *   all bf16, addressed with pa_strides (element strides of the batch, token
+ *   and head dimensions); d is contiguous.  Base pointers must be 16-byte
+ *   aligned and every stride a multiple of 8 elements (16 bytes).
+ *   Proxies q_proxy/k_proxy are contiguous bf16 [B][G][N][d].
+ *   Block scores and ranked lists are [B][G][T] with nb = N/128,
+ *   T = nb(nb+1)/2 and query block qb's row starting at tri(qb) = qb(qb+1)/2
+ *   (entries tri(qb)+0 .. tri(qb)+qb).
+ * Heads.  kv(h) = floor(h*Hkv/H) (GQA), grp(h) = floor(h*G/H) (proxy group).
+ * Memory.  Every pointer is a device pointer owned by the caller unless a
+ *   comment says otherwise.  The library allocates no device memory; calls
+ *   that need scratch take a caller-provided workspace (pa_workspace_size).
+ * Streams.  Every call is asynchronous on `stream` (a cudaStream_t; 0 is the
+ *   legacy default stream).  Argument errors are returned synchronously before
+ *   anything is launched; a failed launch returns PA_ERR_CUDA.  Problems found
+ *   on the device (a wait that timed out, an index out of range) are recorded
+ *   in a device status word read by pa_get_device_status.
+ * Threads.  Calls are reentrant; concurrent calls on different streams are
+ *   independent except for the shared device status word.
+ * Supported.  block = 128, d in {64, 128}, N % 128 == 0, 1 <= N/128 <= 4096,
+ *   H % Hkv == 0, H % G == 0, H <= 128, B >= 1.  Others: PA_ERR_UNSUPPORTED.
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PA_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+typedef struct CUstream_st *pa_stream_t; /* same type as cudaStream_t */
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad stride, gamma out of (0,1], ... */
+    PA_ERR_UNSUPPORTED = 2,   /* shape outside the supported set above */
+    PA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than pa_workspace_size */
+    PA_ERR_CUDA = 4,          /* a CUDA runtime/driver call or a launch failed */
+    PA_ERR_TIMEOUT = 5,       /* device: a bounded wait ran out (kernel abandoned its work) */
+    PA_ERR_DEVICE_BOUNDS = 6, /* device: a block index outside 0..qb was met in a list */
+    PA_ERR_DEVICE_NONFINITE = 7 /* device: a block score or head mass was NaN/inf */
+} pa_status;
+
+typedef struct pa_shape {
+    int32_t batch;        /* B */
+    int32_t seqlen;       /* N, multiple of 128 */
+    int32_t num_q_heads;  /* H */
+    int32_t num_kv_heads; /* Hkv, divides H */
+    int32_t head_dim;     /* d: 64 or 128 */
+    int32_t block;        /* must be 128 */
+    int32_t num_groups;   /* G proxy groups, divides H */
+} pa_shape;
+
+typedef struct pa_strides {
+    int64_t b, s, h;      /* element strides of the batch, token and head dims */
+} pa_strides;
+
+typedef enum pa_budget_mode {
+    PA_BUDGET_DYNAMIC = 0,        /* per-head gamma budget from the last query block */
+    PA_BUDGET_FIXED_FRACTION = 1, /* ceil(frac_permille * (qb+1) / 1000) blocks per row */
+    PA_BUDGET_ALL = 2             /* every causal block (dense causal attention) */
+} pa_budget_mode;
+
+typedef struct pa_budget {
+    int32_t mode;          /* pa_budget_mode */
+    float gamma;           /* DYNAMIC: softmax-mass threshold in (0, 1] */
+    int32_t frac_permille; /* FIXED_FRACTION: 1..1000 */
+} pa_budget;
+
+/* Mask buffers written by pa_build_mask / pa_prefill (device, caller-owned).
+ *   rank   int32 [B][G][T]  ranked list of each query block:
+ *                           [0, qb, then blocks 1..qb-1 by (score desc, index asc)]
+ *   cnt    int32 [B][H][nb] blocks head h visits in query block qb: the first
+ *                           cnt entries of its group's list
+ *   budget int32 [B][H]     per-head budget k_h (= cnt at the last query block)
+ *   mass   float [B][H][nb] last-block softmax mass per KV block (DYNAMIC mode;
+ *                           may be NULL in the other modes) */
+typedef struct pa_mask {
+    int32_t *rank;
+    int32_t *cnt;
+    int32_t *budget;
+    float *mass;
+} pa_mask;
+
+/* Bytes of workspace pa_prefill needs for this shape and budget (it is also
+ * enough for pa_build_mask).  Returns 0 for an invalid or unsupported shape.
+ * The workspace is scratch: its contents need no initialisation and are
+ * meaningless after the call.  Two calls in flight at once need two
+ * workspaces. */
+PA_API size_t pa_workspace_size(const pa_shape *shape, const pa_budget *budget);
+
+/* Step 1, "Head Pooling" (ProxyAttn blog, 4. ProxyAttn method, Step 1):
+ *   q_proxy[b][g][i][:] = mean over the q heads h of group g of q[b][i][h][:]
+ *   k_proxy[b][g][j][:] = mean over the same q heads h of k[b][j][kv(h)][:]
+ * Sums run in fp64 over ascending h, the quotient is rounded to bf16 (round to
+ * nearest even).  q_proxy, k_proxy: contiguous bf16 [B][G][N][d]. */
+PA_API pa_status pa_pool_heads(const pa_shape *shape,
+                        const void *q, pa_strides q_strides,
+                        const void *k, pa_strides k_strides,
+                        void *q_proxy, void *k_proxy, pa_stream_t stream);
+
+/* Step 1, "Score Estimation" (ProxyAttn blog, 4. ProxyAttn method, Step 1;
+ * block size from "2. Background: why block-wise"): the QK product of the
+ * proxies fused with 128x128 max pooling.  For every (b, g, qb, kb <= qb):
+ *   scores[b][g][tri(qb)+kb] = max over i in block qb, j in block kb, j <= i of
+ *                              (q_proxy[i] . k_proxy[j]) / sqrt(d)
+ * bf16 tensor-core products, fp32 accumulation; token scores never reach
+ * memory.  scores: fp32 [B][G][T]. */
+PA_API pa_status pa_block_scores(const pa_shape *shape,
+                          const void *q_proxy, const void *k_proxy,
+                          float *scores, pa_stream_t stream);
+
+/* Step 1 "Block Ranking" + Step 2 "dynamic budget" (ProxyAttn blog,
+ * 4. ProxyAttn method; the threshold rule is XAttention's find_blocks,
+ * XAttention blog 2.2):
+ *  - rank: per (b, g, qb) the list [0, qb, then 1..qb-1 by (score desc,
+ *    lower index first)] of the scores from pa_block_scores;
+ *  - mass (DYNAMIC): for each head h, the exact softmax (scale 1/sqrt(d), causal)
+ *    of the last 128 query rows of q against all keys of kv(h); mass[b][h][kb]
+ *    = mean over those rows of the probability falling in KV block kb;
+ *  - budget: DYNAMIC: with m_fx = rint(mass * 2^40), g_fx = rint(gamma * 2^40),
+ *    k_h = smallest k >= |F| (|F| = 2, or 1 when nb = 1) such that the first k
+ *    entries of the last row's list carry sum m_fx >= g_fx, else nb;
+ *    cnt[b][h][qb] = clamp(ceil(k_h (qb+1) / nb), |F_qb|, qb+1).
+ *    FIXED_FRACTION: cnt = clamp(ceil(p (qb+1) / 1000), |F_qb|, qb+1).
+ *    ALL: cnt = qb+1.  budget = cnt at qb = nb-1.
+ * q and k are only read in DYNAMIC mode (may be NULL otherwise).  ws: device
+ * workspace of ws_bytes >= pa_workspace_size(shape, budget). */
+PA_API pa_status pa_build_mask(const pa_shape *shape, const pa_budget *budget,
+                        const float *scores,
+                        const void *q, pa_strides q_strides,
+                        const void *k, pa_strides k_strides,
+                        const pa_mask *out, void *ws, size_t ws_bytes,
+                        pa_stream_t stream);
+
+/* The block-sparse mask "fed to FlashAttention" (ProxyAttn blog, end of
+ * 4. ProxyAttn method; attention formula of "2. Background"): for every
+ * (b, h, qb) with list L = rank[b][grp(h)][tri(qb) ..] and n = cnt[b][h][qb],
+ *   o[b][i][h] = sum_j softmax_j(softmax_scale * q_i . k_j) v_j
+ * over the keys j of blocks L[0..n-1] with j <= i (i in block qb).
+ * bf16 tensor-core products, fp32 softmax and accumulation, P rounded to bf16
+ * for the PV product.  lse (nullable): fp32 [B][H][N], natural-log
+ * log-sum-exp of the scaled logits of each row.  List entries outside 0..qb
+ * are skipped and flagged PA_ERR_DEVICE_BOUNDS; lists must not repeat a block.
+ * o must not overlap q, k or v. */
+PA_API pa_status pa_block_sparse_attn(const pa_shape *shape,
+                               const void *q, pa_strides q_strides,
+                               const void *k, pa_strides k_strides,
+                               const void *v, pa_strides v_strides,
+                               const int32_t *rank, const int32_t *cnt,
+                               float softmax_scale,
+                               void *o, pa_strides o_strides, float *lse,
+                               pa_stream_t stream);
+
+/* The whole path: pa_pool_heads -> pa_block_scores -> pa_build_mask ->
+ * pa_block_sparse_attn with softmax_scale = 1/sqrt(d).  The proxies and block
+ * scores live in the workspace; the mask is written to *mask_out (all four
+ * buffers required in DYNAMIC mode, mass may be NULL otherwise). */
+PA_API pa_status pa_prefill(const pa_shape *shape, const pa_budget *budget,
+                     const void *q, pa_strides q_strides,
+                     const void *k, pa_strides k_strides,
+                     const void *v, pa_strides v_strides,
+                     void *o, pa_strides o_strides,
+                     const pa_mask *mask_out, void *ws, size_t ws_bytes,
+                     pa_stream_t stream);
+
+/* Synchronises `stream`, then returns the device status word of the current
+ * device (PA_OK, PA_ERR_TIMEOUT, PA_ERR_DEVICE_BOUNDS or PA_ERR_DEVICE_NONFINITE:
+ * the first problem any
+ * kernel recorded since the last clear) and, if `clear` is nonzero, resets it.
+ * The word is shared by every stream of the device. */
+PA_API pa_status pa_get_device_status(pa_stream_t stream, int clear);
+
+/* Static description of a status code. */
+PA_API const char *pa_status_string(pa_status status);
+
+/* Thread-local text of the last error a call on this thread returned
+ * (empty if none). */
+PA_API const char *pa_last_error(void);
+
+/* PA_ABI_VERSION of the loaded library. */
+PA_API int32_t pa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H */

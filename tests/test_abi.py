@@ -1,0 +1,126 @@
+"""The C ABI without a GPU: libpa.so loads, exports every entry point that
+include/pa.h declares, and rejects bad arguments synchronously (before any
+launch) with the documented status codes."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_pa_b200 as pa
+from block_sparse_attention_pa_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return pa.lib()
+
+
+def declared_entry_points():
+    src = open(os.path.join(ROOT, "include", "pa.h")).read()
+    return sorted(set(re.findall(r"PA_API\s+[\w\s\*]*?\b(pa_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_entry_points():
+    assert declared_entry_points() == sorted(pa.ENTRY_POINTS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_entry_points():
+        assert hasattr(L, name), name
+
+
+def test_version_and_status_strings(L):
+    assert L.pa_abi_version() == 1
+    for code in range(8):
+        assert L.pa_status_string(code).decode() not in ("", "unknown status")
+    assert L.pa_status_string(99).decode() == "unknown status"
+
+
+def shape(B=1, N=1024, H=8, Hkv=2, d=64, blk=128, G=1):
+    return pa.Shape(B, N, H, Hkv, d, blk, G)
+
+
+def test_workspace_size_formula(L):
+    s = shape(N=1024, H=8, Hkv=2, d=64, G=2)
+    nb = 8
+    T = nb * (nb + 1) // 2
+    a256 = lambda x: (x + 255) // 256 * 256
+    dyn = pa.workspace_size(s, pa.make_budget(pa.DYNAMIC, 0.9))
+    assert dyn == a256(8 * nb * 128 * 8) + 2 * a256(2 * 1024 * 64 * 2) + a256(2 * T * 4)
+    fixed = pa.workspace_size(s, pa.make_budget(pa.FIXED_FRACTION, 0, 100))
+    assert fixed == 2 * a256(2 * 1024 * 64 * 2) + a256(2 * T * 4)
+    assert pa.workspace_size(shape(N=1000), pa.make_budget()) == 0
+    assert pa.workspace_size(s, pa.make_budget(pa.DYNAMIC, 1.5)) == 0
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(N=1000), 2),          # N % 128
+    (dict(d=96), 2),            # head_dim
+    (dict(blk=64), 2),          # block
+    (dict(H=8, Hkv=3), 2),      # H % Hkv
+    (dict(H=8, G=3), 2),        # H % G
+    (dict(N=128 * 4097), 2),    # too long
+    (dict(H=0), 1),             # non-positive
+    (dict(B=0), 1),
+])
+def test_bad_shapes_rejected_before_launch(L, bad, code):
+    s = shape(**bad)
+    st = pa.Strides(0, 512, 64)
+    r = L.pa_pool_heads(ctypes.byref(s), 16, st, 16, st, 16, 16, None)
+    assert r == code
+    assert L.pa_last_error() != b""
+
+
+def test_null_and_misaligned_pointers_rejected(L):
+    s = shape()
+    st = pa.Strides(0, 512, 64)
+    assert L.pa_pool_heads(ctypes.byref(s), None, st, 16, st, 16, 16, None) == 1
+    assert L.pa_pool_heads(ctypes.byref(s), 8, st, 16, st, 16, 16, None) == 1      # 8-byte aligned only
+    assert L.pa_pool_heads(ctypes.byref(s), 16, pa.Strides(0, 512, 60), 16, st, 16, 16, None) == 1
+    assert L.pa_block_scores(ctypes.byref(s), 16, 16, None, None) == 1
+    assert L.pa_block_scores(None, 16, 16, 16, None) == 1
+
+
+def test_budget_and_workspace_errors(L):
+    s = shape()
+    st = pa.Strides(0, 512, 64)
+    m = pa.MaskBufs(16, 16, 16, 16)
+    for bad in (pa.make_budget(pa.DYNAMIC, 0.0), pa.make_budget(pa.DYNAMIC, 1.01),
+                pa.make_budget(pa.FIXED_FRACTION, 0, 0), pa.make_budget(pa.FIXED_FRACTION, 0, 1001),
+                pa.make_budget(7, 0.5, 0)):
+        assert L.pa_build_mask(ctypes.byref(s), ctypes.byref(bad), 16, 16, st, 16, st, ctypes.byref(m), 256, 1 << 30,
+                               None) == 1
+    good = pa.make_budget(pa.DYNAMIC, 0.9)
+    # dynamic mode needs the mass buffer and a large enough workspace
+    m_nomass = pa.MaskBufs(16, 16, 16, None)
+    assert L.pa_build_mask(ctypes.byref(s), ctypes.byref(good), 16, 16, st, 16, st, ctypes.byref(m_nomass), 256,
+                           1 << 30, None) == 1
+    assert L.pa_build_mask(ctypes.byref(s), ctypes.byref(good), 16, 16, st, 16, st, ctypes.byref(m), 256, 16,
+                           None) == 3
+    need = pa.workspace_size(s, good)
+    assert L.pa_prefill(ctypes.byref(s), ctypes.byref(good), 16, st, 16, st, 16, st, 16, st, ctypes.byref(m), 256,
+                        need - 1, None) == 3
+    assert L.pa_prefill(ctypes.byref(s), ctypes.byref(good), 16, st, 16, st, 16, st, 16, st, ctypes.byref(m), None,
+                        need, None) == 3
+
+
+def test_attention_argument_errors(L):
+    s = shape()
+    st = pa.Strides(0, 512, 64)
+    assert L.pa_block_sparse_attn(ctypes.byref(s), 16, st, 16, st, 16, st, 16, 16, ctypes.c_float(0.0), 16, st, None,
+                                  None) == 1
+    assert L.pa_block_sparse_attn(ctypes.byref(s), 16, st, 16, st, 16, st, None, 16, ctypes.c_float(0.125), 16, st,
+                                  None, None) == 1
+    assert L.pa_block_sparse_attn(ctypes.byref(s), 16, st, 16, st, 16, st, 16, 16, ctypes.c_float(0.125), 16, st,
+                                  2, None) == 1  # misaligned lse
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 128, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        pa.pool_heads(q, q, 1)
