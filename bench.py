@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Benchmark: ProxyAttn-style block-sparse prefill attention on B200.
+
+One step = one pass of the whole path over one attention layer of synthetic
+input already resident in HBM: head pooling -> fused proxy block scores ->
+mask (last-block head mass, ranking, per-head budget) -> block-sparse
+attention, each stage called through the C ABI (libpa.so) on the current
+stream with CUDA events between stages.
+
+Default workload: the Llama-3.1-8B layer at 128K tokens (batch 1, 32 q heads,
+8 KV heads, head_dim 128, G = 1, gamma = 0.95).  The printed JSON line carries
+ms per layer (estimate + sparse), effective TFLOP/s over the visited blocks,
+per-stage times, sparsity, the speedup over the same kernel with every causal
+block selected, the attention kernel's roofline, an end-to-end number through
+the public API with host buffers, SM clocks sampled during the timed region
+and the CPU oracle's time on a bounded sample.
+
+Multi-GPU (torchrun): replicas only -- every rank runs its own independent
+layer (the path needs no exchange); the step time is the max over ranks.
+
+`--impl reference` times the CPU oracle (the only reference there is) on a
+bounded sample of the same workload each step, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from block_sparse_attention_pa_b200 import synth  # noqa: E402
+
+METRIC = ("prefill attention ms/layer (estimate + sparse) and effective TFLOP/s at 128K, 1×B200")
+MODES = {"dynamic": 0, "fixed": 1, "all": 2}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama8b_n128k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--groups", type=int, default=None, help="proxy groups G (default: the workload's)")
+    ap.add_argument("--mode", choices=sorted(MODES), default="dynamic")
+    ap.add_argument("--gamma", type=float, default=None)
+    ap.add_argument("--frac", type=int, default=100, help="fixed budget in per mille of causal blocks")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons of this GPU."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.lines = []
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            sel = str(device_index)
+        self.cmd = ["nvidia-smi", "-i", sel, "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
+                    "--format=csv,noheader,nounits", "-lms", "100"]
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 4:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+                mask = int(parts[3], 16)
+            except ValueError:
+                continue
+            for bit, name in self.REASONS.items():
+                if mask & bit:
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------- the pipeline
+class Pipeline:
+    """Pre-allocated buffers and ctypes arguments for one layer, so that a step is
+    four C-ABI calls with CUDA events between them."""
+
+    def __init__(self, q, k, v, G, mode, gamma, frac):
+        import block_sparse_attention_pa_b200 as pa
+        self.pa = pa
+        self.L = pa.lib()
+        self.q, self.k, self.v = q, k, v
+        B, N, H, d = q.shape
+        self.B, self.N, self.H, self.d, self.G = B, N, H, d, G
+        self.nb = N // 128
+        self.shape = pa.make_shape(q, k, G)
+        self.budget = pa.make_budget(mode, gamma, frac)
+        self.mode = mode
+        dev = q.device
+        self.qp = torch.empty(B, G, N, d, device=dev, dtype=torch.bfloat16)
+        self.kp = torch.empty_like(self.qp)
+        T = self.nb * (self.nb + 1) // 2
+        self.T = T
+        self.scores = torch.empty(B, G, T, device=dev, dtype=torch.float32)
+        self.mask = pa.Mask.empty(self.shape, dev, mode == 0)
+        self.bufs = self.mask.bufs()
+        self.ws = torch.empty(max(pa.workspace_size(self.shape, self.budget), 256), device=dev, dtype=torch.uint8)
+        self.o = torch.empty_like(q)
+        self.qs, self.ks, self.vs, self.os_ = (pa._strides(t) for t in (q, k, v, self.o))
+        self.scale = 1.0 / math.sqrt(d)
+        self.launches_per_step = 5 + (2 if mode == 0 else 0)  # pool, scores, [mass, combine], rank, budget, attn
+
+    def step(self, ev=None):
+        pa, L, st = self.pa, self.L, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        sh, bu = ctypes.byref(self.shape), ctypes.byref(self.budget)
+        if ev: ev[0].record()
+        pa._check(L.pa_pool_heads(sh, self.q.data_ptr(), self.qs, self.k.data_ptr(), self.ks, self.qp.data_ptr(),
+                                  self.kp.data_ptr(), st))
+        if ev: ev[1].record()
+        pa._check(L.pa_block_scores(sh, self.qp.data_ptr(), self.kp.data_ptr(), self.scores.data_ptr(), st))
+        if ev: ev[2].record()
+        pa._check(L.pa_build_mask(sh, bu, self.scores.data_ptr(), self.q.data_ptr(), self.qs, self.k.data_ptr(),
+                                  self.ks, ctypes.byref(self.bufs), self.ws.data_ptr(), self.ws.numel(), st))
+        if ev: ev[3].record()
+        pa._check(L.pa_block_sparse_attn(sh, self.q.data_ptr(), self.qs, self.k.data_ptr(), self.ks,
+                                         self.v.data_ptr(), self.vs, self.mask.rank.data_ptr(),
+                                         self.mask.cnt.data_ptr(), self.scale, self.o.data_ptr(), self.os_, None,
+                                         st))
+        if ev: ev[4].record()
+
+    def visited(self):
+        """(visited blocks, algorithmic attention FLOPs with the diagonal tile
+        counted in full, exact causal FLOPs)."""
+        v = int(self.mask.cnt.sum().item())
+        ndiag = self.B * self.H * self.nb
+        per = 4 * 128 * 128 * self.d
+        exact = (v - ndiag) * per + ndiag * 4 * self.d * (128 * 129 // 2)
+        return v, v * per, exact
+
+
+def time_pipeline(pipe, steps, warmup, dist_on, sampler=None):
+    for _ in range(warmup):
+        pipe.step()
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        pipe.step(evs[i])
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    if dist_on:
+        torch.distributed.barrier()
+    total = evs[0][0].elapsed_time(evs[-1][4])
+    stages = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])
+    return total, stages.mean(0), clocks
+
+
+def counters_for(kernel_key: str, source_files):
+    """DRAM bytes of a kernel from a committed ncu summary, if the kernel's
+    sources still hash to what was profiled; else None."""
+    p = os.path.join(ROOT, "profiles", "counters.json")
+    try:
+        with open(p) as f:
+            c = json.load(f)[kernel_key]
+    except Exception:
+        return None
+    h = hashlib.sha256()
+    for s in source_files:
+        with open(os.path.join(ROOT, s), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != c.get("source_sha256"):
+        return None
+    return c
+
+
+ATTN_SOURCES = ["block_sparse_attention_pa_b200/csrc/attn.cuh", "block_sparse_attention_pa_b200/csrc/sm100.cuh"]
+
+
+# ------------------------------------------------------------ CPU oracle
+def oracle_estimate(x, w: synth.Workload, G, mode, gamma, frac, size="baseline", seed=0):
+    """Time the CPU oracle on a bounded sample of one layer and extrapolate to
+    ms per layer.  x: CPU bf16 tensors.  Returns (ms_per_layer, per-stage
+    seconds, description of the sample)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    q, k, v = x["q"], x["k"], x["v"]
+    B, N, H, d = q.shape
+    Hkv = k.shape[2]
+    nb = N // 128
+    T = nb * (nb + 1) // 2
+    if size == "baseline":   # about 10-30 s of CPU work at 128K
+        pool_tokens, n_tiles, mass_heads, n_items = N, nb, H // Hkv * 2, 8
+    else:                    # one reference-arm step: a few seconds
+        pool_tokens, n_tiles, mass_heads, n_items = min(N, 8192), 64, 1, 1
+    det = {}
+    # o1 pool on the first pool_tokens tokens
+    t0 = time.perf_counter()
+    _, _, qpb, kpb = oracle.pool(q[:, :pool_tokens], k[:, :pool_tokens], G)
+    det["pool_s"] = (time.perf_counter() - t0) * N / pool_tokens
+    # o2 block scores of n_tiles tiles of the last query block inside the pooled tokens
+    nbp = pool_tokens // 128
+    kbs = np.linspace(0, nbp - 1, min(n_tiles, nbp)).astype(int)
+    tiles = [(0, g, nbp - 1, int(kb)) for g in range(G) for kb in kbs]
+    t0 = time.perf_counter()
+    last = oracle.block_score_tiles(qpb, kpb, tiles)
+    det["scores_s"] = (time.perf_counter() - t0) * (B * G * T) / len(tiles)
+    # o3 head mass of mass_heads heads (with their KV heads)
+    hk = max(1, mass_heads * Hkv // H)
+    t0 = time.perf_counter()
+    mass_s = oracle.head_mass(q[:, :, :mass_heads].contiguous(), k[:, :, :hk].contiguous())
+    det["mass_s"] = (time.perf_counter() - t0) * H / mass_heads if mode == 0 else 0.0
+    # o4 ranking over the full [B, G, T] array (seeded fill; the sampled last-row tiles real)
+    scores = rng.standard_normal((B, G, T))
+    if nbp == nb:
+        for (b, g, qb, kb), s in zip(tiles, last):
+            scores[b, g, T - nb + kb] = s
+    t0 = time.perf_counter()
+    rank = oracle.rank(scores, nb)
+    det["rank_s"] = time.perf_counter() - t0
+    # budget with the sampled heads' masses repeated over all heads
+    mass = np.tile(mass_s, (1, -(-H // mass_heads), 1))[:, :H]
+    t0 = time.perf_counter()
+    _, cnt = oracle.budget(rank, mass if mode == 0 else None, H, G, nb, mode, float(np.float32(gamma)), frac)
+    det["budget_s"] = time.perf_counter() - t0
+    # o5 sparse attention on random (b, h, qb) items, extrapolated per visited block
+    items = [(int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(nb))) for _ in range(n_items)]
+    t0 = time.perf_counter()
+    oracle.sparse_attn(q, k, v, rank, cnt, G, items)
+    dt = time.perf_counter() - t0
+    blocks = sum(int(cnt[b, h, qb]) for b, h, qb in items)
+    det["attn_s"] = dt * float(cnt.sum()) / max(blocks, 1)
+    sample = (f"pool of {pool_tokens}/{N} tokens; scores of {len(tiles)}/{B * G * T} tiles; head mass of "
+              f"{mass_heads}/{H} heads; full rank+budget; attention of {n_items} random (b,h,qb) items "
+              f"({blocks} of {int(cnt.sum())} visited blocks); each stage extrapolated linearly")
+    return sum(det.values()) * 1e3, det, sample
+
+
+def run_reference(args, w, G, mode, gamma, frac):
+    """The reference arm: the CPU oracle, timed on the host cores."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    import oracle
+    x = synth.make_inputs(w, device="cpu")
+    vals = []
+    for i in range(args.warmup + args.steps):
+        ms, det, sample = oracle_estimate(x, w, G, mode, gamma, frac, size="step", seed=i)
+        if i >= args.warmup:
+            vals.append(ms)
+    v = statistics.mean(vals)
+    cores = oracle.num_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "ms/layer", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, G, mode, gamma, frac),
+            "cpu_baseline": {"value": v, "unit": "ms/layer", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "ms/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, G, mode, gamma, frac):
+    budget = {0: f"dynamic gamma={gamma}", 1: f"fixed {frac / 10:.1f}% of causal blocks", 2: "all causal blocks"}[mode]
+    return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "q_heads": w.num_q_heads,
+            "kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "groups": G, "budget": budget, "block": 128,
+            "l2": "inputs larger than L2 (q+k+v per layer > 126 MB), no flush"}
+
+
+# ------------------------------------------------------------------- main
+def main():
+    args = parse_args()
+    w = synth.WORKLOADS[args.workload]
+    G = args.groups or w.num_groups
+    mode = MODES[args.mode]
+    gamma = args.gamma if args.gamma is not None else w.gamma
+    frac = args.frac
+    if args.impl == "reference":
+        run_reference(args, w, G, mode, gamma, frac)
+        return
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist_on = world > 1
+    torch.cuda.set_device(local)
+    if dist_on:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    import block_sparse_attention_pa_b200 as pa
+    pa.lib()  # fails loudly when libpa.so is missing
+
+    x = synth.make_inputs(w, device=f"cuda:{local}", seed=w.seed + rank)
+    q, k, v = x["q"], x["k"], x["v"]
+    pipe = Pipeline(q, k, v, G, mode, gamma, frac)
+    sampler = None if args.no_clocks else ClockSampler(local)
+    total_ms, stages, clocks = time_pipeline(pipe, args.steps, args.warmup, dist_on, sampler)
+    status = pa.device_status()
+    if status != 0:
+        raise SystemExit(f"device status {status} after the timed run")
+    t = torch.tensor([total_ms], device=q.device, dtype=torch.float64)
+    if dist_on:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_step = total_ms / args.steps
+    visited, flops, flops_exact = pipe.visited()
+    B, H, nb = w.batch, w.num_q_heads, pipe.nb
+    T = nb * (nb + 1) // 2
+    density = visited / (B * H * T)
+    est_ms = float(stages[:3].sum())
+    attn_ms = float(stages[3])
+
+    peaks, peaks_kind = load_peaks()
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    ctr = counters_for("attn_kernel", ATTN_SOURCES)
+    traffic = None
+    if ctr and ctr.get("dram_bytes_per_visited_block"):
+        traffic = float(ctr["dram_bytes_per_visited_block"]) * visited
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": traffic, "kernel": "attn_kernel<128> (block-sparse attention)",
+                "peak_kind": f"{peaks_kind} bf16 sustained (kernel timed inside back-to-back steps)",
+                "flops_per_launch": flops, "exact_causal_flops_per_launch": flops_exact}
+
+    # per-stage rooflines
+    d = w.head_dim
+    Hkv = w.num_kv_heads
+    pool_bytes = B * w.seqlen * d * 2 * (H + Hkv + 2 * G)
+    score_flops = B * G * T * 2 * 128 * 128 * d
+    stage_roofline = {
+        "pool": {"ms": float(stages[0]), "GB/s": pool_bytes / (stages[0] * 1e-3) / 1e9,
+                 "frac_hbm": pool_bytes / (stages[0] * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "scores": {"ms": float(stages[1]), "TFLOP/s": score_flops / (stages[1] * 1e-3) / 1e12,
+                   "frac_tensor": score_flops / (stages[1] * 1e-3) / 1e12 / peak},
+        "mask": {"ms": float(stages[2])},
+        "attn": {"ms": attn_ms, "TFLOP/s": achieved, "frac_tensor": achieved / peak},
+    }
+
+    line = {"metric": METRIC, "value": ms_step / world, "unit": "ms/layer", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded needle/sink generator; random inputs, no weights)",
+            "config": config_of(w, G, mode, gamma, frac) | {"parallelism": f"replicas x{world}"},
+            "est_ms": est_ms, "sparse_ms": attn_ms,
+            "tflops_effective": achieved, "tflops_exact_causal": flops_exact / (attn_ms * 1e-3) / 1e12,
+            "visited_blocks": visited, "density": density, "sparsity": 1.0 - density,
+            "stages_ms": {"pool": float(stages[0]), "scores": float(stages[1]), "mask": float(stages[2]),
+                          "attn": attn_ms},
+            "stage_roofline": stage_roofline, "roofline": roofline,
+            "gpu_launches": pipe.launches_per_step * args.steps}
+    if clocks:
+        line["clocks"] = clocks
+
+    # dense baseline: the same kernel with every causal block selected
+    if not args.no_dense:
+        dense = Pipeline(q, k, v, G, 2, gamma, frac)
+        dsteps = max(2, min(5, args.steps))
+        _, dstages, _ = time_pipeline(dense, dsteps, 1, dist_on)
+        dense_attn = float(dstages[3])
+        dv, dflops, _ = dense.visited()
+        line["dense_attn_ms"] = dense_attn
+        line["dense_tflops"] = dflops / (dense_attn * 1e-3) / 1e12
+        line["speedup_vs_dense"] = dense_attn / attn_ms
+        line["layer_speedup_vs_dense"] = dense_attn / (est_ms + attn_ms)
+        line["estimate_frac_of_dense"] = est_ms / dense_attn
+        del dense
+
+    # end to end through the public API with pinned host buffers
+    if not args.no_e2e:
+        e2e = run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world)
+        line["e2e"] = e2e
+
+    # the CPU oracle on a bounded sample (rank 0, one GPU only)
+    if not args.no_cpu_baseline and world == 1 and rank == 0:
+        import oracle
+        xc = {n: x[n].cpu() for n in ("q", "k", "v")}
+        ms, det, sample = oracle_estimate(xc, w, G, mode, gamma, frac, size="baseline")
+        line["cpu_baseline"] = {"value": ms, "unit": "ms/layer", "cores": oracle.num_threads(), "kind": "oracle",
+                                "sample": sample, "stage_s": det}
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world):
+    q, k, v = x["q"], x["k"], x["v"]
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    dq, dk, dv = (torch.empty_like(t) for t in (q, k, v))
+    call = pa.Prefill(dq, dk, dv, G, mode, gamma, frac)
+    do = torch.empty_like(dq)
+    ho = torch.empty(do.shape, dtype=do.dtype, pin_memory=True)
+    steps = max(2, min(5, args.steps))
+
+    def one():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        call(dq, dk, dv, do)
+        ho.copy_(do, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        one()
+    e.record()
+    torch.cuda.synchronize()
+    t = torch.tensor([s.elapsed_time(e)], device=q.device, dtype=torch.float64)
+    if dist_on:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms = float(t.item()) / steps
+    if pa.device_status() != 0:
+        raise SystemExit("device status flagged in the end-to-end run")
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    return {"value": ms / world, "unit": "ms/layer", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": ho.numel() * ho.element_size(), "steps": steps}
+
+
+if __name__ == "__main__":
+    main()

@@ -31,6 +31,13 @@ namespace pa {
 
 constexpr int kMaxHeads = 128;
 
+// Of every 8 column pairs of a non-diagonal S tile, this many take their
+// exponentials from the FMA-pipe polynomial instead of the MUFU unit.
+#ifndef PA_POLY_PAIRS_PER8
+#define PA_POLY_PAIRS_PER8 0
+#endif
+constexpr int kPolyPairsPer8 = PA_POLY_PAIRS_PER8;
+
 struct AttnParams {
     int B, N, H, Hkv, G, nb;
     int num_units;             // head units per (b, qb)
@@ -241,36 +248,46 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t o_addr = lane_base + 256 + t * 128;
         float m = -INFINITY, l = 0.0f;
         bool ok = true;
-        uint32_t r[32];
+        uint32_t s[128];
         for (int i = 0; i < ct; ++i) {
             if (!warp_wait(&s_full[t], i & 1, wc)) { ok = false; break; }
             tc_fence_after();
             const int kb = list[i];
             const bool valid = (kb >= 0 && kb <= qb);
-            const bool diag = (kb == qb);
-            // pass 1: row max of this tile
-            float mt = -INFINITY;
+            const bool masked = (kb == qb) || !valid;  // warp-uniform: same tile for the whole CTA
+            tmem_ld128(s_addr, s);
+            if (masked) {
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                tmem_ld32(s_addr + ch * 32, r);
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (valid && (!diag || ch * 32 + j <= row)) mt = fmaxf(mt, __uint_as_float(r[j]));
+                for (int j = 0; j < 128; ++j)
+                    if (!valid || j > row) s[j] = 0xFF800000u;  // -inf: causal mask of the diagonal tile
             }
-            mt *= p.scale_log2;
+            // row max of the tile: a tree of three-input maxima
+            float mx[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const uint32_t *v = s + 8 * j;
+                mx[j] = fmax3(fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2])),
+                              fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5])),
+                              fmaxf(__uint_as_float(v[6]), __uint_as_float(v[7])));
+            }
+            const float mt = p.scale_log2 *
+                fmax3(fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmax3(mx[6], mx[7], mx[8])),
+                      fmax3(mx[9], mx[10], mx[11]), fmax3(mx[12], mx[13], fmaxf(mx[14], mx[15])));
             const float m_new = fmaxf(m, mt);
             if (i > 0) {
                 const bool need = m_new > m + 8.0f;
                 if (__any_sync(0xffffffffu, need)) {
+                    // raise the running max: O (in TMEM) and l scale by 2^(m - m_new)
                     const float alpha = (m == -INFINITY) ? 0.0f : ex2(m - m_new);
                     if (!warp_wait(&o_done[t], (i - 1) & 1, wc)) { ok = false; break; }
                     tc_fence_after();
 #pragma unroll
                     for (int ch = 0; ch < D / 32; ++ch) {
-                        tmem_ld32(o_addr + ch * 32, r);
+                        uint32_t o[32];
+                        tmem_ld32(o_addr + ch * 32, o);
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
-                        tmem_st32(o_addr + ch * 32, r);
+                        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                        tmem_st32(o_addr + ch * 32, o);
                     }
                     tmem_st_wait();
                     l *= alpha;
@@ -279,24 +296,46 @@ __global__ void __launch_bounds__(320, 1)
             } else {
                 m = m_new;
             }
-            const float mref = (m == -INFINITY) ? 0.0f : m;
-            // pass 2: P = exp2(x - m) as bf16 pairs over the S columns, row sum
+            // P = 2^(x - m) as bf16 pairs written over the first 64 columns of S;
+            // a share of the exponentials runs on the FMA pipe (ex2_poly).
+            const float negm = (m == -INFINITY) ? 0.0f : -m;
+            const float c2 = p.scale_log2;
+            float acc[8];
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                tmem_ld32(s_addr + ch * 32, r);
-                uint32_t pk[16];
+            for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int c0 = ch * 32 + 2 * j;
-                    const bool ok0 = valid && (!diag || c0 <= row);
-                    const bool ok1 = valid && (!diag || c0 + 1 <= row);
-                    const float e0 = ok0 ? ex2(fmaf(__uint_as_float(r[2 * j]), p.scale_log2, -mref)) : 0.0f;
-                    const float e1 = ok1 ? ex2(fmaf(__uint_as_float(r[2 * j + 1]), p.scale_log2, -mref)) : 0.0f;
-                    l += e0 + e1;
-                    pk[j] = pack_bf16x2(e0, e1);
+            for (int half = 0; half < 2; ++half) {
+                uint32_t pk[32];
+                if (masked) {
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const int j = half * 32 + jj;
+                        const float e0 = ex2(fmaf(__uint_as_float(s[2 * j]), c2, negm));
+                        const float e1 = ex2(fmaf(__uint_as_float(s[2 * j + 1]), c2, negm));
+                        acc[j & 7] += e0 + e1;
+                        pk[jj] = pack_bf16x2(e0, e1);
+                    }
+                } else {
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) {
+                        const int j = half * 32 + jj;
+                        const float x0 = fmaf(__uint_as_float(s[2 * j]), c2, negm);
+                        const float x1 = fmaf(__uint_as_float(s[2 * j + 1]), c2, negm);
+                        float e0, e1;
+                        if ((j & 7) < kPolyPairsPer8) {
+                            e0 = ex2_poly(x0);
+                            e1 = ex2_poly(x1);
+                        } else {
+                            e0 = ex2(x0);
+                            e1 = ex2(x1);
+                        }
+                        acc[j & 7] += e0 + e1;
+                        pk[jj] = pack_bf16x2(e0, e1);
+                    }
                 }
-                tmem_st16(s_addr + ch * 16, pk);
+                tmem_st32(s_addr + half * 32, pk);
             }
+            l += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&p_full[t]);
@@ -308,6 +347,7 @@ __global__ void __launch_bounds__(320, 1)
             __nv_bfloat16 *orow = p.o + b * p.osb + static_cast<int64_t>(qb * 128 + row) * p.oss + h * p.osh;
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t r[32];
                 tmem_ld32(o_addr + ch * 32, r);
                 uint32_t w[16];
 #pragma unroll

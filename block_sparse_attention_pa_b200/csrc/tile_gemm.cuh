@@ -231,21 +231,28 @@ __global__ void __launch_bounds__(192, 1)
                 if (!warp_wait(&acc_full[acc], (tile >> 1) & 1, wc)) { ok = false; break; }
                 tc_fence_after();
                 const bool diag = (kb == un.qb);
-                const uint32_t taddr = lane_base + acc * 128;
-                float mx = -INFINITY;
-                uint32_t r[32];
+                uint32_t r[128];
+                tmem_ld128(lane_base + acc * 128, r);
+                // the accumulator row is in registers: hand TMEM back to the MMA warp
+                tc_fence_before();
+                mbar_arrive(&acc_empty[acc]);
+                if (diag) {
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    tmem_ld32(taddr + ch * 32, r);
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float v = __uint_as_float(r[j]);
-                        if (!diag || ch * 32 + j <= row) mx = fmaxf(mx, v);
-                    }
+                    for (int j = 0; j < 128; ++j)
+                        if (j > row) r[j] = 0xFF800000u;  // -inf above the diagonal (j > i)
                 }
+                float m8[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const uint32_t *v = r + 8 * j;
+                    m8[j] = fmax3(fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2])),
+                                  fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5])),
+                                  fmaxf(__uint_as_float(v[6]), __uint_as_float(v[7])));
+                }
+                const float mx =
+                    fmax3(fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmax3(m8[6], m8[7], m8[8])),
+                          fmax3(m8[9], m8[10], m8[11]), fmax3(m8[12], m8[13], fmaxf(m8[14], m8[15])));
                 if (MODE == MODE_SCORES) {
-                    tc_fence_before();
-                    mbar_arrive(&acc_empty[acc]);
                     float w = mx * p.scale;
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) w = fmaxf(w, __shfl_xor_sync(0xffffffffu, w, o));
@@ -265,18 +272,12 @@ __global__ void __launch_bounds__(192, 1)
                 } else {
                     // log2-domain row max and sum of exp2 over the valid entries
                     const float m = mx * p.scale;
-                    float l = 0.0f;
+                    float acc8[8];
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        tmem_ld32(taddr + ch * 32, r);
+                    for (int j = 0; j < 8; ++j) acc8[j] = 0.0f;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float e = ex2(fmaf(__uint_as_float(r[j]), p.scale, -m));
-                            if (!diag || ch * 32 + j <= row) l += e;
-                        }
-                    }
-                    tc_fence_before();
-                    mbar_arrive(&acc_empty[acc]);
+                    for (int j = 0; j < 128; ++j) acc8[j & 7] += ex2(fmaf(__uint_as_float(r[j]), p.scale, -m));
+                    const float l = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) + ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
                     const long long idx =
                         ((static_cast<long long>(un.b) * p.H + un.bh_head) * p.nb + kb) * 128 + row;
                     p.partial[idx] = make_float2(m, l);
