@@ -31,7 +31,7 @@ STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_E
 # Every entry point declared in include/pa.h.
 ENTRY_POINTS = ("pa_workspace_size", "pa_pool_heads", "pa_block_scores", "pa_build_mask",
                 "pa_block_sparse_attn", "pa_prefill", "pa_get_device_status", "pa_status_string",
-                "pa_last_error", "pa_abi_version")
+                "pa_last_error", "pa_abi_version", "pa_build_mask_noalloc")
 
 
 class PaError(RuntimeError):

@@ -486,3 +486,66 @@ pa_status pa_get_device_status(pa_stream_t stream, int clear) {
 }
 
 }  // extern "C"
+
+// ======================================================== no-allocation mask
+// pa_build_mask_noalloc keeps its scratch (the per-tile softmax statistics of
+// the last query block) in this file-scope device array instead of a
+// caller-provided workspace.  Every GPU that loads the library holds these
+// bytes until the process exits; every call on a device shares them.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+
+// Device address of g_noalloc_scratch on the current device.  The host-side
+// name of the array is only a stand-in, so the address is looked up once per
+// device with cudaGetSymbolAddress (with that device current) and cached.
+pa_status noalloc_scratch(void **out) {
+    static std::mutex mu;
+    static void *addr[kMaxDevices] = {};
+    int dev = 0;
+    PA_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return fail(PA_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(PA_ERR_CUDA, "cudaGetSymbolAddress(scratch) failed: %s", cudaGetErrorString(e));
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return PA_OK;
+}
+
+}  // namespace
+
+extern "C" PA_API pa_status pa_build_mask_noalloc(const pa_shape *shape, const pa_budget *budget,
+                                                  const float *scores, const void *q, pa_strides qs,
+                                                  const void *k, pa_strides ks, const pa_mask *out,
+                                                  pa_stream_t stream) {
+    pa_status r;
+    if ((r = check_shape(shape)) || (r = check_budget(budget))) return r;
+    if ((r = check_ptr(scores, "scores", 4))) return r;
+    if ((r = check_mask(out, budget, true))) return r;
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (budget->mode == PA_BUDGET_DYNAMIC) {
+        if ((r = check_tensor(q, qs, "q")) || (r = check_tensor(k, ks, "k"))) return r;
+        const size_t need = mask_ws_bytes(shape, budget);
+        if (need > kNoAllocScratchBytes)
+            return fail(PA_ERR_UNSUPPORTED,
+                        "pa_build_mask_noalloc: this shape needs %zu bytes of scratch but the built-in scratch holds "
+                        "%zu (batch * q_heads * seqlen/128 must be <= %zu); use pa_build_mask with a workspace",
+                        need, kNoAllocScratchBytes, kNoAllocScratchBytes / (128 * sizeof(float2)));
+        void *scratch = nullptr;
+        if ((r = noalloc_scratch(&scratch))) return r;
+        // every byte of the scratch that is read is written first in this call: nothing to clear
+        if ((r = launch_mass(shape, q, qs, k, ks, static_cast<float2 *>(scratch), out->mass, st))) return r;
+    }
+    if ((r = launch_rank(shape, scores, out->rank, st))) return r;
+    if ((r = launch_budget(shape, budget, out->rank, out->mass, out->cnt, out->budget, st))) return r;
+    return ok();
+}

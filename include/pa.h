@@ -157,6 +157,29 @@ PA_API pa_status pa_build_mask(const pa_shape *shape, const pa_budget *budget,
                         const pa_mask *out, void *ws, size_t ws_bytes,
                         pa_stream_t stream);
 
+/* pa_build_mask without a workspace argument.  The paper has no counterpart:
+ * this entry point exists for callers that cannot hand the library any device
+ * scratch memory -- for example a plugin interface whose per-call hook
+ * receives no workspace pointer, or a runtime that reserved all device memory
+ * up front and does not let the libraries it hosts call cudaMalloc.
+ * Same arguments, results and errors as pa_build_mask, minus ws/ws_bytes.
+ * Its scratch is a 16 MiB array inside the library (device memory held by
+ * every GPU that loads libpa.so until the process exits), so DYNAMIC mode
+ * supports batch * num_q_heads * (seqlen/128) <= 16384 (e.g. 32 heads up to
+ * 64K tokens); larger shapes return PA_ERR_UNSUPPORTED with that limit in
+ * pa_last_error().  The other modes need no scratch.  The first call on each
+ * device looks up the array's device address (cudaGetSymbolAddress, with that
+ * device current); make that first call before any stream capture.  The call
+ * allocates nothing.  All calls on a device share the one array, so two calls
+ * whose kernels overlap on the GPU (different streams, no ordering between
+ * them) race on it; calls ordered on one stream are safe.  No contents carry
+ * over between calls: each call writes every scratch byte it reads. */
+PA_API pa_status pa_build_mask_noalloc(const pa_shape *shape, const pa_budget *budget,
+                                       const float *scores,
+                                       const void *q, pa_strides q_strides,
+                                       const void *k, pa_strides k_strides,
+                                       const pa_mask *out, pa_stream_t stream);
+
 /* The block-sparse mask "fed to FlashAttention" (ProxyAttn blog, end of
  * 4. ProxyAttn method; attention formula of "2. Background"): for every
  * (b, h, qb) with list L = rank[b][grp(h)][tri(qb) ..] and n = cnt[b][h][qb],
