@@ -234,6 +234,17 @@ def counters_for(kernel_key: str, source_files):
     return c
 
 
+def traffic_for(ctr, w, G, mode, gamma):
+    """DRAM bytes per launch from the committed capture, only for the exact
+    workload and budget it was taken on (traffic does not scale linearly)."""
+    if not ctr:
+        return None
+    same = (ctr.get("workload") == w.name and ctr.get("groups") == G and
+            ctr.get("mode") == {0: "dynamic", 1: "fixed", 2: "all"}[mode] and
+            (mode != 0 or abs(ctr.get("gamma", -1) - gamma) < 1e-9))
+    return float(ctr["dram_bytes"]) if same else None
+
+
 ATTN_SOURCES = ["block_sparse_attention_pa_b200/csrc/attn.cuh", "block_sparse_attention_pa_b200/csrc/sm100.cuh"]
 
 
@@ -373,9 +384,7 @@ def main():
     achieved = flops / (attn_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     ctr = counters_for("attn_kernel", ATTN_SOURCES)
-    traffic = None
-    if ctr and ctr.get("dram_bytes_per_visited_block"):
-        traffic = float(ctr["dram_bytes_per_visited_block"]) * visited
+    traffic = traffic_for(ctr, w, G, mode, gamma)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "traffic": traffic, "kernel": "attn_kernel<128> (block-sparse attention)",
                 "peak_kind": f"{peaks_kind} bf16 sustained (kernel timed inside back-to-back steps)",

@@ -41,6 +41,7 @@ constexpr int kPolyPairsPer8 = PA_POLY_PAIRS_PER8;
 struct AttnParams {
     int B, N, H, Hkv, G, nb;
     int num_units;             // head units per (b, qb)
+    int units_per_kv;          // max head units of one KV head (grid stride)
     const int32_t *rank;       // [B][G][T]
     const int32_t *cnt;        // [B][H][nb]
     float scale_log2;          // softmax_scale * log2(e)
@@ -50,13 +51,28 @@ struct AttnParams {
     uint64_t timeout_ns;
     int16_t unit_h0[kMaxHeads];
     int16_t unit_h1[kMaxHeads];  // -1: the unit has one head
+    int16_t kv_unit0[kMaxHeads];  // first unit of KV head kv (units are ordered by KV head)
+    int16_t kv_units[kMaxHeads];  // number of units of KV head kv
 };
+
+// Smallest block index >= from whose bit is set in (a | b), or -1; words
+// bitmap words are in range.
+__device__ __forceinline__ int next_block(const uint32_t *a, const uint32_t *b, int from, int words) {
+    int w = from >> 5;
+    if (w >= words) return -1;
+    uint32_t m = (a[w] | b[w]) & (0xFFFFFFFFu << (from & 31));
+    while (m == 0u) {
+        if (++w >= words) return -1;
+        m = a[w] | b[w];
+    }
+    return (w << 5) + __ffs(static_cast<int>(m)) - 1;
+}
 
 template <int D>
 struct AttnSmem {
     static constexpr int TB = 128 * D * 2;
     static constexpr int KS = (D == 128) ? 2 : 4;
-    static constexpr int BYTES = (2 + 2 * KS) * TB + 1024 + 512;
+    static constexpr int BYTES = (2 + 2 * KS) * TB + 1024 + 512 + 1024;  // + two 4096-bit block bitmaps
 };
 
 template <int D>
@@ -86,13 +102,21 @@ __global__ void __launch_bounds__(320, 1)
     uint64_t *v_empty = bars + 8 + 3 * KS;   // KS
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8 + 4 * KS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    uint32_t *bm = reinterpret_cast<uint32_t *>(smem + (2 + 2 * KS) * TB + 512);  // [2][128] block bitmaps
 
     // ------------------------------------------------------------ work item
-    const int P = p.num_units;
-    const int unit = static_cast<int>(blockIdx.x % P);
-    const int bq = static_cast<int>(blockIdx.x / P);
-    const int b = bq % p.B;
-    const int qb = p.nb - 1 - bq / p.B;  // heaviest query blocks first
+    // Grid order: (batch, KV head) outermost, then query blocks from the
+    // longest down, then the head units of that KV head.  The CTAs resident at
+    // one time therefore share one KV head, whose K/V then stays in L2.
+    const int U = p.units_per_kv;
+    const int j = static_cast<int>(blockIdx.x % U);
+    long long rest = blockIdx.x / U;
+    const int qb = p.nb - 1 - static_cast<int>(rest % p.nb);
+    rest /= p.nb;
+    const int kv_of_cta = static_cast<int>(rest % p.Hkv);
+    const int b = static_cast<int>(rest / p.Hkv);
+    if (j >= p.kv_units[kv_of_cta]) return;  // this KV head has fewer units (whole CTA, before any sync)
+    const int unit = p.kv_unit0[kv_of_cta] + j;
     const int h0 = p.unit_h0[unit];
     const int h1 = p.unit_h1[unit];
     const int g = static_cast<int>(static_cast<long long>(h0) * p.G / p.H);
@@ -107,6 +131,24 @@ __global__ void __launch_bounds__(320, 1)
     for (int t = 0; t < 2; ++t) c[t] = min(max(craw[t], 0), qb + 1);
     const int n = max(c[0], c[1]);
     const int ntiles = (h1 >= 0) ? 2 : 1;
+    const int words = (qb + 32) >> 5;  // bitmap words covering blocks 0..qb
+
+    // The selected blocks of each head as a bitmap over 0..qb: head t takes the
+    // first c[t] entries of the list.  Every role then visits them in
+    // ascending block order (the result does not depend on the order), so the
+    // CTAs resident at one time sweep K/V in step.
+    for (int w = threadIdx.x; w < 256; w += blockDim.x) bm[w] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int kb = list[i];
+        if (kb < 0 || kb > qb) {
+            flag_status(kStBounds);
+            continue;
+        }
+        const uint32_t bit = 1u << (kb & 31);
+        if (i < c[0]) atomicOr(&bm[kb >> 5], bit);
+        if (i < c[1]) atomicOr(&bm[128 + (kb >> 5)], bit);
+    }
 
     const uint32_t warp = warp_id(), lane = lane_id();
     if (threadIdx.x == 0) {
@@ -152,12 +194,9 @@ __global__ void __launch_bounds__(320, 1)
                 if (h1 >= 0) tma_load_4d(sQ + TB + cc * 16384, &tmQ, q_full, cc * 64, h1, qb * 128, b);
             }
             int issued = 0;
-            for (int i = 0; i < n; ++i) {
-                int kb = list[i];
-                if (kb < 0 || kb > qb) {
-                    flag_status(kStBounds);
-                    kb = qb;  // the softmax masks this tile out entirely
-                }
+            int i = 0;
+            for (int kb = next_block(bm, bm + 128, 0, words); kb >= 0;
+                 kb = next_block(bm, bm + 128, kb + 1, words), ++i) {
                 const int s = i % KS;
                 const uint32_t ph = ((i / KS) - 1) & 1;
                 if (i >= KS && !mbar_wait(&k_empty[s], ph, wc)) break;
@@ -184,7 +223,8 @@ __global__ void __launch_bounds__(320, 1)
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
-        if (lane == 0 && n > 0) {
+        const int kb_first = next_block(bm, bm + 128, 0, words);
+        if (lane == 0 && kb_first >= 0) {
             const uint32_t qa[2] = {smem_u32(sQ), smem_u32(sQ + TB)};
             auto issue_qk = [&](int t, int s) {
                 const uint32_t kbase = smem_u32(sK + s * TB);
@@ -204,31 +244,37 @@ __global__ void __launch_bounds__(320, 1)
                             IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
                 umma_commit(&o_done[t]);
             };
+            auto active = [&](int t, int kb) { return (bm[t * 128 + (kb >> 5)] >> (kb & 31)) & 1u; };
+            int pv_done[2] = {0, 0};
             bool ok = mbar_wait(q_full, 0, wc) && mbar_wait(&k_full[0], 0, wc);
             if (ok) {
                 tc_fence_after();
                 for (int t = 0; t < 2; ++t)
-                    if (c[t] > 0) issue_qk(t, 0);
+                    if (active(t, kb_first)) issue_qk(t, 0);
                 umma_commit(&k_empty[0]);
             }
-            for (int i = 0; i < n && ok; ++i) {
+            int i = 0;
+            for (int kb = kb_first; kb >= 0 && ok; ++i) {
                 const int s = i % KS;
                 const int s1 = (i + 1) % KS;
-                const bool has_next = i + 1 < n;
+                const int kb_next = next_block(bm, bm + 128, kb + 1, words);
+                const bool has_next = kb_next >= 0;
                 if (!mbar_wait(&v_full[s], (i / KS) & 1, wc)) break;
                 if (has_next && !mbar_wait(&k_full[s1], ((i + 1) / KS) & 1, wc)) break;
                 tc_fence_after();
                 for (int t = 0; t < 2; ++t) {
-                    if (i < c[t]) {
-                        if (!mbar_wait(&p_full[t], i & 1, wc)) { ok = false; break; }
+                    if (active(t, kb)) {
+                        if (!mbar_wait(&p_full[t], pv_done[t] & 1, wc)) { ok = false; break; }
                         tc_fence_after();
-                        issue_pv(t, s, i > 0);
+                        issue_pv(t, s, pv_done[t] > 0);
+                        ++pv_done[t];
                     }
-                    if (i + 1 < c[t]) issue_qk(t, s1);
+                    if (has_next && active(t, kb_next)) issue_qk(t, s1);
                 }
                 if (!ok) break;
                 umma_commit(&v_empty[s]);
                 if (has_next) umma_commit(&k_empty[s1]);
+                kb = kb_next;
             }
         }
         if (lane == 0) {
@@ -239,8 +285,8 @@ __global__ void __launch_bounds__(320, 1)
     } else {
         // ---------------------------------------------------------- softmax
         const int t = (warp >= 6) ? 1 : 0;
-        const int ct = c[t];
         const int h = t ? h1 : h0;
+        const uint32_t *bmt = bm + t * 128;
         const int q4 = static_cast<int>(warp & 3);
         const int row = q4 * 32 + static_cast<int>(lane);
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
@@ -249,17 +295,16 @@ __global__ void __launch_bounds__(320, 1)
         float m = -INFINITY, l = 0.0f;
         bool ok = true;
         uint32_t s[128];
-        for (int i = 0; i < ct; ++i) {
+        int i = 0;  // tiles of this head so far
+        for (int kb = next_block(bmt, bmt, 0, words); kb >= 0; kb = next_block(bmt, bmt, kb + 1, words), ++i) {
             if (!warp_wait(&s_full[t], i & 1, wc)) { ok = false; break; }
             tc_fence_after();
-            const int kb = list[i];
-            const bool valid = (kb >= 0 && kb <= qb);
-            const bool masked = (kb == qb) || !valid;  // warp-uniform: same tile for the whole CTA
+            const bool masked = (kb == qb);  // the diagonal tile: same for the whole CTA
             tmem_ld128(s_addr, s);
             if (masked) {
 #pragma unroll
                 for (int j = 0; j < 128; ++j)
-                    if (!valid || j > row) s[j] = 0xFF800000u;  // -inf: causal mask of the diagonal tile
+                    if (j > row) s[j] = 0xFF800000u;  // -inf: causal mask of the diagonal tile
             }
             // row max of the tile: a tree of three-input maxima
             float mx[16];
@@ -341,6 +386,7 @@ __global__ void __launch_bounds__(320, 1)
             mbar_arrive(&p_full[t]);
         }
         // epilogue: O / l -> bf16 -> global; LSE
+        const int ct = i;
         if (ct > 0 && ok && warp_wait(&o_done[t], (ct - 1) & 1, wc)) {
             tc_fence_after();
             const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;

@@ -315,7 +315,7 @@ pa_status launch_attn_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUte
     auto kern = pa::attn_kernel<D>;
     const int smem = pa::AttnSmem<D>::BYTES;
     PA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-    const long long grid = static_cast<long long>(p.num_units) * p.B * p.nb;
+    const long long grid = static_cast<long long>(p.units_per_kv) * p.Hkv * p.B * p.nb;
     kern<<<static_cast<unsigned>(grid), 320, smem, st>>>(mq, mk, mv, p);
     PA_CUDA(cudaGetLastError());
     return PA_OK;
@@ -333,6 +333,15 @@ pa_status launch_attn(const pa_shape *s, const void *q, pa_strides qs, const voi
     pa::AttnParams p{};
     p.B = B; p.N = N; p.H = H; p.Hkv = Hkv; p.G = s->num_groups; p.nb = N / kBlk;
     p.num_units = build_units(s, p.unit_h0, p.unit_h1);
+    // units are produced in ascending head order, hence grouped by KV head
+    for (int kv = 0; kv < Hkv; ++kv) p.kv_units[kv] = 0;
+    for (int u = 0; u < p.num_units; ++u) {
+        const int kv = static_cast<int>(static_cast<long long>(p.unit_h0[u]) * Hkv / H);
+        if (p.kv_units[kv] == 0) p.kv_unit0[kv] = static_cast<int16_t>(u);
+        ++p.kv_units[kv];
+    }
+    p.units_per_kv = 0;
+    for (int kv = 0; kv < Hkv; ++kv) p.units_per_kv = std::max<int>(p.units_per_kv, p.kv_units[kv]);
     p.rank = rank; p.cnt = cnt;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.o = static_cast<__nv_bfloat16 *>(o);
