@@ -194,6 +194,22 @@ class Pipeline:
         return v, v * per, exact
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The max of a per-rank time over all ranks (the job's time); the value
+    itself without a process group."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def per_layer(ms_step: float, world: int) -> float:
+    """Replicas: every rank runs one layer per step, so the job processes
+    `world` layers in the (max-over-ranks) step time."""
+    return ms_step / world
+
+
 def time_pipeline(pipe, steps, warmup, dist_on, sampler=None):
     for _ in range(warmup):
         pipe.step()
@@ -368,10 +384,7 @@ def main():
     status = pa.device_status()
     if status != 0:
         raise SystemExit(f"device status {status} after the timed run")
-    t = torch.tensor([total_ms], device=q.device, dtype=torch.float64)
-    if dist_on:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, q.device)
     ms_step = total_ms / args.steps
     visited, flops, flops_exact = pipe.visited()
     B, H, nb = w.batch, w.num_q_heads, pipe.nb
@@ -404,7 +417,7 @@ def main():
         "attn": {"ms": attn_ms, "TFLOP/s": achieved, "frac_tensor": achieved / peak},
     }
 
-    line = {"metric": METRIC, "value": ms_step / world, "unit": "ms/layer", "n_gpus": world, "steps": args.steps,
+    line = {"metric": METRIC, "value": per_layer(ms_step, world), "unit": "ms/layer", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded needle/sink generator; random inputs, no weights)",
@@ -479,14 +492,11 @@ def run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world):
         one()
     e.record()
     torch.cuda.synchronize()
-    t = torch.tensor([s.elapsed_time(e)], device=q.device, dtype=torch.float64)
-    if dist_on:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms = float(t.item()) / steps
+    ms = max_over_ranks(s.elapsed_time(e), q.device) / steps
     if pa.device_status() != 0:
         raise SystemExit("device status flagged in the end-to-end run")
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
-    return {"value": ms / world, "unit": "ms/layer", "h2d_bytes_per_step": h2d,
+    return {"value": per_layer(ms, world), "unit": "ms/layer", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": ho.numel() * ho.element_size(), "steps": steps}
 
 

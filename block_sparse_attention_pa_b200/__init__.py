@@ -31,7 +31,7 @@ STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_E
 # Every entry point declared in include/pa.h.
 ENTRY_POINTS = ("pa_workspace_size", "pa_pool_heads", "pa_block_scores", "pa_build_mask",
                 "pa_block_sparse_attn", "pa_prefill", "pa_get_device_status", "pa_status_string",
-                "pa_last_error", "pa_abi_version", "pa_build_mask_noalloc")
+                "pa_last_error", "pa_abi_version", "pa_build_mask_noalloc", "pa_selftest_wait_timeout")
 
 
 class PaError(RuntimeError):
@@ -81,12 +81,13 @@ def lib() -> ctypes.CDLL:
         L.pa_prefill.argtypes = [P(Shape), P(Budget), vp, st, vp, st, vp, st, vp, st, P(MaskBufs), vp,
                                  ctypes.c_size_t, vp]
         L.pa_get_device_status.argtypes = [vp, ctypes.c_int]
+        L.pa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp]
         L.pa_status_string.restype = ctypes.c_char_p
         L.pa_status_string.argtypes = [ctypes.c_int]
         L.pa_last_error.restype = ctypes.c_char_p
         L.pa_abi_version.restype = ctypes.c_int32
         for name in ("pa_pool_heads", "pa_block_scores", "pa_build_mask", "pa_block_sparse_attn", "pa_prefill",
-                     "pa_get_device_status"):
+                     "pa_get_device_status", "pa_selftest_wait_timeout"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -243,3 +244,8 @@ def prefill(q, k, v, num_groups: int, mode: int = DYNAMIC, gamma: float = 0.95, 
 def device_status(clear: bool = True, device=None) -> int:
     """pa_get_device_status: syncs the current stream; 0 if no kernel recorded a problem."""
     return int(lib().pa_get_device_status(_stream(device), 1 if clear else 0))
+
+
+def selftest_wait_timeout(timeout_us: int = 1000, device=None) -> None:
+    """pa_selftest_wait_timeout: a bounded device wait that is made to run out."""
+    _check(lib().pa_selftest_wait_timeout(int(timeout_us), _stream(device)))

@@ -7,18 +7,20 @@
 // head t visits its first cnt_t entries, so a K/V tile is loaded once for
 // both heads while both still need it.
 //
-// Warp roles (320 threads, one CTA per SM, all 512 TMEM columns):
-//   warp 0     TMA producer: the two Q tiles once, then K and V tiles of the
+// Warp roles (384 threads = three warpgroups, one CTA per SM, all 512 TMEM
+// columns).  At the start the third warpgroup hands registers to the two
+// softmax warpgroups (setmaxnreg: 2 x 128 x 208 + 128 x 88 = 384 x 168):
+//   warps 0-3  softmax of head 0, warps 4-7 softmax of head 1 (below)
+//   warp 8     TMA producer: the two Q tiles once, then K and V tiles of the
 //              listed blocks into a ring (128-byte swizzle).
-//   warp 1     TMEM owner and single-thread tcgen05.mma issuer:
+//   warp 9     TMEM owner and single-thread tcgen05.mma issuer:
 //                S_t = Q_t K^T   (M=128, N=128, K=16 steps; A, B K-major smem)
 //                O_t += P_t V    (M=128, N=d,   A = P_t read from TMEM,
 //                                 B = V, MN-major smem)
 //              in ping-pong order  PV_0(i), QK_0(i+1), PV_1(i), QK_1(i+1), so
 //              the tensor core computes one head's products while the other
 //              head's softmax runs.
-//   warps 2-5  softmax of head 0, warps 6-9 softmax of head 1: one thread per
-//              query row (TMEM lane).  Two passes over S in TMEM (row max,
+//   softmax    one thread per query row (TMEM lane).  Two passes over S in TMEM (row max,
 //              then exp2/row sum/bf16 pack of P written back over S), online
 //              softmax with the running max raised only when it grows by more
 //              than 2^8 (then O is rescaled in TMEM), final O/l and LSE.
@@ -30,6 +32,16 @@
 namespace pa {
 
 constexpr int kMaxHeads = 128;
+
+// 12 warps: 0-7 softmax (two warpgroups), 8 producer, 9 MMA, 10-11 idle.
+constexpr int kAttnThreads = 384;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kRegsLaunch = 168;   // 65536 / 384, rounded down to a multiple of 8
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsAux = 88;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsAux <= kAttnThreads * kRegsLaunch,
+              "setmaxnreg split exceeds the registers the CTA is launched with");
 
 // Of every 8 column pairs of a non-diagonal S tile, this many take their
 // exponentials from the FMA-pipe polynomial instead of the MUFU unit.
@@ -76,7 +88,7 @@ struct AttnSmem {
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
     using SM = AttnSmem<D>;
@@ -169,12 +181,12 @@ __global__ void __launch_bounds__(320, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) {
+    if (warp == kProducerWarp && lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
@@ -184,7 +196,11 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t tmem = *tmem_slot;
     const WaitCtl wc{abort_flag, p.timeout_ns};
 
-    if (warp == 0) {
+    if (warp >= 8) {
+      // warpgroup 2 (producer, MMA issuer, two idle warps) hands registers to
+      // the softmax warpgroups; the branch is uniform per warpgroup
+      reg_release<kRegsAux>();
+      if (warp == kProducerWarp) {
         // ---------------------------------------------------------- producer
         if (lane == 0) {
             mbar_arrive_expect_tx(q_full, ntiles * TB);
@@ -221,31 +237,37 @@ __global__ void __launch_bounds__(320, 1)
             for (int i = max(nk - KS, 0); i < nk; ++i) mbar_wait_drain(&k_full[i % KS], (i / KS) & 1, p.timeout_ns);
             for (int i = max(nv - KS, 0); i < nv; ++i) mbar_wait_drain(&v_full[i % KS], (i / KS) & 1, p.timeout_ns);
         }
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------- MMA issuer
         const int kb_first = next_block(bm, bm + 128, 0, words);
         if (lane == 0 && kb_first >= 0) {
-            const uint32_t qa[2] = {smem_u32(sQ), smem_u32(sQ + TB)};
+            // smem descriptors precomputed once; a K step only moves the start
+            // address (+32 B within a 128-byte swizzle row, +16 KB per 64-column
+            // chunk; +2 KB per 16 keys of V)
+            const uint64_t dq[2] = {sdesc_sw128(smem_u32(sQ), 16, 1024), sdesc_sw128(smem_u32(sQ + TB), 16, 1024)};
+            const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+            const uint64_t dv0 = sdesc_sw128(smem_u32(sV), 16384, 1024);
             auto issue_qk = [&](int t, int s) {
-                const uint32_t kbase = smem_u32(sK + s * TB);
+                const uint64_t a = t ? dq[1] : dq[0];
+                const uint64_t bk = dk0 + static_cast<uint64_t>((s * TB) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    umma_ss(tmem + t * 128, sdesc_sw128(qa[t] + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024),
-                            IDESC_QK, kk > 0 ? 1u : 0u);
+                    const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+                    umma_ss(tmem + t * 128, a + off, bk + off, IDESC_QK, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&s_full[t]);
             };
             auto issue_pv = [&](int t, int s, bool accumulate) {
-                const uint32_t vbase = smem_u32(sV + s * TB);
+                const uint64_t bv = dv0 + static_cast<uint64_t>((s * TB) >> 4);
+                const uint32_t acc0 = accumulate ? 1u : 0u;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)  // 128 keys, 16 per step
-                    umma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, sdesc_sw128(vbase + kk * 2048, 16384, 1024),
-                            IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
+                    umma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, bv + static_cast<uint64_t>(kk * 128),
+                            IDESC_PV, kk > 0 ? 1u : acc0);
                 umma_commit(&o_done[t]);
             };
             auto active = [&](int t, int kb) { return (bm[t * 128 + (kb >> 5)] >> (kb & 31)) & 1u; };
-            int pv_done[2] = {0, 0};
+            int pv_done0 = 0, pv_done1 = 0;
             bool ok = mbar_wait(q_full, 0, wc) && mbar_wait(&k_full[0], 0, wc);
             if (ok) {
                 tc_fence_after();
@@ -264,10 +286,11 @@ __global__ void __launch_bounds__(320, 1)
                 tc_fence_after();
                 for (int t = 0; t < 2; ++t) {
                     if (active(t, kb)) {
-                        if (!mbar_wait(&p_full[t], pv_done[t] & 1, wc)) { ok = false; break; }
+                        int &pv_done = t ? pv_done1 : pv_done0;
+                        if (!mbar_wait(&p_full[t], pv_done & 1, wc)) { ok = false; break; }
                         tc_fence_after();
-                        issue_pv(t, s, pv_done[t] > 0);
-                        ++pv_done[t];
+                        issue_pv(t, s, pv_done > 0);
+                        ++pv_done;
                     }
                     if (has_next && active(t, kb_next)) issue_qk(t, s1);
                 }
@@ -282,9 +305,11 @@ __global__ void __launch_bounds__(320, 1)
             mbar_wait_drain(drain, 0, p.timeout_ns);
         }
         __syncwarp();
+      }
     } else {
+        reg_acquire<kRegsSoftmax>();
         // ---------------------------------------------------------- softmax
-        const int t = (warp >= 6) ? 1 : 0;
+        const int t = static_cast<int>(warp >> 2);
         const int h = t ? h1 : h0;
         const uint32_t *bmt = bm + t * 128;
         const int q4 = static_cast<int>(warp & 3);
@@ -415,7 +440,7 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, 512);
+    if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace pa

@@ -315,8 +315,15 @@ pa_status launch_attn_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUte
     auto kern = pa::attn_kernel<D>;
     const int smem = pa::AttnSmem<D>::BYTES;
     PA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    // The kernel's warpgroups re-split the registers it is launched with; the
+    // split only adds up if every thread starts with kRegsLaunch registers.
+    cudaFuncAttributes fa;
+    PA_CUDA(cudaFuncGetAttributes(&fa, kern));
+    if (fa.numRegs != pa::kRegsLaunch)
+        return fail(PA_ERR_CUDA, "attn_kernel built with %d registers per thread, expected %d", fa.numRegs,
+                    pa::kRegsLaunch);
     const long long grid = static_cast<long long>(p.units_per_kv) * p.Hkv * p.B * p.nb;
-    kern<<<static_cast<unsigned>(grid), 320, smem, st>>>(mq, mk, mv, p);
+    kern<<<static_cast<unsigned>(grid), pa::kAttnThreads, smem, st>>>(mq, mk, mv, p);
     PA_CUDA(cudaGetLastError());
     return PA_OK;
 }
@@ -556,5 +563,32 @@ extern "C" PA_API pa_status pa_build_mask_noalloc(const pa_shape *shape, const p
     }
     if ((r = launch_rank(shape, scores, out->rank, st))) return r;
     if ((r = launch_budget(shape, budget, out->rank, out->mass, out->cnt, out->budget, st))) return r;
+    return ok();
+}
+
+// ========================================================== wait self-test
+namespace pa {
+// One warp waits on an mbarrier that nothing ever completes; the bounded wait
+// gives up after timeout_ns, records PA_ERR_TIMEOUT and the kernel returns.
+__global__ void selftest_wait_timeout_kernel(uint64_t timeout_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const WaitCtl wc{&abort_flag, timeout_ns};
+    (void)warp_wait(&bar, 0, wc);
+}
+}  // namespace pa
+
+extern "C" PA_API pa_status pa_selftest_wait_timeout(uint32_t timeout_us, pa_stream_t stream) {
+    if (timeout_us < 1 || timeout_us > 1000000)
+        return fail(PA_ERR_INVALID_ARG, "timeout_us must be in 1..1000000 (got %u)", timeout_us);
+    pa::selftest_wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint64_t>(timeout_us) * 1000u);
+    PA_CUDA(cudaGetLastError());
     return ok();
 }

@@ -32,12 +32,18 @@ __device__ __forceinline__ void add_bf16x8(double (&acc)[8], const uint4 &v) {
     }
 }
 
+// sum / n rounded to bf16.  When n is a power of two, sum * (1/n) is exact and
+// therefore the same IEEE result as the (slow) fp64 division.
 __device__ __forceinline__ uint4 mean_to_bf16x8(const double (&acc)[8], int n) {
+    const bool pow2 = (n & (n - 1)) == 0;
+    const double inv = 1.0 / static_cast<double>(n);
     uint32_t w[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat16 lo = __double2bfloat16(acc[2 * i] / n);
-        const __nv_bfloat16 hi = __double2bfloat16(acc[2 * i + 1] / n);
+        const double m0 = pow2 ? acc[2 * i] * inv : acc[2 * i] / n;
+        const double m1 = pow2 ? acc[2 * i + 1] * inv : acc[2 * i + 1] / n;
+        const __nv_bfloat16 lo = __double2bfloat16(m0);
+        const __nv_bfloat16 hi = __double2bfloat16(m1);
         w[i] = static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
                (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
     }
@@ -45,7 +51,7 @@ __device__ __forceinline__ uint4 mean_to_bf16x8(const double (&acc)[8], int n) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(256) pool_heads_kernel(PoolParams p) {
+__global__ void __launch_bounds__(256, 2) pool_heads_kernel(PoolParams p) {
     constexpr int TPR = D / 8;  // threads per (token, group) row
     const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t rows = static_cast<int64_t>(p.B) * p.N * p.G;
@@ -66,25 +72,25 @@ __global__ void __launch_bounds__(256) pool_heads_kernel(PoolParams p) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) aq[j] = ak[j] = 0.0;
 
-    int last_kv = -1;
-    uint4 kv_raw = make_uint4(0, 0, 0, 0);
-    for (int t0 = 0; t0 < hpg; t0 += 8) {
-        const int n = min(8, hpg - t0);
-        uint4 qv[8];
+    // all 16-byte loads of a block of 6 heads are in flight before the first
+    // add; the adds then run in ascending head order (the oracle's order)
+    for (int t0 = 0; t0 < hpg; t0 += 6) {
+        const int n = min(6, hpg - t0);
+        uint4 qv[6], kvv[6];
 #pragma unroll
-        for (int t = 0; t < 8; ++t)
-            if (t < n) qv[t] = __ldg(reinterpret_cast<const uint4 *>(qrow + (h0 + t0 + t) * p.qsh));
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
+        for (int t = 0; t < 6; ++t) {
             if (t < n) {
                 const int h = h0 + t0 + t;
-                add_bf16x8(aq, qv[t]);
                 const int kvh = static_cast<int>(static_cast<int64_t>(h) * p.Hkv / p.H);
-                if (kvh != last_kv) {
-                    kv_raw = __ldg(reinterpret_cast<const uint4 *>(krow + kvh * p.ksh));
-                    last_kv = kvh;
-                }
-                add_bf16x8(ak, kv_raw);
+                qv[t] = __ldg(reinterpret_cast<const uint4 *>(qrow + h * p.qsh));
+                kvv[t] = __ldg(reinterpret_cast<const uint4 *>(krow + kvh * p.ksh));
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < 6; ++t) {
+            if (t < n) {
+                add_bf16x8(aq, qv[t]);
+                add_bf16x8(ak, kvv[t]);
             }
         }
     }

@@ -218,6 +218,15 @@ PA_API pa_status pa_prefill(const pa_shape *shape, const pa_budget *budget,
  * The word is shared by every stream of the device. */
 PA_API pa_status pa_get_device_status(pa_stream_t stream, int clear);
 
+/* Diagnostic for failure detection, with no counterpart on the pages: launches
+ * one warp that waits on a device barrier nothing ever completes, bounded by
+ * timeout_us (1..1000000).  The wait gives up, records PA_ERR_TIMEOUT in the
+ * device status word and the kernel returns normally -- the same path every
+ * bounded wait in the other kernels takes -- so a caller can check that a
+ * timed-out wait is reported (pa_get_device_status) and leaves the context
+ * usable, without faulting or hanging the GPU. */
+PA_API pa_status pa_selftest_wait_timeout(uint32_t timeout_us, pa_stream_t stream);
+
 /* Static description of a status code. */
 PA_API const char *pa_status_string(pa_status status);
 

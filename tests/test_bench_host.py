@@ -1,0 +1,56 @@
+"""The benchmark's multi-rank host logic on CPU (gloo, world size 2): the job
+time is the max over ranks and `value` counts every rank's layer; the
+reference arm prints only on rank 0."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        t = bench.max_over_ranks(10.0 + 5.0 * rank, torch.device("cpu"))
+        dist.barrier()
+        out[rank] = t
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2():
+    port = 29500 + os.getpid() % 1000
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
+        assert out[0] == out[1] == 15.0
+
+
+def test_single_process_and_per_layer():
+    assert bench.max_over_ranks(3.5, torch.device("cpu")) == 3.5
+    assert bench.per_layer(100.0, 4) == 25.0
+
+
+@pytest.mark.parametrize("rank,expect_line", [(0, True), (1, False)])
+def test_reference_arm_prints_on_rank0_only(rank, expect_line):
+    env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank))
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                        "tiny_gqa_n1024", "--steps", "1", "--warmup", "0", "--gpus", "2"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    if expect_line:
+        d = json.loads(lines[-1])
+        assert d["impl"] == "reference" and d["unit"] == "ms/layer" and d["e2e"]["h2d_bytes_per_step"] == 0
+        assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    else:
+        assert lines == []
