@@ -13,9 +13,11 @@
 //
 // Persistent, warp-specialised CTA (one per SM, 192 threads):
 //   warp 0     TMA producer: the unit's A tile (double-buffered) and a ring of
-//              B tiles, 128 rows x d, 128-byte swizzle.
-//   warp 1     allocates 256 TMEM columns (two fp32 128x128 accumulators) and
-//              issues tcgen05.mma (M=128, N=128, K=16) from one thread.
+//              B stages of two 128-row key tiles, 128-byte swizzle.
+//   warp 1     allocates 512 TMEM columns (two fp32 128x256 accumulators) and
+//              issues tcgen05.mma (M=128, N=256, K=16: two key tiles per
+//              instruction, so each wait of the issuing thread covers twice
+//              the tensor work) from one thread.
 //   warps 2-5  epilogue: each thread owns one accumulator row (TMEM lane),
 //              reads it with tcgen05.ld and reduces it.
 // A unit is a run of up to `chunk` consecutive tiles sharing one A tile.
@@ -78,12 +80,20 @@ __device__ __forceinline__ float ord2f(uint32_t o) {
     return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
 }
 
+// Shared memory: A (the unit's 128-row Q tile) double-buffered, then a ring
+// of B stages that each hold two consecutive 128-row K tiles as one 256-row
+// K-major operand (per 64-column chunk: 256 rows x 128 B, 128-byte swizzle).
 template <int D>
 struct TileSmem {
     static constexpr int TILE_BYTES = 128 * D * 2;
-    static constexpr int STAGES = (D == 128) ? 4 : 8;
-    static constexpr int BYTES = (2 + STAGES) * TILE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
+    static constexpr int PAIR_BYTES = 2 * TILE_BYTES;
+    static constexpr int STAGES = (D == 128) ? 2 : 4;
+    static constexpr int BYTES = 2 * TILE_BYTES + STAGES * PAIR_BYTES + 1024 /*align*/ + 512 /*barriers*/;
 };
+
+// Tiles of a unit are processed in pairs (kb, kb+1) with one N=256 MMA per K
+// step; a unit with an odd tile count ends with a single N=128 tile.
+__device__ __forceinline__ int pairs_of(const Unit &un) { return (un.kb1 - un.kb0 + 1) >> 1; }
 
 template <int D, int MODE>
 __global__ void __launch_bounds__(192, 1)
@@ -91,26 +101,28 @@ __global__ void __launch_bounds__(192, 1)
                      TileParams p) {
     using S = TileSmem<D>;
     constexpr int TB = S::TILE_BYTES;
+    constexpr int PB = S::PAIR_BYTES;
     constexpr int NST = S::STAGES;
     constexpr int KSTEPS = D / 16;
-    constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, false, false);
+    constexpr uint32_t IDESC256 = idesc_bf16_f32(128, 256, false, false);
+    constexpr uint32_t IDESC128 = idesc_bf16_f32(128, 128, false, false);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;                       // [2][TB]
-    uint8_t *sB = smem + 2 * TB;              // [NST][TB]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (2 + NST) * TB);
+    uint8_t *sB = smem + 2 * TB;              // [NST][PB]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 2 * TB + NST * PB);
     uint64_t *a_full = bars;                  // 2
     uint64_t *a_empty = bars + 2;             // 2
     uint64_t *acc_full = bars + 4;            // 2
     uint64_t *acc_empty = bars + 6;           // 2
-    uint64_t *b_full = bars + 8;              // NST
-    uint64_t *b_empty = bars + 8 + NST;       // NST
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8 + 2 * NST);
+    uint64_t *drain = bars + 8;               // 1
+    uint64_t *b_full = bars + 9;              // NST
+    uint64_t *b_empty = bars + 9 + NST;       // NST
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 9 + 2 * NST);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    uint32_t *red_max = tmem_slot + 2;        // [4]
-    uint32_t *red_cnt = tmem_slot + 6;        // [4]
-    uint64_t *drain = reinterpret_cast<uint64_t *>(tmem_slot + 10);  // 8-byte aligned: bars + 8 + 2*NST + 5
+    uint32_t *red_max = tmem_slot + 2;        // [8] per-tile cross-warp max (ring)
+    uint32_t *red_cnt = tmem_slot + 10;       // [8]
 
     const uint32_t warp = warp_id(), lane = lane_id();
     if (threadIdx.x == 0) {
@@ -124,7 +136,7 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(&b_full[i], 1);
             mbar_init(&b_empty[i], 1);
         }
-        for (int i = 0; i < 4; ++i) red_max[i] = red_cnt[i] = 0;
+        for (int i = 0; i < 8; ++i) red_max[i] = red_cnt[i] = 0;
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -134,7 +146,7 @@ __global__ void __launch_bounds__(192, 1)
         tma_prefetch_desc(&tmB);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, 512);  // two 128x256 fp32 accumulators
         tmem_relinquish();
     }
     tc_fence_before();
@@ -146,9 +158,10 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 0) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
-            long long tile = 0;
+            long long pair = 0;
             int local = 0;
-            for (long long u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
+            bool ok = true;
+            for (long long u = blockIdx.x; u < p.num_units && ok && !*abort_flag; u += gridDim.x) {
                 const Unit un = decode_unit(p, u, MODE);
                 const int a = local & 1;
                 if (local >= 2 && !mbar_wait(&a_empty[a], ((local >> 1) - 1) & 1, wc)) break;
@@ -163,24 +176,26 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 const int kvh = (MODE == MODE_MASS)
                                     ? static_cast<int>(static_cast<long long>(un.bh_head) * p.Hkv / p.H) : 0;
-                bool ok = true;
-                for (int kb = un.kb0; kb < un.kb1; ++kb, ++tile) {
-                    const int s = static_cast<int>(tile % NST);
-                    const long long n = tile / NST;
-                    if (tile >= NST && !mbar_wait(&b_empty[s], (n - 1) & 1, wc)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&b_full[s], TB);
+                for (int kb = un.kb0; kb < un.kb1; kb += 2, ++pair) {
+                    const int s = static_cast<int>(pair % NST);
+                    const int nt = min(2, un.kb1 - kb);
+                    if (pair >= NST && !mbar_wait(&b_empty[s], ((pair / NST) - 1) & 1, wc)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&b_full[s], nt * TB);
+                    for (int j = 0; j < nt; ++j) {
 #pragma unroll
-                    for (int cc = 0; cc < D / 64; ++cc) {
-                        if (MODE == MODE_SCORES)
-                            tma_load_4d(sB + s * TB + cc * 16384, &tmB, &b_full[s], cc * 64, kb * 128, un.bh_head, un.b);
-                        else
-                            tma_load_4d(sB + s * TB + cc * 16384, &tmB, &b_full[s], cc * 64, kvh, kb * 128, un.b);
+                        for (int cc = 0; cc < D / 64; ++cc) {
+                            // chunk cc of the 256-row operand: rows 128 j .. 128 j + 127
+                            uint8_t *dst = sB + s * PB + cc * (2 * 16384) + j * 16384;
+                            if (MODE == MODE_SCORES)
+                                tma_load_4d(dst, &tmB, &b_full[s], cc * 64, (kb + j) * 128, un.bh_head, un.b);
+                            else
+                                tma_load_4d(dst, &tmB, &b_full[s], cc * 64, kvh, (kb + j) * 128, un.b);
+                        }
                     }
                 }
-                if (!ok) break;
             }
             // Let in-flight copies land before the CTA can exit.
-            for (long long t = (tile > NST ? tile - NST : 0); t < tile; ++t)
+            for (long long t = (pair > NST ? pair - NST : 0); t < pair; ++t)
                 mbar_wait_drain(&b_full[t % NST], (t / NST) & 1, p.timeout_ns);
             for (int l = (local > 2 ? local - 2 : 0); l < local; ++l)
                 mbar_wait_drain(&a_full[l & 1], (l >> 1) & 1, p.timeout_ns);
@@ -188,27 +203,29 @@ __global__ void __launch_bounds__(192, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            long long tile = 0;
+            const uint64_t da0 = sdesc_sw128(smem_u32(sA), 16, 1024);
+            const uint64_t db0 = sdesc_sw128(smem_u32(sB), 16, 1024);
+            long long pair = 0;
             int local = 0;
             bool ok = true;
             for (long long u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++local) {
                 const Unit un = decode_unit(p, u, MODE);
                 const int a = local & 1;
                 if (!mbar_wait(&a_full[a], (local >> 1) & 1, wc)) break;
-                tc_fence_after();
-                const uint32_t a_base = smem_u32(sA + a * TB);
-                for (int kb = un.kb0; kb < un.kb1; ++kb, ++tile) {
-                    const int s = static_cast<int>(tile % NST);
-                    if (!mbar_wait(&b_full[s], (tile / NST) & 1, wc)) { ok = false; break; }
-                    const int acc = static_cast<int>(tile & 1);
-                    if (tile >= 2 && !mbar_wait(&acc_empty[acc], ((tile >> 1) - 1) & 1, wc)) { ok = false; break; }
+                const uint64_t da = da0 + static_cast<uint64_t>((a * TB) >> 4);
+                for (int kb = un.kb0; kb < un.kb1; kb += 2, ++pair) {
+                    const int s = static_cast<int>(pair % NST);
+                    const int acc = static_cast<int>(pair & 1);
+                    if (!mbar_wait(&b_full[s], (pair / NST) & 1, wc)) { ok = false; break; }
+                    if (pair >= 2 && !mbar_wait(&acc_empty[acc], ((pair >> 1) - 1) & 1, wc)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t b_base = smem_u32(sB + s * TB);
+                    const uint64_t db = db0 + static_cast<uint64_t>((s * PB) >> 4);
+                    const uint32_t idesc = (un.kb1 - kb >= 2) ? IDESC256 : IDESC128;
 #pragma unroll
                     for (int kk = 0; kk < KSTEPS; ++kk) {
-                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                        umma_ss(tmem + acc * 128, sdesc_sw128(a_base + off, 16, 1024),
-                                sdesc_sw128(b_base + off, 16, 1024), IDESC, kk > 0 ? 1u : 0u);
+                        const uint64_t oa = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+                        const uint64_t ob = static_cast<uint64_t>(((kk >> 2) * 32768 + (kk & 3) * 32) >> 4);
+                        umma_ss(tmem + acc * 256, da + oa, db + ob, idesc, kk > 0 ? 1u : 0u);
                     }
                     umma_commit(&b_empty[s]);
                     umma_commit(&acc_full[acc]);
@@ -222,65 +239,78 @@ __global__ void __launch_bounds__(192, 1)
         const int q4 = static_cast<int>(warp & 3);
         const int row = q4 * 32 + static_cast<int>(lane);
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-        long long tile = 0;
+        long long pair = 0, tile = 0;
         bool ok = true;
         for (long long u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
             const Unit un = decode_unit(p, u, MODE);
-            for (int kb = un.kb0; kb < un.kb1; ++kb, ++tile) {
-                const int acc = static_cast<int>(tile & 1);
-                if (!warp_wait(&acc_full[acc], (tile >> 1) & 1, wc)) { ok = false; break; }
+            for (int kb0 = un.kb0; kb0 < un.kb1; kb0 += 2, ++pair) {
+                const int acc = static_cast<int>(pair & 1);
+                const int nt = min(2, un.kb1 - kb0);
+                if (!warp_wait(&acc_full[acc], (pair >> 1) & 1, wc)) { ok = false; break; }
                 tc_fence_after();
-                const bool diag = (kb == un.qb);
-                uint32_t r[128];
-                tmem_ld128(lane_base + acc * 128, r);
-                // the accumulator row is in registers: hand TMEM back to the MMA warp
-                tc_fence_before();
-                mbar_arrive(&acc_empty[acc]);
-                if (diag) {
-#pragma unroll
-                    for (int j = 0; j < 128; ++j)
-                        if (j > row) r[j] = 0xFF800000u;  // -inf above the diagonal (j > i)
-                }
-                float m8[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const uint32_t *v = r + 8 * j;
-                    m8[j] = fmax3(fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2])),
-                                  fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5])),
-                                  fmaxf(__uint_as_float(v[6]), __uint_as_float(v[7])));
-                }
-                const float mx =
-                    fmax3(fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmax3(m8[6], m8[7], m8[8])),
-                          fmax3(m8[9], m8[10], m8[11]), fmax3(m8[12], m8[13], fmaxf(m8[14], m8[15])));
-                if (MODE == MODE_SCORES) {
-                    float w = mx * p.scale;
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) w = fmaxf(w, __shfl_xor_sync(0xffffffffu, w, o));
-                    if (lane == 0) {
-                        const int slot = static_cast<int>(tile & 3);
-                        atomicMax(&red_max[slot], f2ord(w));
-                        __threadfence_block();
-                        if (atomicAdd(&red_cnt[slot], 1u) == 3u) {
-                            const uint32_t best = atomicExch(&red_max[slot], 0u);
-                            atomicExch(&red_cnt[slot], 0u);
-                            const long long T = static_cast<long long>(p.nb) * (p.nb + 1) / 2;
-                            const long long idx = (static_cast<long long>(un.b) * p.NH + un.bh_head) * T +
-                                                  static_cast<long long>(un.qb) * (un.qb + 1) / 2 + kb;
-                            p.scores[idx] = ord2f(best);
-                        }
+                float mx[2];
+                float lsum[2];
+                for (int j = 0; j < nt; ++j, ++tile) {
+                    const int kb = kb0 + j;
+                    const bool diag = (kb == un.qb);
+                    uint32_t r[128];
+                    tmem_ld128(lane_base + acc * 256 + j * 128, r);
+                    if (j == nt - 1) {
+                        // the accumulator pair is in registers: hand TMEM back to the MMA warp
+                        tc_fence_before();
+                        mbar_arrive(&acc_empty[acc]);
                     }
-                } else {
-                    // log2-domain row max and sum of exp2 over the valid entries
-                    const float m = mx * p.scale;
-                    float acc8[8];
+                    if (diag) {
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) acc8[j] = 0.0f;
+                        for (int c = 0; c < 128; ++c)
+                            if (c > row) r[c] = 0xFF800000u;  // -inf above the diagonal (j > i)
+                    }
+                    float m8[16];
 #pragma unroll
-                    for (int j = 0; j < 128; ++j) acc8[j & 7] += ex2(fmaf(__uint_as_float(r[j]), p.scale, -m));
-                    const float l = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) + ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
-                    const long long idx =
-                        ((static_cast<long long>(un.b) * p.H + un.bh_head) * p.nb + kb) * 128 + row;
-                    p.partial[idx] = make_float2(m, l);
+                    for (int c = 0; c < 16; ++c) {
+                        const uint32_t *v = r + 8 * c;
+                        m8[c] = fmax3(fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2])),
+                                      fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5])),
+                                      fmaxf(__uint_as_float(v[6]), __uint_as_float(v[7])));
+                    }
+                    mx[j] = fmax3(fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmax3(m8[6], m8[7], m8[8])),
+                                  fmax3(m8[9], m8[10], m8[11]), fmax3(m8[12], m8[13], fmaxf(m8[14], m8[15])));
+                    if (MODE == MODE_MASS) {
+                        // log2-domain row max and sum of exp2 over the valid entries
+                        const float m = mx[j] * p.scale;
+                        float acc8[8];
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) acc8[c] = 0.0f;
+#pragma unroll
+                        for (int c = 0; c < 128; ++c) acc8[c & 7] += ex2(fmaf(__uint_as_float(r[c]), p.scale, -m));
+                        lsum[j] = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) + ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
+                    }
+                }
+                for (int j = 0; j < nt; ++j) {
+                    const int kb = kb0 + j;
+                    const long long tj = tile - nt + j;
+                    if (MODE == MODE_SCORES) {
+                        float w = mx[j] * p.scale;
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) w = fmaxf(w, __shfl_xor_sync(0xffffffffu, w, o));
+                        if (lane == 0) {
+                            const int slot = static_cast<int>(tj & 7);
+                            atomicMax(&red_max[slot], f2ord(w));
+                            __threadfence_block();
+                            if (atomicAdd(&red_cnt[slot], 1u) == 3u) {
+                                const uint32_t best = atomicExch(&red_max[slot], 0u);
+                                atomicExch(&red_cnt[slot], 0u);
+                                const long long T = static_cast<long long>(p.nb) * (p.nb + 1) / 2;
+                                const long long idx = (static_cast<long long>(un.b) * p.NH + un.bh_head) * T +
+                                                      static_cast<long long>(un.qb) * (un.qb + 1) / 2 + kb;
+                                p.scores[idx] = ord2f(best);
+                            }
+                        }
+                    } else {
+                        const long long idx =
+                            ((static_cast<long long>(un.b) * p.H + un.bh_head) * p.nb + kb) * 128 + row;
+                        p.partial[idx] = make_float2(mx[j] * p.scale, lsum[j]);
+                    }
                 }
             }
         }
@@ -298,7 +328,7 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, 256);
+    if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace pa
