@@ -100,6 +100,15 @@ def test_pool_matches_numpy_mean_and_head_permutation():
         np.testing.assert_allclose(qp[0, g], qn[0][:, heads].mean(axis=1), rtol=1e-15, atol=0)
         kvs = [h * 4 // 8 for h in heads]
         np.testing.assert_allclose(kp[0, g], kn[0][:, kvs].mean(axis=1), rtol=1e-15, atol=0)
+    # the bf16 proxies are the mean rounded to nearest even: where the mean of
+    # the four bf16 values is exact in fp32 (almost everywhere), torch's
+    # fp32 -> bf16 conversion is an independent reference
+    qmean = np.stack([qn[0][:, list(range(4 * g, 4 * g + 4))].mean(axis=1) for g in range(2)])
+    exact = qmean.astype(np.float32).astype(np.float64) == qmean
+    assert exact.mean() > 0.9
+    ref = torch.from_numpy(qmean.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy()
+    got = qpb[0].view(torch.int16).numpy()
+    assert np.array_equal(got[exact], ref[exact])
     # permuting the heads inside each group leaves the proxies unchanged
     perm = [3, 1, 0, 2, 7, 6, 4, 5]
     qp2, _, qpb2, _ = oracle.pool(q[:, :, perm].contiguous(), k, 2)
