@@ -100,25 +100,30 @@ def _proxy_bits(t: torch.Tensor) -> np.ndarray:
     return t.view(torch.int16).numpy().view(np.uint16)
 
 
-def block_scores(qp_bf16: torch.Tensor, kp_bf16: torch.Tensor, scale: float | None = None) -> np.ndarray:
-    """o2: scores [B, G, T] fp64 from the bf16 proxies [B, G, N, d]."""
+def block_scores(qp_bf16: torch.Tensor, kp_bf16: torch.Tensor, scale: float | None = None,
+                 stride: int = 1) -> np.ndarray:
+    """o2: scores [B, G, T] fp64 from the bf16 proxies [B, G, N, d]; with
+    stride r only the query rows i = r-1 (mod r) are scored."""
     B, G, N, d = qp_bf16.shape
     nb = N // BLK
     scale = 1.0 / np.sqrt(d) if scale is None else scale
+    assert stride >= 1 and BLK % stride == 0
     out = np.empty((B, G, nb * (nb + 1) // 2), np.float64)
     lib().pa_oracle_block_scores(_i(B), _i(N), _i(G), _i(d), _p(_proxy_bits(qp_bf16)),
-                                 _p(_proxy_bits(kp_bf16)), _d(scale), _p(out))
+                                 _p(_proxy_bits(kp_bf16)), _d(scale), _i(stride), _p(out))
     return out
 
 
-def block_score_tiles(qp_bf16: torch.Tensor, kp_bf16: torch.Tensor, tiles, scale: float | None = None) -> np.ndarray:
+def block_score_tiles(qp_bf16: torch.Tensor, kp_bf16: torch.Tensor, tiles, scale: float | None = None,
+                      stride: int = 1) -> np.ndarray:
     """o2 on a sample: tiles is an int array [n, 4] of (b, g, qb, kb)."""
     B, G, N, d = qp_bf16.shape
     scale = 1.0 / np.sqrt(d) if scale is None else scale
+    assert stride >= 1 and BLK % stride == 0
     tiles = np.ascontiguousarray(np.asarray(tiles, np.int32).reshape(-1, 4))
     out = np.empty(len(tiles), np.float64)
     lib().pa_oracle_block_score_tiles(_i(N), _i(G), _i(d), _p(_proxy_bits(qp_bf16)),
-                                      _p(_proxy_bits(kp_bf16)), _d(scale), _i(len(tiles)),
+                                      _p(_proxy_bits(kp_bf16)), _d(scale), _i(stride), _i(len(tiles)),
                                       _p(tiles), _p(out))
     return out
 
@@ -207,13 +212,13 @@ def dense_attn(q, k, v, rows, scale: float | None = None):
     return out, lse
 
 
-def prefill_masks(q, k, G: int, mode=DYNAMIC, gamma=0.95, frac_permille=0):
+def prefill_masks(q, k, G: int, mode=DYNAMIC, gamma=0.95, frac_permille=0, stride=1):
     """o1-o4 end to end on the oracle's own fp64 scores and masses:
     dict(qp, kp, scores, mass, rank, budget, cnt)."""
     B, N, H, d = q.shape
     nb = N // BLK
     _, _, qpb, kpb = pool(q, k, G)
-    scores = block_scores(qpb, kpb)
+    scores = block_scores(qpb, kpb, stride=stride)
     mass = head_mass(q, k) if mode == DYNAMIC else None
     r = rank(scores, nb)
     bud, cnt = budget(r, mass, H, G, nb, mode, gamma, frac_permille)

@@ -127,11 +127,19 @@ void pa_oracle_pool(int B, int N, int H, int Hkv, int d, int G,
 /* ------------------------------------------------------- o2 block scores */
 /* s_ij = scale * sum_c Qp[i,c] Kp[j,c] from the bf16 proxies (the values the
  * GPU multiplies), causal j <= i; score(qb,kb) = max of s_ij over the valid
- * entries of the 128x128 tile.  scores[b][g][tri(qb)+kb], kb <= qb. */
-static double tile_score(const uint16_t *qp, const uint16_t *kp, int d, int qb, int kb, double scale)
+ * entries of the 128x128 tile.  scores[b][g][tri(qb)+kb], kb <= qb.
+ *
+ * Query-row stride (ProxyAttn blog, "5. Experiments", estimation cost: the
+ * pages credit a sequence-level "sliding skip" for the low estimation cost
+ * and do not define it).  Reading: with stride r only the query rows i with
+ * i mod r == r-1 of each tile are scored -- the last row of every window of r
+ * rows, the one whose causal key range covers the others'.  r = 1 scores
+ * every row. */
+static double tile_score(const uint16_t *qp, const uint16_t *kp, int d, int qb, int kb, double scale,
+                         int stride)
 {
     double best = -INFINITY;
-    for (int ii = 0; ii < BLK; ii++) {
+    for (int ii = stride - 1; ii < BLK; ii += stride) {
         int i = qb * BLK + ii;
         for (int jj = 0; jj < BLK; jj++) {
             int j = kb * BLK + jj;
@@ -148,7 +156,7 @@ static double tile_score(const uint16_t *qp, const uint16_t *kp, int d, int qb, 
 
 void pa_oracle_block_scores(int B, int N, int G, int d,
                             const uint16_t *qp, const uint16_t *kp, double scale,
-                            double *scores)
+                            int stride, double *scores)
 {
     int nb = N / BLK;
     int64_t T = tri(nb);
@@ -159,13 +167,14 @@ void pa_oracle_block_scores(int B, int N, int G, int d,
                 const uint16_t *qpg = qp + ((int64_t)b * G + g) * N * d;
                 const uint16_t *kpg = kp + ((int64_t)b * G + g) * N * d;
                 for (int kb = 0; kb <= qb; kb++)
-                    scores[((int64_t)b * G + g) * T + tri(qb) + kb] = tile_score(qpg, kpg, d, qb, kb, scale);
+                    scores[((int64_t)b * G + g) * T + tri(qb) + kb] =
+                        tile_score(qpg, kpg, d, qb, kb, scale, stride);
             }
 }
 
 /* Score of a list of single tiles (b, g, qb, kb): used to sample large sizes. */
 void pa_oracle_block_score_tiles(int N, int G, int d, const uint16_t *qp, const uint16_t *kp,
-                                 double scale, int n_tiles, const int32_t *tiles /* [n][4] */,
+                                 double scale, int stride, int n_tiles, const int32_t *tiles /* [n][4] */,
                                  double *out)
 {
     #pragma omp parallel for schedule(dynamic, 1)
@@ -173,7 +182,7 @@ void pa_oracle_block_score_tiles(int N, int G, int d, const uint16_t *qp, const 
         int b = tiles[4 * t], g = tiles[4 * t + 1], qb = tiles[4 * t + 2], kb = tiles[4 * t + 3];
         const uint16_t *qpg = qp + ((int64_t)b * G + g) * N * d;
         const uint16_t *kpg = kp + ((int64_t)b * G + g) * N * d;
-        out[t] = tile_score(qpg, kpg, d, qb, kb, scale);
+        out[t] = tile_score(qpg, kpg, d, qb, kb, scale, stride);
     }
 }
 

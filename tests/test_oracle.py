@@ -183,6 +183,62 @@ def test_scores_planted_pair_and_causal_mask():
     assert sc2[2] == pytest.approx(-kv[128] / 8)     # tile (1,1)
 
 
+@pytest.mark.parametrize("r", [2, 4, 8])
+def test_strided_scores_planted_rows(r):
+    """Query-row stride r: only rows i = r-1 (mod r) are scored.  A product
+    planted on a scored row sets its tile's score; a larger one planted on a
+    skipped row of another tile leaves that tile at 0; in the diagonal tile a
+    key at j = i counts and a key at j = i + 1 does not."""
+    N, d = 512, 64
+    tri = lambda qb: qb * (qb + 1) // 2
+    qp = torch.zeros(1, 1, N, d)
+    kp = torch.zeros(1, 1, N, d)
+    i_on = 2 * 128 + 5 * r + (r - 1)        # scored row of qb 2
+    i_off = 3 * 128 + 7 * r                  # skipped row of qb 3 (i_off mod r == 0)
+    qp[0, 0, i_on, 3] = 2.0
+    kp[0, 0, 130, 3] = 3.0                   # kb 1: tile (2, 1) = 6/8; tile (3, 1) sees it through no scored row
+    qp[0, 0, i_off, 9] = 4.0
+    kp[0, 0, 20, 9] = 4.0                    # kb 0: 16/8 only through the skipped row
+    sc = oracle.block_scores(qp.bfloat16(), kp.bfloat16(), stride=r)[0, 0]
+    assert sc[tri(2) + 1] == pytest.approx(6.0 / 8.0)
+    assert sc[tri(3) + 0] == 0.0
+    rest = np.ones_like(sc, bool)
+    rest[tri(2) + 1] = False
+    assert np.all(sc[rest] == 0.0)
+    # diagonal tile: key j = i_on counts, j = i_on + 1 does not
+    kp2 = torch.zeros(1, 1, N, d)
+    kp2[0, 0, i_on, 3] = 1.0
+    kp2[0, 0, i_on + 1, 3] = 8.0
+    sc2 = oracle.block_scores(qp.bfloat16(), kp2.bfloat16(), stride=r)[0, 0]
+    assert sc2[tri(2) + 2] == pytest.approx(2.0 / 8.0)
+    # stride 1 sees the skipped row's product
+    sc1 = oracle.block_scores(qp.bfloat16(), kp.bfloat16(), stride=1)[0, 0]
+    assert sc1[tri(3) + 0] == pytest.approx(16.0 / 8.0)
+
+
+@pytest.mark.parametrize("r", [2, 4, 8])
+def test_strided_scores_equal_full_scores_of_window_copies(r):
+    """Replacing every query row by the scored row of its window (the last of
+    each r rows) gives a proxy whose every-row scores equal the strided
+    scores of the original: each copy sees a subset of the keys the scored row
+    sees.  Scores also shrink as the stride doubles (the scored rows of 2r are
+    a subset of those of r)."""
+    w = synth.small_workload(seqlen=640, heads=4, kv_heads=2, head_dim=64, groups=2)
+    x = synth.make_inputs(w)
+    _, _, qpb, kpb = oracle.pool(x["q"], x["k"], 2)
+    N = qpb.shape[2]
+    src = (np.arange(N) // r) * r + (r - 1)
+    dup = qpb[:, :, torch.as_tensor(src)].contiguous()
+    strided = oracle.block_scores(qpb, kpb, stride=r)
+    full_dup = oracle.block_scores(dup, kpb, stride=1)
+    assert np.array_equal(strided, full_dup)
+    full = oracle.block_scores(qpb, kpb, stride=1)
+    assert np.all(strided <= full)
+    if r < 8:
+        assert np.all(oracle.block_scores(qpb, kpb, stride=2 * r) <= strided)
+    assert np.any(strided < full)
+
+
 def test_score_tiles_equal_full_scores():
     w = synth.small_workload(seqlen=384, heads=4, kv_heads=2, head_dim=64, groups=2)
     x = synth.make_inputs(w)

@@ -53,6 +53,10 @@ MUTANTS = [
     ("sparse_v_from_q_head", "o[c] += p * bf16_to_f64(v[b * vsb + (int64_t)j * vss + kvh * vsh + c]);\n                }\n            if (lse)",
      "o[c] += p * bf16_to_f64(v[b * vsb + (int64_t)j * vss + (h % Hkv) * vsh + c]);\n                }\n            if (lse)"),
     ("dense_wrong_scale", "            z[j] = scale * s;", "            z[j] = s;"),
+    ("stride_first_row_of_window", "for (int ii = stride - 1; ii < BLK; ii += stride) {",
+     "for (int ii = 0; ii < BLK; ii += stride) {"),
+    ("stride_ignored", "for (int ii = stride - 1; ii < BLK; ii += stride) {",
+     "for (int ii = 0; ii < BLK; ii++) {"),
 ]
 
 # The pins each mutant runs against (all of them are cheap).
@@ -63,6 +67,7 @@ PINS = [
     T.test_pool_matches_numpy_mean_and_head_permutation,
     T.test_scores_one_head_per_group_equal_per_head_scores,
     T.test_scores_planted_pair_and_causal_mask,
+    lambda: T.test_strided_scores_planted_rows(4),
     T.test_mass_rows_sum_to_one_and_match_scipy_softmax,
     lambda: T.test_rank_brute_force_with_ties(0),
     lambda: T.test_budget_brute_force_and_invariants(0),
