@@ -59,6 +59,8 @@ def parse_args():
     ap.add_argument("--mode", choices=sorted(MODES), default="dynamic")
     ap.add_argument("--gamma", type=float, default=None)
     ap.add_argument("--frac", type=int, default=100, help="fixed budget in per mille of causal blocks")
+    ap.add_argument("--score-stride", type=int, default=1, choices=[1, 2, 4, 8],
+                    help="query-row stride of the proxy block scores (1: every row)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
@@ -141,7 +143,7 @@ class Pipeline:
     """Pre-allocated buffers and ctypes arguments for one layer, so that a step is
     four C-ABI calls with CUDA events between them."""
 
-    def __init__(self, q, k, v, G, mode, gamma, frac):
+    def __init__(self, q, k, v, G, mode, gamma, frac, stride=1):
         import block_sparse_attention_pa_b200 as pa
         self.pa = pa
         self.L = pa.lib()
@@ -150,11 +152,12 @@ class Pipeline:
         self.B, self.N, self.H, self.d, self.G = B, N, H, d, G
         self.nb = N // 128
         self.shape = pa.make_shape(q, k, G)
-        self.budget = pa.make_budget(mode, gamma, frac)
+        self.budget = pa.make_budget(mode, gamma, frac, stride)
         self.mode = mode
+        self.stride = stride
         dev = q.device
-        self.qp = torch.empty(B, G, N, d, device=dev, dtype=torch.bfloat16)
-        self.kp = torch.empty_like(self.qp)
+        self.qp = torch.empty(B, G, N // stride, d, device=dev, dtype=torch.bfloat16)
+        self.kp = torch.empty(B, G, N, d, device=dev, dtype=torch.bfloat16)
         T = self.nb * (self.nb + 1) // 2
         self.T = T
         self.scores = torch.empty(B, G, T, device=dev, dtype=torch.float32)
@@ -170,10 +173,11 @@ class Pipeline:
         pa, L, st = self.pa, self.L, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
         sh, bu = ctypes.byref(self.shape), ctypes.byref(self.budget)
         if ev: ev[0].record()
-        pa._check(L.pa_pool_heads(sh, self.q.data_ptr(), self.qs, self.k.data_ptr(), self.ks, self.qp.data_ptr(),
-                                  self.kp.data_ptr(), st))
+        pa._check(L.pa_pool_heads_strided(sh, self.stride, self.q.data_ptr(), self.qs, self.k.data_ptr(), self.ks,
+                                          self.qp.data_ptr(), self.kp.data_ptr(), st))
         if ev: ev[1].record()
-        pa._check(L.pa_block_scores(sh, self.qp.data_ptr(), self.kp.data_ptr(), self.scores.data_ptr(), st))
+        pa._check(L.pa_block_scores_strided(sh, self.stride, self.qp.data_ptr(), self.kp.data_ptr(),
+                                            self.scores.data_ptr(), st))
         if ev: ev[2].record()
         pa._check(L.pa_build_mask(sh, bu, self.scores.data_ptr(), self.q.data_ptr(), self.qs, self.k.data_ptr(),
                                   self.ks, ctypes.byref(self.bufs), self.ws.data_ptr(), self.ws.numel(), st))
@@ -265,7 +269,7 @@ ATTN_SOURCES = ["block_sparse_attention_pa_b200/csrc/attn.cuh", "block_sparse_at
 
 
 # ------------------------------------------------------------ CPU oracle
-def oracle_estimate(x, w: synth.Workload, G, mode, gamma, frac, size="baseline", seed=0):
+def oracle_estimate(x, w: synth.Workload, G, mode, gamma, frac, size="baseline", seed=0, stride=1):
     """Time the CPU oracle on a bounded sample of one layer and extrapolate to
     ms per layer.  x: CPU bf16 tensors.  Returns (ms_per_layer, per-stage
     seconds, description of the sample)."""
@@ -290,7 +294,7 @@ def oracle_estimate(x, w: synth.Workload, G, mode, gamma, frac, size="baseline",
     kbs = np.linspace(0, nbp - 1, min(n_tiles, nbp)).astype(int)
     tiles = [(0, g, nbp - 1, int(kb)) for g in range(G) for kb in kbs]
     t0 = time.perf_counter()
-    last = oracle.block_score_tiles(qpb, kpb, tiles)
+    last = oracle.block_score_tiles(qpb, kpb, tiles, stride=stride)
     det["scores_s"] = (time.perf_counter() - t0) * (B * G * T) / len(tiles)
     # o3 head mass of mass_heads heads (with their KV heads)
     hk = max(1, mass_heads * Hkv // H)
@@ -331,7 +335,8 @@ def run_reference(args, w, G, mode, gamma, frac):
     x = synth.make_inputs(w, device="cpu")
     vals = []
     for i in range(args.warmup + args.steps):
-        ms, det, sample = oracle_estimate(x, w, G, mode, gamma, frac, size="step", seed=i)
+        ms, det, sample = oracle_estimate(x, w, G, mode, gamma, frac, size="step", seed=i,
+                                          stride=args.score_stride)
         if i >= args.warmup:
             vals.append(ms)
     v = statistics.mean(vals)
@@ -339,16 +344,17 @@ def run_reference(args, w, G, mode, gamma, frac):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "ms/layer", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": v, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_of(w, G, mode, gamma, frac),
+            "config": config_of(w, G, mode, gamma, frac, args.score_stride),
             "cpu_baseline": {"value": v, "unit": "ms/layer", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "ms/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def config_of(w, G, mode, gamma, frac):
+def config_of(w, G, mode, gamma, frac, stride=1):
     budget = {0: f"dynamic gamma={gamma}", 1: f"fixed {frac / 10:.1f}% of causal blocks", 2: "all causal blocks"}[mode]
     return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "q_heads": w.num_q_heads,
             "kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "groups": G, "budget": budget, "block": 128,
+            "score_stride": stride,
             "l2": "inputs larger than L2 (q+k+v per layer > 126 MB), no flush"}
 
 
@@ -378,7 +384,8 @@ def main():
 
     x = synth.make_inputs(w, device=f"cuda:{local}", seed=w.seed + rank)
     q, k, v = x["q"], x["k"], x["v"]
-    pipe = Pipeline(q, k, v, G, mode, gamma, frac)
+    stride = args.score_stride
+    pipe = Pipeline(q, k, v, G, mode, gamma, frac, stride)
     sampler = None if args.no_clocks else ClockSampler(local)
     total_ms, stages, clocks = time_pipeline(pipe, args.steps, args.warmup, dist_on, sampler)
     status = pa.device_status()
@@ -406,8 +413,9 @@ def main():
     # per-stage rooflines
     d = w.head_dim
     Hkv = w.num_kv_heads
-    pool_bytes = B * w.seqlen * d * 2 * (H + Hkv + 2 * G)
-    score_flops = B * G * T * 2 * 128 * 128 * d
+    # strided scores read and pool only the scored q rows (1/stride of them)
+    pool_bytes = B * w.seqlen * d * 2 * ((H + G) / stride + Hkv + G)
+    score_flops = B * G * T * 2 * 128 * 128 * d / stride
     stage_roofline = {
         "pool": {"ms": float(stages[0]), "GB/s": pool_bytes / (stages[0] * 1e-3) / 1e9,
                  "frac_hbm": pool_bytes / (stages[0] * 1e-3) / 1e9 / peaks["hbm_gbs"]},
@@ -421,7 +429,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded needle/sink generator; random inputs, no weights)",
-            "config": config_of(w, G, mode, gamma, frac) | {"parallelism": f"replicas x{world}"},
+            "config": config_of(w, G, mode, gamma, frac, stride) | {"parallelism": f"replicas x{world}"},
             "est_ms": est_ms, "sparse_ms": attn_ms,
             "tflops_effective": achieved, "tflops_exact_causal": flops_exact / (attn_ms * 1e-3) / 1e12,
             "visited_blocks": visited, "density": density, "sparsity": 1.0 - density,
@@ -434,7 +442,7 @@ def main():
 
     # dense baseline: the same kernel with every causal block selected
     if not args.no_dense:
-        dense = Pipeline(q, k, v, G, 2, gamma, frac)
+        dense = Pipeline(q, k, v, G, 2, gamma, frac, stride)
         dsteps = max(2, min(5, args.steps))
         _, dstages, _ = time_pipeline(dense, dsteps, 1, dist_on)
         dense_attn = float(dstages[3])
@@ -448,14 +456,14 @@ def main():
 
     # end to end through the public API with pinned host buffers
     if not args.no_e2e:
-        e2e = run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world)
+        e2e = run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world, stride)
         line["e2e"] = e2e
 
     # the CPU oracle on a bounded sample (rank 0, one GPU only)
     if not args.no_cpu_baseline and world == 1 and rank == 0:
         import oracle
         xc = {n: x[n].cpu() for n in ("q", "k", "v")}
-        ms, det, sample = oracle_estimate(xc, w, G, mode, gamma, frac, size="baseline")
+        ms, det, sample = oracle_estimate(xc, w, G, mode, gamma, frac, size="baseline", stride=stride)
         line["cpu_baseline"] = {"value": ms, "unit": "ms/layer", "cores": oracle.num_threads(), "kind": "oracle",
                                 "sample": sample, "stage_s": det}
 
@@ -466,7 +474,7 @@ def main():
         torch.distributed.destroy_process_group()
 
 
-def run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world):
+def run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world, stride=1):
     """The metric through the public API with host buffers, as a user runs
     consecutive layers: every step copies its q, k, v from pinned host memory
     and reads its o back.  Two device buffer sets and two copy streams let the
@@ -475,7 +483,7 @@ def run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world):
     q, k, v = x["q"], x["k"], x["v"]
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
     bufs = [tuple(torch.empty_like(t) for t in (q, k, v, q)) for _ in range(2)]
-    call = pa.Prefill(bufs[0][0], bufs[0][1], bufs[0][2], G, mode, gamma, frac)
+    call = pa.Prefill(bufs[0][0], bufs[0][1], bufs[0][2], G, mode, gamma, frac, stride)
     ho = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(2)]
     ms = torch.cuda.current_stream()
     hs, ds = torch.cuda.Stream(), torch.cuda.Stream()

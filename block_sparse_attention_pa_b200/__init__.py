@@ -31,7 +31,10 @@ STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_E
 # Every entry point declared in include/pa.h.
 ENTRY_POINTS = ("pa_workspace_size", "pa_pool_heads", "pa_block_scores", "pa_build_mask",
                 "pa_block_sparse_attn", "pa_prefill", "pa_get_device_status", "pa_status_string",
-                "pa_last_error", "pa_abi_version", "pa_build_mask_noalloc", "pa_selftest_wait_timeout")
+                "pa_last_error", "pa_abi_version", "pa_build_mask_noalloc", "pa_selftest_wait_timeout",
+                "pa_pool_heads_strided", "pa_block_scores_strided")
+
+SCORE_STRIDES = (1, 2, 4, 8)
 
 
 class PaError(RuntimeError):
@@ -51,7 +54,8 @@ class Strides(ctypes.Structure):
 
 
 class Budget(ctypes.Structure):
-    _fields_ = [("mode", ctypes.c_int32), ("gamma", ctypes.c_float), ("frac_permille", ctypes.c_int32)]
+    _fields_ = [("mode", ctypes.c_int32), ("gamma", ctypes.c_float), ("frac_permille", ctypes.c_int32),
+                ("score_stride", ctypes.c_int32)]
 
 
 class MaskBufs(ctypes.Structure):
@@ -76,6 +80,8 @@ def lib() -> ctypes.CDLL:
         L.pa_workspace_size.argtypes = [P(Shape), P(Budget)]
         L.pa_pool_heads.argtypes = [P(Shape), vp, st, vp, st, vp, vp, vp]
         L.pa_block_scores.argtypes = [P(Shape), vp, vp, vp, vp]
+        L.pa_pool_heads_strided.argtypes = [P(Shape), ctypes.c_int32, vp, st, vp, st, vp, vp, vp]
+        L.pa_block_scores_strided.argtypes = [P(Shape), ctypes.c_int32, vp, vp, vp, vp]
         L.pa_build_mask.argtypes = [P(Shape), P(Budget), vp, vp, st, vp, st, P(MaskBufs), vp, ctypes.c_size_t, vp]
         L.pa_block_sparse_attn.argtypes = [P(Shape), vp, st, vp, st, vp, st, vp, vp, ctypes.c_float, vp, st, vp, vp]
         L.pa_prefill.argtypes = [P(Shape), P(Budget), vp, st, vp, st, vp, st, vp, st, P(MaskBufs), vp,
@@ -87,7 +93,8 @@ def lib() -> ctypes.CDLL:
         L.pa_last_error.restype = ctypes.c_char_p
         L.pa_abi_version.restype = ctypes.c_int32
         for name in ("pa_pool_heads", "pa_block_scores", "pa_build_mask", "pa_block_sparse_attn", "pa_prefill",
-                     "pa_get_device_status", "pa_selftest_wait_timeout"):
+                     "pa_get_device_status", "pa_selftest_wait_timeout", "pa_pool_heads_strided",
+                     "pa_block_scores_strided"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -119,8 +126,8 @@ def make_shape(q: torch.Tensor, k: torch.Tensor, num_groups: int) -> Shape:
     return Shape(B, N, H, k.shape[2], d, 128, num_groups)
 
 
-def make_budget(mode: int = DYNAMIC, gamma: float = 0.95, frac_permille: int = 0) -> Budget:
-    return Budget(mode, gamma, frac_permille)
+def make_budget(mode: int = DYNAMIC, gamma: float = 0.95, frac_permille: int = 0, score_stride: int = 1) -> Budget:
+    return Budget(mode, gamma, frac_permille, score_stride)
 
 
 def workspace_size(shape: Shape, budget: Budget) -> int:
@@ -151,31 +158,46 @@ class Mask:
                         self.mass.data_ptr() if self.mass is not None else None)
 
 
-def pool_heads(q: torch.Tensor, k: torch.Tensor, num_groups: int):
-    """pa_pool_heads -> (q_proxy, k_proxy), bf16 [B, G, N, d]."""
+def pool_heads(q: torch.Tensor, k: torch.Tensor, num_groups: int, score_stride: int = 1):
+    """pa_pool_heads (score_stride 1) or pa_pool_heads_strided -> (q_proxy,
+    k_proxy): q_proxy bf16 [B, G, N/score_stride, d], k_proxy [B, G, N, d]."""
     _cuda_bf16(q, "q")
     _cuda_bf16(k, "k")
     shape = make_shape(q, k, num_groups)
     B, N, H, d = q.shape
-    qp = torch.empty(B, num_groups, N, d, device=q.device, dtype=torch.bfloat16)
-    kp = torch.empty_like(qp)
-    _check(lib().pa_pool_heads(ctypes.byref(shape), q.data_ptr(), _strides(q), k.data_ptr(), _strides(k),
-                               qp.data_ptr(), kp.data_ptr(), _stream(q.device)))
+    r = int(score_stride)
+    qp = torch.empty(B, num_groups, N // r if r in SCORE_STRIDES else N, d, device=q.device, dtype=torch.bfloat16)
+    kp = torch.empty(B, num_groups, N, d, device=q.device, dtype=torch.bfloat16)
+    if r == 1:
+        _check(lib().pa_pool_heads(ctypes.byref(shape), q.data_ptr(), _strides(q), k.data_ptr(), _strides(k),
+                                   qp.data_ptr(), kp.data_ptr(), _stream(q.device)))
+    else:
+        _check(lib().pa_pool_heads_strided(ctypes.byref(shape), r, q.data_ptr(), _strides(q), k.data_ptr(),
+                                           _strides(k), qp.data_ptr(), kp.data_ptr(), _stream(q.device)))
     return qp, kp
 
 
-def block_scores(q_proxy: torch.Tensor, k_proxy: torch.Tensor, num_q_heads: int = 1, num_kv_heads: int = 1):
-    """pa_block_scores -> fp32 [B, G, T]."""
+def block_scores(q_proxy: torch.Tensor, k_proxy: torch.Tensor, num_q_heads: int = 1, num_kv_heads: int = 1,
+                 score_stride: int = 1):
+    """pa_block_scores (score_stride 1) or pa_block_scores_strided -> fp32
+    [B, G, T].  k_proxy is [B, G, N, d]; q_proxy [B, G, N/score_stride, d]."""
     for t, n in ((q_proxy, "q_proxy"), (k_proxy, "k_proxy")):
         if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and t.dim() == 4):
             raise ValueError(f"{n} must be a contiguous bf16 CUDA tensor [B, G, N, d]")
-    B, G, N, d = q_proxy.shape
+    B, G, N, d = k_proxy.shape
+    r = int(score_stride)
+    if tuple(q_proxy.shape) != (B, G, N // max(r, 1), d):
+        raise ValueError(f"q_proxy must be [B, G, N/{r}, d] = {(B, G, N // max(r, 1), d)}, got {tuple(q_proxy.shape)}")
     H = max(num_q_heads, G)
     shape = Shape(B, N, H, min(num_kv_heads, H), d, 128, G)
     nb = N // 128
     scores = torch.empty(B, G, nb * (nb + 1) // 2, device=q_proxy.device, dtype=torch.float32)
-    _check(lib().pa_block_scores(ctypes.byref(shape), q_proxy.data_ptr(), k_proxy.data_ptr(), scores.data_ptr(),
-                                 _stream(q_proxy.device)))
+    if r == 1:
+        _check(lib().pa_block_scores(ctypes.byref(shape), q_proxy.data_ptr(), k_proxy.data_ptr(), scores.data_ptr(),
+                                     _stream(q_proxy.device)))
+    else:
+        _check(lib().pa_block_scores_strided(ctypes.byref(shape), r, q_proxy.data_ptr(), k_proxy.data_ptr(),
+                                             scores.data_ptr(), _stream(q_proxy.device)))
     return scores
 
 
@@ -216,11 +238,12 @@ def block_sparse_attn(q, k, v, rank, cnt, num_groups: int, softmax_scale: float 
 class Prefill:
     """A reusable pa_prefill call: workspace and mask buffers allocated once."""
 
-    def __init__(self, q, k, v, num_groups: int, mode: int = DYNAMIC, gamma: float = 0.95, frac_permille: int = 0):
+    def __init__(self, q, k, v, num_groups: int, mode: int = DYNAMIC, gamma: float = 0.95, frac_permille: int = 0,
+                 score_stride: int = 1):
         for t, n in ((q, "q"), (k, "k"), (v, "v")):
             _cuda_bf16(t, n)
         self.shape = make_shape(q, k, num_groups)
-        self.budget = make_budget(mode, gamma, frac_permille)
+        self.budget = make_budget(mode, gamma, frac_permille, score_stride)
         self.mask = Mask.empty(self.shape, q.device, mode == DYNAMIC)
         self.ws = torch.empty(workspace_size(self.shape, self.budget), device=q.device, dtype=torch.uint8)
         self._bufs = self.mask.bufs()
@@ -233,9 +256,10 @@ class Prefill:
         return out
 
 
-def prefill(q, k, v, num_groups: int, mode: int = DYNAMIC, gamma: float = 0.95, frac_permille: int = 0):
+def prefill(q, k, v, num_groups: int, mode: int = DYNAMIC, gamma: float = 0.95, frac_permille: int = 0,
+            score_stride: int = 1):
     """pa_prefill -> (o, Mask)."""
-    call = Prefill(q, k, v, num_groups, mode, gamma, frac_permille)
+    call = Prefill(q, k, v, num_groups, mode, gamma, frac_permille, score_stride)
     o = torch.empty_like(q, memory_format=torch.contiguous_format)
     call(q, k, v, o)
     return o, call.mask

@@ -79,8 +79,19 @@ pa_status check_shape(const pa_shape *s) {
     return PA_OK;
 }
 
+// Query-row stride of the block scores: 1, 2, 4 or 8.
+pa_status check_stride(int r) {
+    if (r != 1 && r != 2 && r != 4 && r != 8)
+        return fail(PA_ERR_INVALID_ARG, "score_stride must be 1, 2, 4 or 8 (got %d)", r);
+    return PA_OK;
+}
+
+// pa_budget.score_stride with 0 (a zero-initialised struct) read as 1.
+int stride_of(const pa_budget *bu) { return (bu && bu->score_stride > 0) ? bu->score_stride : 1; }
+
 pa_status check_budget(const pa_budget *bu) {
     if (!bu) return fail(PA_ERR_INVALID_ARG, "budget is NULL");
+    if (bu->score_stride != 0 && check_stride(bu->score_stride)) return PA_ERR_INVALID_ARG;
     if (bu->mode == PA_BUDGET_DYNAMIC) {
         if (!(bu->gamma > 0.0f && bu->gamma <= 1.0f))
             return fail(PA_ERR_INVALID_ARG, "gamma must be in (0, 1] (got %g)", static_cast<double>(bu->gamma));
@@ -178,7 +189,7 @@ WsLayout ws_layout(const pa_shape *s, const pa_budget *bu) {
     w.partial = 0;
     const size_t part = (bu && bu->mode == PA_BUDGET_DYNAMIC) ? align256(B * H * nb * 128 * sizeof(float2)) : 0;
     w.qp = part;
-    w.kp = w.qp + align256(B * G * N * d * 2);
+    w.kp = w.qp + align256(B * G * (N / stride_of(bu)) * d * 2);  // strided q proxy: scored rows only
     w.scores = w.kp + align256(B * G * N * d * 2);
     w.total = w.scores + align256(B * G * T * sizeof(float));
     return w;
@@ -189,8 +200,8 @@ size_t mask_ws_bytes(const pa_shape *s, const pa_budget *bu) {
 }
 
 // ------------------------------------------------------------- launches
-pa_status launch_pool(const pa_shape *s, const void *q, pa_strides qs, const void *k, pa_strides ks, void *qp,
-                      void *kp, cudaStream_t st) {
+pa_status launch_pool(const pa_shape *s, int stride, const void *q, pa_strides qs, const void *k, pa_strides ks,
+                      void *qp, void *kp, cudaStream_t st) {
     pa::PoolParams p;
     p.q = static_cast<const __nv_bfloat16 *>(q);
     p.k = static_cast<const __nv_bfloat16 *>(k);
@@ -200,6 +211,7 @@ pa_status launch_pool(const pa_shape *s, const void *q, pa_strides qs, const voi
     p.ksb = ks.b; p.kss = ks.s; p.ksh = ks.h;
     p.B = s->batch; p.N = s->seqlen; p.H = s->num_q_heads; p.Hkv = s->num_kv_heads;
     p.G = s->num_groups; p.d = s->head_dim;
+    p.stride = stride;
     const long long threads = static_cast<long long>(p.B) * p.N * p.G * (p.d / 8);
     const unsigned grid = static_cast<unsigned>((threads + 255) / 256);
     if (p.d == 128) pa::pool_heads_kernel<128><<<grid, 256, 0, st>>>(p);
@@ -220,17 +232,22 @@ pa_status launch_tile_gemm_t(const CUtensorMap &a, const CUtensorMap &b, const p
     return PA_OK;
 }
 
-pa_status launch_scores(const pa_shape *s, const void *qp, const void *kp, float *scores, cudaStream_t st) {
+pa_status launch_scores(const pa_shape *s, int stride, const void *qp, const void *kp, float *scores,
+                        cudaStream_t st) {
     const int B = s->batch, G = s->num_groups, N = s->seqlen, d = s->head_dim, nb = N / kBlk;
     CUtensorMap ma, mb;
-    pa_status r = map_proxy(&ma, qp, B, G, N, d, "q_proxy");
+    pa_status r = map_proxy(&ma, qp, B, G, N / stride, d, "q_proxy");
     if (r) return r;
     if ((r = map_proxy(&mb, kp, B, G, N, d, "k_proxy"))) return r;
     pa::TileParams p{};
     p.B = B; p.nb = nb; p.NH = G; p.H = s->num_q_heads; p.Hkv = s->num_kv_heads;
     p.chunk = kScoreChunk;
+    p.stride = stride;
+    // A tile m (query blocks m*r .. m*r+r-1) owns ceil((m+1) / (chunk/r)) units
+    const int cr = kScoreChunk / stride;
+    const int a_tiles = (nb + stride - 1) / stride;
     long long per = 0;
-    for (int qb = 0; qb < nb; ++qb) per += (qb + kScoreChunk) / kScoreChunk;
+    for (int m = 0; m < a_tiles; ++m) per += (m + cr) / cr;
     p.units_per_bh = per;
     p.num_units = per * B * G;
     p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
@@ -252,6 +269,7 @@ pa_status launch_mass(const pa_shape *s, const void *q, pa_strides qs, const voi
     pa::TileParams p{};
     p.B = B; p.nb = nb; p.NH = H; p.H = H; p.Hkv = Hkv;
     p.chunk = kScoreChunk;
+    p.stride = 1;
     p.units_per_bh = (nb + kScoreChunk - 1) / kScoreChunk;
     p.num_units = p.units_per_bh * B * H;
     p.scale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
@@ -398,24 +416,36 @@ size_t pa_workspace_size(const pa_shape *shape, const pa_budget *budget) {
     return ws_layout(shape, budget).total;
 }
 
-pa_status pa_pool_heads(const pa_shape *shape, const void *q, pa_strides qs, const void *k, pa_strides ks,
-                        void *q_proxy, void *k_proxy, pa_stream_t stream) {
+pa_status pa_pool_heads_strided(const pa_shape *shape, int32_t score_stride, const void *q, pa_strides qs,
+                                const void *k, pa_strides ks, void *q_proxy, void *k_proxy, pa_stream_t stream) {
     pa_status r;
-    if ((r = check_shape(shape))) return r;
+    if ((r = check_shape(shape)) || (r = check_stride(score_stride))) return r;
     if ((r = check_tensor(q, qs, "q")) || (r = check_tensor(k, ks, "k"))) return r;
     if ((r = check_ptr(q_proxy, "q_proxy")) || (r = check_ptr(k_proxy, "k_proxy"))) return r;
-    if ((r = launch_pool(shape, q, qs, k, ks, q_proxy, k_proxy, reinterpret_cast<cudaStream_t>(stream)))) return r;
+    if ((r = launch_pool(shape, score_stride, q, qs, k, ks, q_proxy, k_proxy, reinterpret_cast<cudaStream_t>(stream))))
+        return r;
+    return ok();
+}
+
+pa_status pa_pool_heads(const pa_shape *shape, const void *q, pa_strides qs, const void *k, pa_strides ks,
+                        void *q_proxy, void *k_proxy, pa_stream_t stream) {
+    return pa_pool_heads_strided(shape, 1, q, qs, k, ks, q_proxy, k_proxy, stream);
+}
+
+pa_status pa_block_scores_strided(const pa_shape *shape, int32_t score_stride, const void *q_proxy,
+                                  const void *k_proxy, float *scores, pa_stream_t stream) {
+    pa_status r;
+    if ((r = check_shape(shape)) || (r = check_stride(score_stride))) return r;
+    if ((r = check_ptr(q_proxy, "q_proxy")) || (r = check_ptr(k_proxy, "k_proxy"))) return r;
+    if ((r = check_ptr(scores, "scores", 4))) return r;
+    if ((r = launch_scores(shape, score_stride, q_proxy, k_proxy, scores, reinterpret_cast<cudaStream_t>(stream))))
+        return r;
     return ok();
 }
 
 pa_status pa_block_scores(const pa_shape *shape, const void *q_proxy, const void *k_proxy, float *scores,
                           pa_stream_t stream) {
-    pa_status r;
-    if ((r = check_shape(shape))) return r;
-    if ((r = check_ptr(q_proxy, "q_proxy")) || (r = check_ptr(k_proxy, "k_proxy"))) return r;
-    if ((r = check_ptr(scores, "scores", 4))) return r;
-    if ((r = launch_scores(shape, q_proxy, k_proxy, scores, reinterpret_cast<cudaStream_t>(stream)))) return r;
-    return ok();
+    return pa_block_scores_strided(shape, 1, q_proxy, k_proxy, scores, stream);
 }
 
 pa_status pa_build_mask(const pa_shape *shape, const pa_budget *budget, const float *scores, const void *q,
@@ -475,8 +505,9 @@ pa_status pa_prefill(const pa_shape *shape, const pa_budget *budget, const void 
     void *qp = base + w.qp;
     void *kp = base + w.kp;
     float *scores = reinterpret_cast<float *>(base + w.scores);
-    if ((r = launch_pool(shape, q, qs, k, ks, qp, kp, st))) return r;
-    if ((r = launch_scores(shape, qp, kp, scores, st))) return r;
+    const int stride = stride_of(budget);
+    if ((r = launch_pool(shape, stride, q, qs, k, ks, qp, kp, st))) return r;
+    if ((r = launch_scores(shape, stride, qp, kp, scores, st))) return r;
     if (budget->mode == PA_BUDGET_DYNAMIC &&
         (r = launch_mass(shape, q, qs, k, ks, reinterpret_cast<float2 *>(base + w.partial), mask_out->mass, st)))
         return r;

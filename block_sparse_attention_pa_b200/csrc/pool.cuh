@@ -9,6 +9,10 @@
 // rounded once to bf16, so the result equals the exact-mean definition bit for
 // bit whenever the sum of the group's bf16 values is exact in fp64 (always,
 // unless the values span more than ~2^40 in magnitude).
+//
+// With a query-row stride r only the q rows i = r-1 (mod r) are pooled (the
+// only rows the strided block scores read), into row i/r of a [B][G][N/r][d]
+// q proxy; the k proxy is always complete.
 #pragma once
 #include "sm100.cuh"
 
@@ -21,6 +25,7 @@ struct PoolParams {
     __nv_bfloat16 *kp;
     int64_t qsb, qss, qsh, ksb, kss, ksh;
     int B, N, H, Hkv, G, d;
+    int stride;  // query-row stride r (1: every row)
 };
 
 __device__ __forceinline__ void add_bf16x8(double (&acc)[8], const uint4 &v) {
@@ -67,6 +72,7 @@ __global__ void __launch_bounds__(256, 2) pool_heads_kernel(PoolParams p) {
     const int h0 = g * hpg;
     const __nv_bfloat16 *qrow = p.q + b * p.qsb + i * p.qss + c;
     const __nv_bfloat16 *krow = p.k + b * p.ksb + i * p.kss + c;
+    const bool doq = (i % p.stride) == p.stride - 1;
 
     double aq[8], ak[8];
 #pragma unroll
@@ -82,21 +88,25 @@ __global__ void __launch_bounds__(256, 2) pool_heads_kernel(PoolParams p) {
             if (t < n) {
                 const int h = h0 + t0 + t;
                 const int kvh = static_cast<int>(static_cast<int64_t>(h) * p.Hkv / p.H);
-                qv[t] = __ldg(reinterpret_cast<const uint4 *>(qrow + h * p.qsh));
+                if (doq) qv[t] = __ldg(reinterpret_cast<const uint4 *>(qrow + h * p.qsh));
                 kvv[t] = __ldg(reinterpret_cast<const uint4 *>(krow + kvh * p.ksh));
             }
         }
 #pragma unroll
         for (int t = 0; t < 6; ++t) {
             if (t < n) {
-                add_bf16x8(aq, qv[t]);
+                if (doq) add_bf16x8(aq, qv[t]);
                 add_bf16x8(ak, kvv[t]);
             }
         }
     }
     const int64_t o = ((static_cast<int64_t>(b) * p.G + g) * p.N + i) * D + c;
-    *reinterpret_cast<uint4 *>(p.qp + o) = mean_to_bf16x8(aq, hpg);
     *reinterpret_cast<uint4 *>(p.kp + o) = mean_to_bf16x8(ak, hpg);
+    if (doq) {
+        const int nq = p.N / p.stride;
+        const int64_t oq = ((static_cast<int64_t>(b) * p.G + g) * nq + i / p.stride) * D + c;
+        *reinterpret_cast<uint4 *>(p.qp + oq) = mean_to_bf16x8(aq, hpg);
+    }
 }
 
 }  // namespace pa

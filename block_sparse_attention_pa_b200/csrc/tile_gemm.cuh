@@ -5,7 +5,11 @@
 //                Estimation": the QK product of the proxy heads fused with
 //                block-level max pooling).  For every causal tile (qb, kb<=qb)
 //                of every proxy group: score = max over the tile's valid
-//                entries of (q_p . k_p)/sqrt(d).
+//                entries of (q_p . k_p)/sqrt(d).  With a query-row stride r
+//                (the sequence-level skip of "5. Experiments", read as scoring
+//                every r-th query row) the A operand holds only the scored
+//                rows, so one 128-row A tile spans r query blocks of 128/r
+//                scored rows each and the tensor work drops by r.
 //   MODE_MASS    (Step 2, budget from the last query block).  For every head,
 //                the last query block against every key block: per row, the
 //                max m and sum l of exp2 of the log2-scaled logits over the
@@ -31,7 +35,8 @@ enum { MODE_SCORES = 0, MODE_MASS = 1 };
 struct TileParams {
     int B, nb, NH;         // NH: proxy groups (scores) or q heads (mass)
     int H, Hkv;            // mass: q head -> KV head
-    int chunk;             // tiles per unit
+    int chunk;             // tiles per unit (a multiple of stride)
+    int stride;            // scores: query-row stride r in {1,2,4,8}; mass: 1
     long long units_per_bh;
     long long num_units;
     float scale;           // scores: 1/sqrt(d); mass: scale*log2(e)
@@ -41,11 +46,13 @@ struct TileParams {
 };
 
 struct Unit {
-    int b, bh_head, qb, kb0, kb1;  // tiles kb0 .. kb1-1
+    int b, bh_head, qb, kb0, kb1;  // tiles kb0 .. kb1-1; scores: qb is the A tile (query blocks qb*r ..)
 };
 
-// Scores: within one (b, g) the rows qb = C*a + t (t < C) own a+1 units each,
-// so the units before row C*a number C*a(a+1)/2.
+// Scores: A tile m covers query blocks m*r .. m*r+r-1 and so key tiles
+// 0 .. min(r(m+1), nb)-1, split into units of C tiles: ceil((m+1)/Cr) units
+// with Cr = C/r.  Within one (b, g) the A tiles m = Cr*a + t (t < Cr) own a+1
+// units each, so the units before A tile Cr*a number Cr*a(a+1)/2.
 __device__ __forceinline__ Unit decode_unit(const TileParams &p, long long u, int mode) {
     Unit r;
     const long long bh = u / p.units_per_bh;
@@ -54,15 +61,16 @@ __device__ __forceinline__ Unit decode_unit(const TileParams &p, long long u, in
     r.bh_head = static_cast<int>(bh % p.NH);
     const int C = p.chunk;
     if (mode == MODE_SCORES) {
-        long long a = static_cast<long long>((sqrt(1.0 + 8.0 * static_cast<double>(w) / C) - 1.0) * 0.5);
-        while (a > 0 && static_cast<long long>(C) * a * (a + 1) / 2 > w) --a;
-        while (static_cast<long long>(C) * (a + 1) * (a + 2) / 2 <= w) ++a;
-        const long long rem = w - static_cast<long long>(C) * a * (a + 1) / 2;
+        const int Cr = C / p.stride;
+        long long a = static_cast<long long>((sqrt(1.0 + 8.0 * static_cast<double>(w) / Cr) - 1.0) * 0.5);
+        while (a > 0 && static_cast<long long>(Cr) * a * (a + 1) / 2 > w) --a;
+        while (static_cast<long long>(Cr) * (a + 1) * (a + 2) / 2 <= w) ++a;
+        const long long rem = w - static_cast<long long>(Cr) * a * (a + 1) / 2;
         const int t = static_cast<int>(rem / (a + 1));
         const int c = static_cast<int>(rem % (a + 1));
-        r.qb = static_cast<int>(C * a + t);
+        r.qb = static_cast<int>(Cr * a + t);
         r.kb0 = c * C;
-        r.kb1 = min(r.kb0 + C, r.qb + 1);
+        r.kb1 = min(r.kb0 + C, min(p.stride * (r.qb + 1), p.nb));
     } else {
         r.qb = p.nb - 1;
         r.kb0 = static_cast<int>(w) * C;
@@ -121,8 +129,8 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t *b_empty = bars + 9 + NST;       // NST
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 9 + 2 * NST);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    uint32_t *red_max = tmem_slot + 2;        // [8] per-tile cross-warp max (ring)
-    uint32_t *red_cnt = tmem_slot + 10;       // [8]
+    uint32_t *red_max = tmem_slot + 2;        // [16] per-(tile, query block) cross-warp max (ring)
+    uint32_t *red_cnt = tmem_slot + 18;       // [16]
 
     const uint32_t warp = warp_id(), lane = lane_id();
     if (threadIdx.x == 0) {
@@ -136,7 +144,7 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(&b_full[i], 1);
             mbar_init(&b_empty[i], 1);
         }
-        for (int i = 0; i < 8; ++i) red_max[i] = red_cnt[i] = 0;
+        for (int i = 0; i < 16; ++i) red_max[i] = red_cnt[i] = 0;
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -239,10 +247,17 @@ __global__ void __launch_bounds__(192, 1)
         const int q4 = static_cast<int>(warp & 3);
         const int row = q4 * 32 + static_cast<int>(lane);
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+        // A row -> (query block within the A tile, token offset inside that block)
+        const int rows_per_qb = 128 / p.stride;
+        const int qsub = row / rows_per_qb;
+        const int toff = (row % rows_per_qb) * p.stride + p.stride - 1;
+        const int span = min(rows_per_qb, 32);  // lanes of a warp that share a query block
+        const int wpq = rows_per_qb / 32;       // warps that share a query block (0: part of one warp)
         long long pair = 0, tile = 0;
         bool ok = true;
         for (long long u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
             const Unit un = decode_unit(p, u, MODE);
+            const int qbw = (MODE == MODE_SCORES) ? un.qb * p.stride + qsub : un.qb;  // this row's query block
             for (int kb0 = un.kb0; kb0 < un.kb1; kb0 += 2, ++pair) {
                 const int acc = static_cast<int>(pair & 1);
                 const int nt = min(2, un.kb1 - kb0);
@@ -252,7 +267,7 @@ __global__ void __launch_bounds__(192, 1)
                 float lsum[2];
                 for (int j = 0; j < nt; ++j, ++tile) {
                     const int kb = kb0 + j;
-                    const bool diag = (kb == un.qb);
+                    const bool diag = (kb == qbw);
                     uint32_t r[128];
                     tmem_ld128(lane_base + acc * 256 + j * 128, r);
                     if (j == nt - 1) {
@@ -263,7 +278,7 @@ __global__ void __launch_bounds__(192, 1)
                     if (diag) {
 #pragma unroll
                         for (int c = 0; c < 128; ++c)
-                            if (c > row) r[c] = 0xFF800000u;  // -inf above the diagonal (j > i)
+                            if (c > toff) r[c] = 0xFF800000u;  // -inf above the diagonal (j > i)
                     }
                     float m8[16];
 #pragma unroll
@@ -292,18 +307,26 @@ __global__ void __launch_bounds__(192, 1)
                     if (MODE == MODE_SCORES) {
                         float w = mx[j] * p.scale;
 #pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) w = fmaxf(w, __shfl_xor_sync(0xffffffffu, w, o));
-                        if (lane == 0) {
-                            const int slot = static_cast<int>(tj & 7);
-                            atomicMax(&red_max[slot], f2ord(w));
-                            __threadfence_block();
-                            if (atomicAdd(&red_cnt[slot], 1u) == 3u) {
-                                const uint32_t best = atomicExch(&red_max[slot], 0u);
-                                atomicExch(&red_cnt[slot], 0u);
-                                const long long T = static_cast<long long>(p.nb) * (p.nb + 1) / 2;
-                                const long long idx = (static_cast<long long>(un.b) * p.NH + un.bh_head) * T +
-                                                      static_cast<long long>(un.qb) * (un.qb + 1) / 2 + kb;
-                                p.scores[idx] = ord2f(best);
+                        for (int o = 16; o > 0; o >>= 1)
+                            if (o < span) w = fmaxf(w, __shfl_xor_sync(0xffffffffu, w, o));
+                        // tiles above this query block's diagonal, and A rows past the last
+                        // block (zero-filled), give no score
+                        const bool valid = kb <= qbw && qbw < p.nb;
+                        if (valid && (static_cast<int>(lane) & (span - 1)) == 0) {
+                            const long long T = static_cast<long long>(p.nb) * (p.nb + 1) / 2;
+                            const long long idx = (static_cast<long long>(un.b) * p.NH + un.bh_head) * T +
+                                                  static_cast<long long>(qbw) * (qbw + 1) / 2 + kb;
+                            if (wpq <= 1) {
+                                p.scores[idx] = w;
+                            } else {
+                                const int slot = static_cast<int>(tj & 7) * 2 + (qsub & 1);
+                                atomicMax(&red_max[slot], f2ord(w));
+                                __threadfence_block();
+                                if (atomicAdd(&red_cnt[slot], 1u) == static_cast<uint32_t>(wpq - 1)) {
+                                    const uint32_t best = atomicExch(&red_max[slot], 0u);
+                                    atomicExch(&red_cnt[slot], 0u);
+                                    p.scores[idx] = ord2f(best);
+                                }
                             }
                         }
                     } else {

@@ -16,7 +16,9 @@
  *   all bf16, addressed with pa_strides (element strides of the batch, token
  *   and head dimensions); d is contiguous.  Base pointers must be 16-byte
  *   aligned and every stride a multiple of 8 elements (16 bytes).
- *   Proxies q_proxy/k_proxy are contiguous bf16 [B][G][N][d].
+ *   Proxies q_proxy/k_proxy are contiguous bf16 [B][G][N][d]; with a
+ *   query-row stride r > 1 (see pa_budget.score_stride) q_proxy holds only
+ *   the scored rows, [B][G][N/r][d].
  *   Block scores and ranked lists are [B][G][T] with nb = N/128,
  *   T = nb(nb+1)/2 and query block qb's row starting at tri(qb) = qb(qb+1)/2
  *   (entries tri(qb)+0 .. tri(qb)+qb).
@@ -44,7 +46,7 @@
 extern "C" {
 #endif
 
-#define PA_ABI_VERSION 1
+#define PA_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define PA_API __attribute__((visibility("default")))
@@ -89,6 +91,10 @@ typedef struct pa_budget {
     int32_t mode;          /* pa_budget_mode */
     float gamma;           /* DYNAMIC: softmax-mass threshold in (0, 1] */
     int32_t frac_permille; /* FIXED_FRACTION: 1..1000 */
+    int32_t score_stride;  /* query-row stride r of the block scores: 0 or 1
+                              scores every row; 2, 4 or 8 scores only rows
+                              i with i mod r == r-1 (pa_block_scores_strided).
+                              Used by pa_prefill and pa_workspace_size. */
 } pa_budget;
 
 /* Mask buffers written by pa_build_mask / pa_prefill (device, caller-owned).
@@ -133,6 +139,28 @@ PA_API pa_status pa_pool_heads(const pa_shape *shape,
 PA_API pa_status pa_block_scores(const pa_shape *shape,
                           const void *q_proxy, const void *k_proxy,
                           float *scores, pa_stream_t stream);
+
+/* Step 1 with a query-row stride r in {1, 2, 4, 8} (ProxyAttn blog,
+ * "5. Experiments", estimation cost: the pages credit a sequence-level
+ * "sliding skip" for keeping the estimate cheap but do not define it; here it
+ * is read as scoring only every r-th query row).  The scored rows of a block
+ * are i with i mod r == r-1, the last row of each window of r rows.
+ *   pa_pool_heads_strided: as pa_pool_heads, but q_proxy is [B][G][N/r][d]
+ *     and its row t is the proxy of query row i = t*r + r-1; k_proxy is the
+ *     full [B][G][N][d].
+ *   pa_block_scores_strided: as pa_block_scores from those proxies, with the
+ *     max over the scored rows i of block qb only:
+ *       scores[b][g][tri(qb)+kb] = max over i in block qb, i mod r == r-1,
+ *                                  j in block kb, j <= i of (q_p[i].k_p[j])/sqrt(d)
+ * r = 1 is exactly pa_pool_heads / pa_block_scores.  Other r: PA_ERR_INVALID_ARG. */
+PA_API pa_status pa_pool_heads_strided(const pa_shape *shape, int32_t score_stride,
+                                       const void *q, pa_strides q_strides,
+                                       const void *k, pa_strides k_strides,
+                                       void *q_proxy, void *k_proxy, pa_stream_t stream);
+
+PA_API pa_status pa_block_scores_strided(const pa_shape *shape, int32_t score_stride,
+                                         const void *q_proxy, const void *k_proxy,
+                                         float *scores, pa_stream_t stream);
 
 /* Step 1 "Block Ranking" + Step 2 "dynamic budget" (ProxyAttn blog,
  * 4. ProxyAttn method; the threshold rule is XAttention's find_blocks,
@@ -200,7 +228,8 @@ PA_API pa_status pa_block_sparse_attn(const pa_shape *shape,
                                pa_stream_t stream);
 
 /* The whole path: pa_pool_heads -> pa_block_scores -> pa_build_mask ->
- * pa_block_sparse_attn with softmax_scale = 1/sqrt(d).  The proxies and block
+ * pa_block_sparse_attn with softmax_scale = 1/sqrt(d) (the strided pooling
+ * and scores when budget->score_stride > 1).  The proxies and block
  * scores live in the workspace; the mask is written to *mask_out (all four
  * buffers required in DYNAMIC mode, mass may be NULL otherwise). */
 PA_API pa_status pa_prefill(const pa_shape *shape, const pa_budget *budget,

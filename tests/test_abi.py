@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_version_and_status_strings(L):
-    assert L.pa_abi_version() == 1
+    assert L.pa_abi_version() == 2
     for code in range(8):
         assert L.pa_status_string(code).decode() not in ("", "unknown status")
     assert L.pa_status_string(99).decode() == "unknown status"
@@ -55,6 +55,13 @@ def test_workspace_size_formula(L):
     assert fixed == 2 * a256(2 * 1024 * 64 * 2) + a256(2 * T * 4)
     assert pa.workspace_size(shape(N=1000), pa.make_budget()) == 0
     assert pa.workspace_size(s, pa.make_budget(pa.DYNAMIC, 1.5)) == 0
+    # a query-row stride r keeps only N/r rows of the q proxy; 0 reads as 1
+    for r in (2, 4, 8):
+        st = pa.workspace_size(s, pa.make_budget(pa.FIXED_FRACTION, 0, 100, r))
+        assert st == a256(2 * (1024 // r) * 64 * 2) + a256(2 * 1024 * 64 * 2) + a256(2 * T * 4)
+    assert pa.workspace_size(s, pa.make_budget(pa.FIXED_FRACTION, 0, 100, 0)) == fixed
+    for r in (3, 16, -1):
+        assert pa.workspace_size(s, pa.make_budget(pa.FIXED_FRACTION, 0, 100, r)) == 0
 
 
 @pytest.mark.parametrize("bad,code", [
@@ -83,6 +90,20 @@ def test_null_and_misaligned_pointers_rejected(L):
     assert L.pa_pool_heads(ctypes.byref(s), 16, pa.Strides(0, 512, 60), 16, st, 16, 16, None) == 1
     assert L.pa_block_scores(ctypes.byref(s), 16, 16, None, None) == 1
     assert L.pa_block_scores(None, 16, 16, 16, None) == 1
+
+
+@pytest.mark.parametrize("r", [0, 3, 16, -2])
+def test_bad_score_stride_rejected(L, r):
+    s = shape()
+    st = pa.Strides(0, 512, 64)
+    assert L.pa_pool_heads_strided(ctypes.byref(s), r, 16, st, 16, st, 16, 16, None) == 1
+    assert b"score_stride" in L.pa_last_error()
+    assert L.pa_block_scores_strided(ctypes.byref(s), r, 16, 16, 16, None) == 1
+    if r != 0:  # 0 in pa_budget means "every row"
+        m = pa.MaskBufs(16, 16, 16, 16)
+        bad = pa.make_budget(pa.FIXED_FRACTION, 0, 100, r)
+        assert L.pa_prefill(ctypes.byref(s), ctypes.byref(bad), 16, st, 16, st, 16, st, 16, st, ctypes.byref(m),
+                            256, 1 << 30, None) == 1
 
 
 def test_budget_and_workspace_errors(L):
