@@ -198,6 +198,23 @@ class Pipeline:
         return v, v * per, exact
 
 
+def selected_blocks(pipe) -> torch.Tensor:
+    """Bool [B, H, T]: entry tri(qb)+kb is set when head h visits KV block kb
+    in query block qb (the first cnt entries of its group's ranked list)."""
+    B, H, G, nb, T = pipe.B, pipe.H, pipe.G, pipe.nb, pipe.T
+    dev = pipe.mask.rank.device
+    pos = torch.arange(T, device=dev)
+    starts = torch.arange(nb, device=dev) * (torch.arange(nb, device=dev) + 1) // 2
+    row = torch.searchsorted(starts, pos, right=True) - 1
+    t = pos - starts[row]
+    grp = torch.arange(H, device=dev) * G // H
+    rank_h = pipe.mask.rank.long()[:, grp]                      # [B, H, T]
+    inlist = t[None, None] < pipe.mask.cnt.long()[:, :, row]    # [B, H, T]
+    sel = torch.zeros(B, H, T, dtype=torch.bool, device=dev)
+    sel.scatter_(2, starts[row][None, None] + rank_h, inlist)
+    return sel
+
+
 def max_over_ranks(value: float, device) -> float:
     """The max of a per-rank time over all ranks (the job's time); the value
     itself without a process group."""
@@ -453,6 +470,19 @@ def main():
         line["layer_speedup_vs_dense"] = dense_attn / (est_ms + attn_ms)
         line["estimate_frac_of_dense"] = est_ms / dense_attn
         del dense
+
+    # the strided estimate's selection against the every-row estimate's
+    if stride > 1:
+        every = Pipeline(q, k, v, G, mode, gamma, frac, 1)
+        every.step()
+        torch.cuda.synchronize()
+        a, b = selected_blocks(pipe), selected_blocks(every)
+        both = int((a & b).sum().item())
+        line["selection_vs_every_row"] = {
+            "recall": both / max(int(b.sum().item()), 1),
+            "jaccard": both / max(int((a | b).sum().item()), 1),
+            "density_every_row": int(b.sum().item()) / b.numel()}
+        del every, a, b
 
     # end to end through the public API with pinned host buffers
     if not args.no_e2e:

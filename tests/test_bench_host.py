@@ -54,3 +54,33 @@ def test_reference_arm_prints_on_rank0_only(rank, expect_line):
         assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     else:
         assert lines == []
+
+
+def test_selected_blocks_matches_loops():
+    """The bench's selection map (used to compare two estimates) against plain
+    loops over the ranked lists and counts."""
+    import types
+    import numpy as np
+    import torch
+    rng = np.random.default_rng(3)
+    B, H, G, nb = 2, 4, 2, 6
+    T = nb * (nb + 1) // 2
+    rank = np.zeros((B, G, T), np.int32)
+    for b in range(B):
+        for g in range(G):
+            for qb in range(nb):
+                rank[b, g, qb * (qb + 1) // 2: qb * (qb + 1) // 2 + qb + 1] = rng.permutation(qb + 1)
+    cnt = np.stack([[[int(rng.integers(1, qb + 2)) for qb in range(nb)] for _ in range(H)] for _ in range(B)])
+    pipe = types.SimpleNamespace(B=B, H=H, G=G, nb=nb, T=T,
+                                 mask=types.SimpleNamespace(rank=torch.from_numpy(rank),
+                                                            cnt=torch.from_numpy(cnt.astype(np.int32))))
+    got = bench.selected_blocks(pipe).numpy()
+    ref = np.zeros((B, H, T), bool)
+    for b in range(B):
+        for h in range(H):
+            g = h * G // H
+            for qb in range(nb):
+                s = qb * (qb + 1) // 2
+                for kb in rank[b, g, s:s + cnt[b, h, qb]]:
+                    ref[b, h, s + kb] = True
+    assert np.array_equal(got, ref)
