@@ -193,6 +193,39 @@ def sparse_attn(q, k, v, rank_lists, cnt, G: int, items, scale: float | None = N
     return out, lse
 
 
+def sparse_attn_skip(q, k, v, rank_lists, cnt, G: int, items, lam: float, skip_in=None,
+                     scale: float | None = None):
+    """o7: o5 with the running-max block skip at threshold lam.  Returns
+    (O [n, 128, d], lse [n, 128], skip [B, H, T] uint8, gap [B, H, T] fp64):
+    skip and gap hold the oracle's own decision and its margin (log2 units)
+    for every visited block of the items (gap NaN elsewhere, +inf for each
+    item's first block).  skip_in ([B, H, T], nonzero = skipped) replaces the
+    oracle's decisions in the output."""
+    B, N, H, d = q.shape
+    Hkv = k.shape[2]
+    nb = N // BLK
+    T = nb * (nb + 1) // 2
+    scale = 1.0 / np.sqrt(d) if scale is None else scale
+    qa, qs = _bits(q)
+    ka, ks = _bits(k)
+    va, vs = _bits(v)
+    items = np.ascontiguousarray(np.asarray(items, np.int32).reshape(-1, 3))
+    r = np.ascontiguousarray(np.asarray(rank_lists, np.int32))
+    c = np.ascontiguousarray(np.asarray(cnt, np.int32))
+    out = np.empty((len(items), BLK, d), np.float64)
+    lse = np.empty((len(items), BLK), np.float64)
+    skip = np.zeros((B, H, T), np.uint8)
+    gap = np.full((B, H, T), np.nan, np.float64)
+    sin = None if skip_in is None else np.ascontiguousarray(np.asarray(skip_in, np.uint8).reshape(B, H, T))
+    lib().pa_oracle_sparse_attn_skip(_i(N), _i(H), _i(Hkv), _i(d), _i(G),
+                                     _p(qa), _i64(qs[0]), _i64(qs[1]), _i64(qs[2]),
+                                     _p(ka), _i64(ks[0]), _i64(ks[1]), _i64(ks[2]),
+                                     _p(va), _i64(vs[0]), _i64(vs[1]), _i64(vs[2]),
+                                     _p(r), _p(c), _d(scale), _d(lam), _i(len(items)), _p(items),
+                                     _p(sin) if sin is not None else None, _p(skip), _p(gap), _p(out), _p(lse))
+    return out, lse, skip, gap
+
+
 def dense_attn(q, k, v, rows, scale: float | None = None):
     """o6: for rows [n, 3] of (b, h, i) returns (O [n, d], lse [n]) fp64."""
     B, N, H, d = q.shape

@@ -33,6 +33,9 @@
  *                             the scaled Q.K products (section 2 "Background"),
  *                             restricted to the selected causal keys.
  *   o6 pa_oracle_dense_attn   Plain causal softmax attention, written separately.
+ *   o7 pa_oracle_sparse_attn_skip  o5 with BLASST's running-max block skip
+ *                             (BLASST introduction, 3.1): a visited block far
+ *                             below the running max is left out.
  *
  * Readings where the pages are silent (all listed in the design notes):
  *   mean pooling; K pooled over the expanded KV heads of the group's q heads;
@@ -370,6 +373,130 @@ void pa_oracle_sparse_attn(int N, int H, int Hkv, int d, int G,
             if (lse) lse[(int64_t)it * BLK + ii] = zmax + log(den);
         }
         free(z);
+    }
+}
+
+/* ------------------------------------------------ o7 running-max block skip */
+/* BLASST (BLASST introduction; "3.1 pruning attention with the running max"):
+ * while the online softmax walks the blocks, a block whose largest score lies
+ * far below the running maximum of the blocks before it adds almost nothing
+ * after normalisation, so its exponentials and its V product are skipped.
+ * The rule's own text is cut off on the pages; readings:
+ *  - visit order: the selected blocks of (b, h, qb) by ascending block index;
+ *  - running max M_i of row i: the max of its scaled logits over the blocks
+ *    visited before (a skipped block never raises it);
+ *  - a block after the first is skipped when every row i of the query block
+ *    has max_{j in block, j <= i} z_ij - M_i < ln(lambda), lambda in [0, 1]
+ *    ("softmax thresholding": the block's largest probability relative to
+ *    the running max is below lambda); lambda = 0 never skips;
+ *  - the output is the softmax over the keys of the blocks not skipped.
+ * skip_in (nullable, [B][H][T], entry tri(qb)+kb): decisions to apply instead
+ * of the oracle's own.  skip_out and gap (nullable, [B][H][T]) receive, for
+ * every visited block, the oracle's own decision and its margin
+ * (max_i (max_j z_ij - M_i) - ln(lambda)) * log2(e) (+inf for the first
+ * block); entries of blocks not visited are left as they are. */
+void pa_oracle_sparse_attn_skip(int N, int H, int Hkv, int d, int G,
+                                const uint16_t *q, int64_t qsb, int64_t qss, int64_t qsh,
+                                const uint16_t *k, int64_t ksb, int64_t kss, int64_t ksh,
+                                const uint16_t *v, int64_t vsb, int64_t vss, int64_t vsh,
+                                const int32_t *rank, const int32_t *cnt, double scale, double lambda,
+                                int n_items, const int32_t *items /* [n][3] = b,h,qb */,
+                                const uint8_t *skip_in, uint8_t *skip_out, double *gap,
+                                double *out, double *lse)
+{
+    int nb = N / BLK;
+    int64_t T = tri(nb);
+    double lnl = (lambda > 0.0) ? log(lambda) : -INFINITY;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int it = 0; it < n_items; it++) {
+        int b = items[3 * it], h = items[3 * it + 1], qb = items[3 * it + 2];
+        int g = grp_of(h, H, G), kvh = kv_of(h, H, Hkv);
+        const int32_t *list = rank + ((int64_t)b * G + g) * T + tri(qb);
+        int n = cnt[((int64_t)b * H + h) * nb + qb];
+        int64_t base = ((int64_t)b * H + h) * T + tri(qb);
+        int *blk = (int *)malloc(sizeof(int) * (n > 0 ? n : 1));
+        double *mt = (double *)malloc(sizeof(double) * BLK * (n > 0 ? n : 1));
+        unsigned char *use = (unsigned char *)malloc(n > 0 ? n : 1);
+        double *row_max = (double *)malloc(sizeof(double) * BLK);
+        /* visit order: ascending block index (insertion sort of the list prefix) */
+        for (int t = 0; t < n; t++) {
+            int x = list[t], u = t;
+            while (u > 0 && blk[u - 1] > x) { blk[u] = blk[u - 1]; u--; }
+            blk[u] = x;
+        }
+        /* every row's maximum scaled logit in every visited block */
+        for (int ii = 0; ii < BLK; ii++) {
+            int i = qb * BLK + ii;
+            for (int t = 0; t < n; t++) {
+                double best = -INFINITY;
+                for (int jj = 0; jj < BLK; jj++) {
+                    int j = blk[t] * BLK + jj;
+                    if (j > i) continue;
+                    double s = 0.0;
+                    for (int c = 0; c < d; c++)
+                        s += bf16_to_f64(q[b * qsb + (int64_t)i * qss + h * qsh + c]) *
+                             bf16_to_f64(k[b * ksb + (int64_t)j * kss + kvh * ksh + c]);
+                    s *= scale;
+                    if (s > best) best = s;
+                }
+                mt[ii * n + t] = best;
+            }
+        }
+        /* decisions in visit order against each row's running max */
+        for (int ii = 0; ii < BLK; ii++) row_max[ii] = -INFINITY;
+        for (int t = 0; t < n; t++) {
+            int own = 0;
+            double margin = INFINITY;
+            if (t > 0) {
+                double worst = -INFINITY;
+                for (int ii = 0; ii < BLK; ii++) {
+                    double e = mt[ii * n + t] - row_max[ii];
+                    if (e > worst) worst = e;
+                }
+                own = worst < lnl;
+                margin = (worst - lnl) * 1.4426950408889634;
+            }
+            for (int ii = 0; ii < BLK; ii++)
+                if (mt[ii * n + t] > row_max[ii]) row_max[ii] = mt[ii * n + t];
+            if (skip_out) skip_out[base + blk[t]] = (uint8_t)own;
+            if (gap) gap[base + blk[t]] = margin;
+            use[t] = skip_in ? !skip_in[base + blk[t]] : !own;
+        }
+        /* softmax over the keys of the blocks kept */
+        for (int ii = 0; ii < BLK; ii++) {
+            int i = qb * BLK + ii;
+            double zmax = -INFINITY;
+            for (int t = 0; t < n; t++)
+                if (use[t] && mt[ii * n + t] > zmax) zmax = mt[ii * n + t];
+            double den = 0.0;
+            double *o = out + ((int64_t)it * BLK + ii) * d;
+            for (int c = 0; c < d; c++) o[c] = 0.0;
+            for (int pass = 0; pass < 2; pass++)
+                for (int t = 0; t < n; t++) {
+                    if (!use[t]) continue;
+                    for (int jj = 0; jj < BLK; jj++) {
+                        int j = blk[t] * BLK + jj;
+                        if (j > i) continue;
+                        double s = 0.0;
+                        for (int c = 0; c < d; c++)
+                            s += bf16_to_f64(q[b * qsb + (int64_t)i * qss + h * qsh + c]) *
+                                 bf16_to_f64(k[b * ksb + (int64_t)j * kss + kvh * ksh + c]);
+                        double e = exp(s * scale - zmax);
+                        if (pass == 0) {
+                            den += e;
+                        } else {
+                            double pr = e / den;
+                            for (int c = 0; c < d; c++)
+                                o[c] += pr * bf16_to_f64(v[b * vsb + (int64_t)j * vss + kvh * vsh + c]);
+                        }
+                    }
+                }
+            if (lse) lse[(int64_t)it * BLK + ii] = zmax + log(den);
+        }
+        free(blk);
+        free(mt);
+        free(use);
+        free(row_max);
     }
 }
 

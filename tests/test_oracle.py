@@ -499,3 +499,140 @@ def test_attention_head_dim_one_textbook_softmax():
         p = np.exp(z - z.max())
         p /= p.sum()
         assert o[0, i, 0] == pytest.approx(float(p @ vd[:i + 1]), abs=1e-13)
+
+
+# ------------------------------------------------ o7 running-max block skip
+def _skip_inputs(N=512, d=16, seed=21, scales=(1.0, 0.25, 3.0, 0.5)):
+    """One head, random bf16 q, k, v; K of block kb scaled by scales[kb] so
+    that some blocks sit far below the running max and some do not."""
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(1, N, 1, d, generator=g)
+    k = torch.randn(1, N, 1, d, generator=g)
+    v = torch.randn(1, N, 1, d, generator=g)
+    for kb, s in enumerate(scales):
+        k[:, kb * 128:(kb + 1) * 128] *= s
+    return q.bfloat16(), k.bfloat16(), v.bfloat16()
+
+
+def _full_lists(nb, shuffle_seed=None):
+    """Every causal block listed, each row's list in a shuffled order."""
+    T = nb * (nb + 1) // 2
+    rank = np.zeros((1, 1, T), np.int32)
+    rng = np.random.default_rng(shuffle_seed)
+    for qb in range(nb):
+        lst = np.arange(qb + 1)
+        if shuffle_seed is not None:
+            rng.shuffle(lst)
+        rank[0, 0, qb * (qb + 1) // 2: qb * (qb + 1) // 2 + qb + 1] = lst
+    cnt = np.array([[[qb + 1 for qb in range(nb)]]], np.int32)
+    return rank, cnt
+
+
+def brute_skip(q, k, v, qb, blocks, lam, scale):
+    """numpy: the query block's logits against the listed blocks in ascending
+    order, each row's running max, the block decisions, and the softmax over
+    the keys of the blocks kept."""
+    qf = q[0, :, 0].double().numpy()
+    kf = k[0, :, 0].double().numpy()
+    vf = v[0, :, 0].double().numpy()
+    rows = np.arange(qb * 128, qb * 128 + 128)
+    z = scale * qf[rows] @ kf.T
+    z[np.arange(128)[:, None] + qb * 128 < np.arange(kf.shape[0])[None, :]] = -np.inf
+    run = np.full(128, -np.inf)
+    keep = []
+    for t, kb in enumerate(sorted(blocks)):
+        tile_max = z[:, kb * 128:(kb + 1) * 128].max(axis=1)
+        skip = t > 0 and lam > 0 and np.max(tile_max - run) < np.log(lam)
+        run = np.maximum(run, tile_max)
+        keep.append((kb, not skip))
+    cols = np.concatenate([np.arange(kb * 128, kb * 128 + 128) for kb, kp in keep if kp])
+    zz = z[:, cols]
+    p = np.exp(zz - zz.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    return p @ vf[cols], {kb: not kp for kb, kp in keep}
+
+
+@pytest.mark.parametrize("lam", [0.02, 0.2, 0.6])
+def test_skip_brute_force(lam):
+    """o7 against a numpy restatement on a tiny case (decisions and O)."""
+    q, k, v = _skip_inputs()
+    nb = 4
+    rank, cnt = _full_lists(nb, shuffle_seed=1)
+    items = [(0, 0, qb) for qb in range(nb)]
+    out, _, skip, gap = oracle.sparse_attn_skip(q, k, v, rank, cnt, 1, items, lam)
+    scale = 1 / 4.0
+    for n, (_, _, qb) in enumerate(items):
+        ref, dec = brute_skip(q, k, v, qb, list(range(qb + 1)), lam, scale)
+        np.testing.assert_allclose(out[n], ref, rtol=1e-10, atol=1e-12)
+        for kb, sk in dec.items():
+            assert skip[0, 0, qb * (qb + 1) // 2 + kb] == sk
+            assert abs(gap[0, 0, qb * (qb + 1) // 2 + kb]) > 1e-9  # no decision on a knife edge
+
+
+def test_skip_sweep_skips_some_and_nests():
+    """The decisions are nested in lambda, and the sweep above both skips and
+    keeps later blocks (so the brute-force pin is not vacuous)."""
+    q, k, v = _skip_inputs()
+    rank, cnt = _full_lists(4)
+    items = [(0, 0, qb) for qb in range(4)]
+    prev = None
+    counts = []
+    for lam in (0.0, 0.02, 0.2, 0.6, 1.0):
+        _, _, skip, _ = oracle.sparse_attn_skip(q, k, v, rank, cnt, 1, items, lam)
+        if prev is not None:
+            assert np.all(skip >= prev)
+        prev = skip
+        counts.append(int(skip.sum()))
+    assert counts[0] == 0 and counts[-1] > counts[1] and counts[-1] < 6
+
+
+def test_skip_planted_running_max():
+    """Logits 0 (block 0), 8 (block 1), 4 (blocks 2, 3) for every row of query
+    block 3; lambda = e^-2.  Block 1 raises the running max to 8, so blocks 2
+    and 3 (4 - 8 < -2) are skipped though they lie far above block 0; the
+    output is the softmax over blocks 0 and 1 alone (o5 with the list [0, 1]),
+    and the margins are (4 - 8 + 2) log2(e)."""
+    N, d = 512, 16
+    q = torch.zeros(1, N, 1, d)
+    q[..., 0] = 2.0
+    k = torch.zeros(1, N, 1, d)
+    k[:, 128:256, 0, 0] = 16.0
+    k[:, 256:512, 0, 0] = 8.0
+    v = torch.randn(1, N, 1, d, generator=torch.Generator().manual_seed(3))
+    q, k, v = q.bfloat16(), k.bfloat16(), v.bfloat16()
+    rank, cnt = _full_lists(4, shuffle_seed=2)
+    out, _, skip, gap = oracle.sparse_attn_skip(q, k, v, rank, cnt, 1, [(0, 0, 3)], math.exp(-2.0))
+    assert list(skip[0, 0, 6:10]) == [0, 0, 1, 1]
+    np.testing.assert_allclose(gap[0, 0, 8:10], (4 - 8 + 2) / math.log(2), rtol=1e-12)
+    assert gap[0, 0, 7] == pytest.approx((8 - 0 + 2) / math.log(2))
+    r2 = rank.copy()
+    r2[0, 0, 6:10] = [0, 1, 2, 3]
+    c2 = cnt.copy()
+    c2[0, 0, 3] = 2
+    ref, _ = oracle.sparse_attn(q, k, v, r2, c2, 1, [(0, 0, 3)])
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-14)
+
+
+def test_skip_zero_threshold_and_given_decisions():
+    """lambda = 0 skips nothing and equals o5; decisions passed in are the
+    ones applied (none skipped -> o5; the oracle's own -> its own output)."""
+    w = synth.small_workload(seqlen=512, heads=4, kv_heads=2, head_dim=64, groups=2, gamma=0.9)
+    x = synth.make_inputs(w)
+    m = oracle.prefill_masks(x["q"], x["k"], 2, mode=oracle.FIXED_FRACTION, frac_permille=700)
+    items = [(0, h, qb) for h in range(4) for qb in range(4)]
+    ref, lref = oracle.sparse_attn(x["q"], x["k"], x["v"], m["rank"], m["cnt"], 2, items)
+    o0, l0, s0, _ = oracle.sparse_attn_skip(x["q"], x["k"], x["v"], m["rank"], m["cnt"], 2, items, 0.0)
+    assert s0.sum() == 0
+    np.testing.assert_allclose(o0, ref, rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(l0, lref, rtol=1e-12)
+    # a case with skips: decisions passed in replace the oracle's own
+    q, k, v = _skip_inputs()
+    rank, cnt = _full_lists(4, shuffle_seed=4)
+    items = [(0, 0, qb) for qb in range(4)]
+    ref, _ = oracle.sparse_attn(q, k, v, rank, cnt, 1, items)
+    o1, _, s1, _ = oracle.sparse_attn_skip(q, k, v, rank, cnt, 1, items, 0.6)
+    assert s1.sum() > 0
+    o2, _, _, _ = oracle.sparse_attn_skip(q, k, v, rank, cnt, 1, items, 0.6, skip_in=np.zeros_like(s1))
+    np.testing.assert_allclose(o2, ref, rtol=1e-11, atol=1e-13)
+    o3, _, _, _ = oracle.sparse_attn_skip(q, k, v, rank, cnt, 1, items, 0.0, skip_in=s1)
+    np.testing.assert_array_equal(o3, o1)

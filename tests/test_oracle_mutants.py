@@ -26,7 +26,7 @@ MUTANTS = [
     ("rne_ties_away", "double r = nearbyint(x / q) * q;", "double r = round(x / q) * q;"),
     ("scores_no_causal_mask", "            if (j > i) continue;\n            double s = 0.0;",
      "            double s = 0.0;"),
-    ("scores_min_not_max", "            if (s > best) best = s;", "            if (best == -INFINITY || s < best) best = s;"),
+    ("scores_min_not_max", "\n            if (s > best) best = s;", "\n            if (best == -INFINITY || s < best) best = s;"),
     ("scores_no_scale", "            s *= scale;\n            if (s > best) best = s;", "            if (s > best) best = s;"),
     ("mass_not_mean_over_rows", "m[j / BLK] += p / BLK;", "m[j / BLK] += p;"),
     ("mass_no_causal", [("for (int j = 0; j <= i; j++) {\n                    double s = 0.0;",
@@ -57,6 +57,14 @@ MUTANTS = [
      "for (int ii = 0; ii < BLK; ii += stride) {"),
     ("stride_ignored", "for (int ii = stride - 1; ii < BLK; ii += stride) {",
      "for (int ii = 0; ii < BLK; ii++) {"),
+    ("skip_when_any_row_below", "                    if (e > worst) worst = e;",
+     "                    if (worst == -INFINITY || e < worst) worst = e;"),
+    ("skip_running_max_frozen", "                if (mt[ii * n + t] > row_max[ii]) row_max[ii] = mt[ii * n + t];",
+     "                if (t == 0) row_max[ii] = mt[ii * n + t];"),
+    ("skip_block_still_counted", "            use[t] = skip_in ? !skip_in[base + blk[t]] : !own;",
+     "            use[t] = skip_in ? !skip_in[base + blk[t]] : 1;"),
+    ("skip_threshold_log2", "double lnl = (lambda > 0.0) ? log(lambda) : -INFINITY;",
+     "double lnl = (lambda > 0.0) ? log2(lambda) : -INFINITY;"),
 ]
 
 # The pins each mutant runs against (all of them are cheap).
@@ -76,6 +84,9 @@ PINS = [
     T.test_dense_matches_torch_sdpa,
     T.test_sparse_all_equals_dense,
     T.test_sparse_matches_sdpa_with_block_mask,
+    lambda: T.test_skip_brute_force(0.2),
+    T.test_skip_planted_running_max,
+    T.test_skip_sweep_skips_some_and_nests,
     G.test_golden_rank,
     G.test_golden_budget,
 ]
