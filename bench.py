@@ -54,13 +54,16 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="llama8b_n128k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default="llama8b_n128k",
+                    choices=sorted(synth.WORKLOADS) + sorted(synth.EXTRA_WORKLOADS))
     ap.add_argument("--groups", type=int, default=None, help="proxy groups G (default: the workload's)")
     ap.add_argument("--mode", choices=sorted(MODES), default="dynamic")
     ap.add_argument("--gamma", type=float, default=None)
     ap.add_argument("--frac", type=int, default=100, help="fixed budget in per mille of causal blocks")
     ap.add_argument("--score-stride", type=int, default=1, choices=[1, 2, 4, 8],
                     help="query-row stride of the proxy block scores (1: every row)")
+    ap.add_argument("--skip-threshold", type=float, default=0.0,
+                    help="running-max block skip in the attention: lambda in [0, 1] (0: off)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
@@ -143,7 +146,7 @@ class Pipeline:
     """Pre-allocated buffers and ctypes arguments for one layer, so that a step is
     four C-ABI calls with CUDA events between them."""
 
-    def __init__(self, q, k, v, G, mode, gamma, frac, stride=1):
+    def __init__(self, q, k, v, G, mode, gamma, frac, stride=1, skip=0.0):
         import block_sparse_attention_pa_b200 as pa
         self.pa = pa
         self.L = pa.lib()
@@ -152,9 +155,11 @@ class Pipeline:
         self.B, self.N, self.H, self.d, self.G = B, N, H, d, G
         self.nb = N // 128
         self.shape = pa.make_shape(q, k, G)
-        self.budget = pa.make_budget(mode, gamma, frac, stride)
+        self.budget = pa.make_budget(mode, gamma, frac, stride, skip)
         self.mode = mode
         self.stride = stride
+        self.skip = skip
+        self.skipped = None  # uint8 [B, H, T] when counting skipped blocks
         dev = q.device
         self.qp = torch.empty(B, G, N // stride, d, device=dev, dtype=torch.bfloat16)
         self.kp = torch.empty(B, G, N, d, device=dev, dtype=torch.bfloat16)
@@ -182,10 +187,18 @@ class Pipeline:
         pa._check(L.pa_build_mask(sh, bu, self.scores.data_ptr(), self.q.data_ptr(), self.qs, self.k.data_ptr(),
                                   self.ks, ctypes.byref(self.bufs), self.ws.data_ptr(), self.ws.numel(), st))
         if ev: ev[3].record()
-        pa._check(L.pa_block_sparse_attn(sh, self.q.data_ptr(), self.qs, self.k.data_ptr(), self.ks,
-                                         self.v.data_ptr(), self.vs, self.mask.rank.data_ptr(),
-                                         self.mask.cnt.data_ptr(), self.scale, self.o.data_ptr(), self.os_, None,
-                                         st))
+        if self.skip > 0.0:
+            pa._check(L.pa_block_sparse_attn_skip(sh, self.q.data_ptr(), self.qs, self.k.data_ptr(), self.ks,
+                                                  self.v.data_ptr(), self.vs, self.mask.rank.data_ptr(),
+                                                  self.mask.cnt.data_ptr(), self.scale, self.skip, self.o.data_ptr(),
+                                                  self.os_, None,
+                                                  self.skipped.data_ptr() if self.skipped is not None else None,
+                                                  st))
+        else:
+            pa._check(L.pa_block_sparse_attn(sh, self.q.data_ptr(), self.qs, self.k.data_ptr(), self.ks,
+                                             self.v.data_ptr(), self.vs, self.mask.rank.data_ptr(),
+                                             self.mask.cnt.data_ptr(), self.scale, self.o.data_ptr(), self.os_, None,
+                                             st))
         if ev: ev[4].record()
 
     def visited(self):
@@ -196,6 +209,17 @@ class Pipeline:
         per = 4 * 128 * 128 * self.d
         exact = (v - ndiag) * per + ndiag * 4 * self.d * (128 * 129 // 2)
         return v, v * per, exact
+
+    def count_skipped(self) -> int:
+        """One more (untimed) step with a zeroed map of skipped blocks."""
+        if self.skip <= 0.0:
+            return 0
+        self.skipped = torch.zeros(self.B, self.H, self.T, device=self.q.device, dtype=torch.uint8)
+        self.step()
+        torch.cuda.synchronize()
+        n = int(self.skipped.sum().item())
+        self.skipped = None
+        return n
 
 
 def selected_blocks(pipe) -> torch.Tensor:
@@ -271,14 +295,15 @@ def counters_for(kernel_key: str, source_files):
     return c
 
 
-def traffic_for(ctr, w, G, mode, gamma):
+def traffic_for(ctr, w, G, mode, gamma, stride=1, skip=0.0):
     """DRAM bytes per launch from the committed capture, only for the exact
     workload and budget it was taken on (traffic does not scale linearly)."""
     if not ctr:
         return None
     same = (ctr.get("workload") == w.name and ctr.get("groups") == G and
             ctr.get("mode") == {0: "dynamic", 1: "fixed", 2: "all"}[mode] and
-            (mode != 0 or abs(ctr.get("gamma", -1) - gamma) < 1e-9))
+            (mode != 0 or abs(ctr.get("gamma", -1) - gamma) < 1e-9) and
+            ctr.get("score_stride", 1) == stride and ctr.get("skip_threshold", 0.0) == skip)
     return float(ctr["dram_bytes"]) if same else None
 
 
@@ -286,7 +311,7 @@ ATTN_SOURCES = ["block_sparse_attention_pa_b200/csrc/attn.cuh", "block_sparse_at
 
 
 # ------------------------------------------------------------ CPU oracle
-def oracle_estimate(x, w: synth.Workload, G, mode, gamma, frac, size="baseline", seed=0, stride=1):
+def oracle_estimate(x, w: synth.Workload, G, mode, gamma, frac, size="baseline", seed=0, stride=1, skip=0.0):
     """Time the CPU oracle on a bounded sample of one layer and extrapolate to
     ms per layer.  x: CPU bf16 tensors.  Returns (ms_per_layer, per-stage
     seconds, description of the sample)."""
@@ -334,7 +359,10 @@ def oracle_estimate(x, w: synth.Workload, G, mode, gamma, frac, size="baseline",
     # o5 sparse attention on random (b, h, qb) items, extrapolated per visited block
     items = [(int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(nb))) for _ in range(n_items)]
     t0 = time.perf_counter()
-    oracle.sparse_attn(q, k, v, rank, cnt, G, items)
+    if skip > 0.0:
+        oracle.sparse_attn_skip(q, k, v, rank, cnt, G, items, skip)
+    else:
+        oracle.sparse_attn(q, k, v, rank, cnt, G, items)
     dt = time.perf_counter() - t0
     blocks = sum(int(cnt[b, h, qb]) for b, h, qb in items)
     det["attn_s"] = dt * float(cnt.sum()) / max(blocks, 1)
@@ -353,7 +381,7 @@ def run_reference(args, w, G, mode, gamma, frac):
     vals = []
     for i in range(args.warmup + args.steps):
         ms, det, sample = oracle_estimate(x, w, G, mode, gamma, frac, size="step", seed=i,
-                                          stride=args.score_stride)
+                                          stride=args.score_stride, skip=args.skip_threshold)
         if i >= args.warmup:
             vals.append(ms)
     v = statistics.mean(vals)
@@ -361,24 +389,24 @@ def run_reference(args, w, G, mode, gamma, frac):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "ms/layer", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": v, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_of(w, G, mode, gamma, frac, args.score_stride),
+            "config": config_of(w, G, mode, gamma, frac, args.score_stride, args.skip_threshold),
             "cpu_baseline": {"value": v, "unit": "ms/layer", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "ms/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def config_of(w, G, mode, gamma, frac, stride=1):
+def config_of(w, G, mode, gamma, frac, stride=1, skip=0.0):
     budget = {0: f"dynamic gamma={gamma}", 1: f"fixed {frac / 10:.1f}% of causal blocks", 2: "all causal blocks"}[mode]
     return {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "q_heads": w.num_q_heads,
             "kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "groups": G, "budget": budget, "block": 128,
-            "score_stride": stride,
+            "score_stride": stride, "skip_threshold": skip,
             "l2": "inputs larger than L2 (q+k+v per layer > 126 MB), no flush"}
 
 
 # ------------------------------------------------------------------- main
 def main():
     args = parse_args()
-    w = synth.WORKLOADS[args.workload]
+    w = {**synth.WORKLOADS, **synth.EXTRA_WORKLOADS}[args.workload]
     G = args.groups or w.num_groups
     mode = MODES[args.mode]
     gamma = args.gamma if args.gamma is not None else w.gamma
@@ -402,7 +430,8 @@ def main():
     x = synth.make_inputs(w, device=f"cuda:{local}", seed=w.seed + rank)
     q, k, v = x["q"], x["k"], x["v"]
     stride = args.score_stride
-    pipe = Pipeline(q, k, v, G, mode, gamma, frac, stride)
+    skip = args.skip_threshold
+    pipe = Pipeline(q, k, v, G, mode, gamma, frac, stride, skip)
     sampler = None if args.no_clocks else ClockSampler(local)
     total_ms, stages, clocks = time_pipeline(pipe, args.steps, args.warmup, dist_on, sampler)
     status = pa.device_status()
@@ -417,15 +446,20 @@ def main():
     est_ms = float(stages[:3].sum())
     attn_ms = float(stages[3])
 
+    # with the block skip a skipped tile runs its QK product only
+    n_skipped = pipe.count_skipped()
+    flops_exec = flops - n_skipped * 2 * 128 * 128 * w.head_dim
+
     peaks, peaks_kind = load_peaks()
-    achieved = flops / (attn_ms * 1e-3) / 1e12
+    achieved = flops_exec / (attn_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     ctr = counters_for("attn_kernel", ATTN_SOURCES)
-    traffic = traffic_for(ctr, w, G, mode, gamma)
+    traffic = traffic_for(ctr, w, G, mode, gamma, stride, skip)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "traffic": traffic, "kernel": "attn_kernel<128> (block-sparse attention)",
                 "peak_kind": f"{peaks_kind} bf16 sustained (kernel timed inside back-to-back steps)",
-                "flops_per_launch": flops, "exact_causal_flops_per_launch": flops_exact}
+                "flops_per_launch": flops_exec, "visited_tile_flops_per_launch": flops,
+                "exact_causal_flops_per_launch": flops_exact}
 
     # per-stage rooflines
     d = w.head_dim
@@ -446,10 +480,11 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded needle/sink generator; random inputs, no weights)",
-            "config": config_of(w, G, mode, gamma, frac, stride) | {"parallelism": f"replicas x{world}"},
+            "config": config_of(w, G, mode, gamma, frac, stride, skip) | {"parallelism": f"replicas x{world}"},
             "est_ms": est_ms, "sparse_ms": attn_ms,
-            "tflops_effective": achieved, "tflops_exact_causal": flops_exact / (attn_ms * 1e-3) / 1e12,
+            "tflops_effective": flops / (attn_ms * 1e-3) / 1e12, "tflops_exact_causal": flops_exact / (attn_ms * 1e-3) / 1e12,
             "visited_blocks": visited, "density": density, "sparsity": 1.0 - density,
+            "skipped_blocks": n_skipped, "skip_fraction_of_visited": n_skipped / max(visited, 1),
             "stages_ms": {"pool": float(stages[0]), "scores": float(stages[1]), "mask": float(stages[2]),
                           "attn": attn_ms},
             "stage_roofline": stage_roofline, "roofline": roofline,
@@ -471,6 +506,16 @@ def main():
         line["estimate_frac_of_dense"] = est_ms / dense_attn
         del dense
 
+    # what the block skip changes in O: the same mask without skipping
+    if skip > 0.0:
+        plain = Pipeline(q, k, v, G, mode, gamma, frac, stride, 0.0)
+        plain.step()
+        pipe.step()
+        torch.cuda.synchronize()
+        diff = (pipe.o.float() - plain.o.float()).abs_()
+        line["skip_o_error_vs_no_skip"] = {"max_abs": float(diff.max().item()), "mean_abs": float(diff.mean().item())}
+        del plain, diff
+
     # the strided estimate's selection against the every-row estimate's
     if stride > 1:
         every = Pipeline(q, k, v, G, mode, gamma, frac, 1)
@@ -486,14 +531,14 @@ def main():
 
     # end to end through the public API with pinned host buffers
     if not args.no_e2e:
-        e2e = run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world, stride)
+        e2e = run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world, stride, skip)
         line["e2e"] = e2e
 
     # the CPU oracle on a bounded sample (rank 0, one GPU only)
     if not args.no_cpu_baseline and world == 1 and rank == 0:
         import oracle
         xc = {n: x[n].cpu() for n in ("q", "k", "v")}
-        ms, det, sample = oracle_estimate(xc, w, G, mode, gamma, frac, size="baseline", stride=stride)
+        ms, det, sample = oracle_estimate(xc, w, G, mode, gamma, frac, size="baseline", stride=stride, skip=skip)
         line["cpu_baseline"] = {"value": ms, "unit": "ms/layer", "cores": oracle.num_threads(), "kind": "oracle",
                                 "sample": sample, "stage_s": det}
 
@@ -504,7 +549,7 @@ def main():
         torch.distributed.destroy_process_group()
 
 
-def run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world, stride=1):
+def run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world, stride=1, skip=0.0):
     """The metric through the public API with host buffers, as a user runs
     consecutive layers: every step copies its q, k, v from pinned host memory
     and reads its o back.  Two device buffer sets and two copy streams let the
@@ -513,7 +558,7 @@ def run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world, stride=1):
     q, k, v = x["q"], x["k"], x["v"]
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
     bufs = [tuple(torch.empty_like(t) for t in (q, k, v, q)) for _ in range(2)]
-    call = pa.Prefill(bufs[0][0], bufs[0][1], bufs[0][2], G, mode, gamma, frac, stride)
+    call = pa.Prefill(bufs[0][0], bufs[0][1], bufs[0][2], G, mode, gamma, frac, stride, skip)
     ho = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(2)]
     ms = torch.cuda.current_stream()
     hs, ds = torch.cuda.Stream(), torch.cuda.Stream()

@@ -32,7 +32,7 @@ STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_E
 ENTRY_POINTS = ("pa_workspace_size", "pa_pool_heads", "pa_block_scores", "pa_build_mask",
                 "pa_block_sparse_attn", "pa_prefill", "pa_get_device_status", "pa_status_string",
                 "pa_last_error", "pa_abi_version", "pa_build_mask_noalloc", "pa_selftest_wait_timeout",
-                "pa_pool_heads_strided", "pa_block_scores_strided")
+                "pa_pool_heads_strided", "pa_block_scores_strided", "pa_block_sparse_attn_skip")
 
 SCORE_STRIDES = (1, 2, 4, 8)
 
@@ -55,7 +55,7 @@ class Strides(ctypes.Structure):
 
 class Budget(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("gamma", ctypes.c_float), ("frac_permille", ctypes.c_int32),
-                ("score_stride", ctypes.c_int32)]
+                ("score_stride", ctypes.c_int32), ("skip_threshold", ctypes.c_float)]
 
 
 class MaskBufs(ctypes.Structure):
@@ -84,6 +84,8 @@ def lib() -> ctypes.CDLL:
         L.pa_block_scores_strided.argtypes = [P(Shape), ctypes.c_int32, vp, vp, vp, vp]
         L.pa_build_mask.argtypes = [P(Shape), P(Budget), vp, vp, st, vp, st, P(MaskBufs), vp, ctypes.c_size_t, vp]
         L.pa_block_sparse_attn.argtypes = [P(Shape), vp, st, vp, st, vp, st, vp, vp, ctypes.c_float, vp, st, vp, vp]
+        L.pa_block_sparse_attn_skip.argtypes = [P(Shape), vp, st, vp, st, vp, st, vp, vp, ctypes.c_float,
+                                                ctypes.c_float, vp, st, vp, vp, vp]
         L.pa_prefill.argtypes = [P(Shape), P(Budget), vp, st, vp, st, vp, st, vp, st, P(MaskBufs), vp,
                                  ctypes.c_size_t, vp]
         L.pa_get_device_status.argtypes = [vp, ctypes.c_int]
@@ -94,7 +96,7 @@ def lib() -> ctypes.CDLL:
         L.pa_abi_version.restype = ctypes.c_int32
         for name in ("pa_pool_heads", "pa_block_scores", "pa_build_mask", "pa_block_sparse_attn", "pa_prefill",
                      "pa_get_device_status", "pa_selftest_wait_timeout", "pa_pool_heads_strided",
-                     "pa_block_scores_strided"):
+                     "pa_block_scores_strided", "pa_block_sparse_attn_skip"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -126,8 +128,9 @@ def make_shape(q: torch.Tensor, k: torch.Tensor, num_groups: int) -> Shape:
     return Shape(B, N, H, k.shape[2], d, 128, num_groups)
 
 
-def make_budget(mode: int = DYNAMIC, gamma: float = 0.95, frac_permille: int = 0, score_stride: int = 1) -> Budget:
-    return Budget(mode, gamma, frac_permille, score_stride)
+def make_budget(mode: int = DYNAMIC, gamma: float = 0.95, frac_permille: int = 0, score_stride: int = 1,
+                skip_threshold: float = 0.0) -> Budget:
+    return Budget(mode, gamma, frac_permille, score_stride, skip_threshold)
 
 
 def workspace_size(shape: Shape, budget: Budget) -> int:
@@ -219,31 +222,43 @@ def build_mask(scores: torch.Tensor, q: torch.Tensor, k: torch.Tensor, num_group
 
 
 def block_sparse_attn(q, k, v, rank, cnt, num_groups: int, softmax_scale: float | None = None,
-                      out: torch.Tensor | None = None, return_lse: bool = False):
-    """pa_block_sparse_attn -> o (bf16 [B, N, H, d]) [, lse fp32 [B, H, N]]."""
+                      out: torch.Tensor | None = None, return_lse: bool = False, skip_threshold: float = 0.0,
+                      return_skipped: bool = False):
+    """pa_block_sparse_attn (skip_threshold 0) or pa_block_sparse_attn_skip ->
+    o (bf16 [B, N, H, d]) [, lse fp32 [B, H, N]] [, skipped uint8 [B, H, T]]."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _cuda_bf16(t, n)
     shape = make_shape(q, k, num_groups)
     B, N, H, d = q.shape
+    nb = N // 128
     scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
     o = torch.empty_like(q, memory_format=torch.contiguous_format) if out is None else out
     lse = torch.empty(B, H, N, device=q.device, dtype=torch.float32) if return_lse else None
-    _check(lib().pa_block_sparse_attn(ctypes.byref(shape), q.data_ptr(), _strides(q), k.data_ptr(), _strides(k),
-                                      v.data_ptr(), _strides(v), rank.data_ptr(), cnt.data_ptr(), scale,
-                                      o.data_ptr(), _strides(o), lse.data_ptr() if lse is not None else None,
-                                      _stream(q.device)))
-    return (o, lse) if return_lse else o
+    skipped = torch.zeros(B, H, nb * (nb + 1) // 2, device=q.device, dtype=torch.uint8) if return_skipped else None
+    lse_p = lse.data_ptr() if lse is not None else None
+    if skip_threshold == 0.0 and not return_skipped:
+        _check(lib().pa_block_sparse_attn(ctypes.byref(shape), q.data_ptr(), _strides(q), k.data_ptr(), _strides(k),
+                                          v.data_ptr(), _strides(v), rank.data_ptr(), cnt.data_ptr(), scale,
+                                          o.data_ptr(), _strides(o), lse_p, _stream(q.device)))
+    else:
+        _check(lib().pa_block_sparse_attn_skip(ctypes.byref(shape), q.data_ptr(), _strides(q), k.data_ptr(),
+                                               _strides(k), v.data_ptr(), _strides(v), rank.data_ptr(),
+                                               cnt.data_ptr(), scale, skip_threshold, o.data_ptr(), _strides(o),
+                                               lse_p, skipped.data_ptr() if skipped is not None else None,
+                                               _stream(q.device)))
+    res = (o,) + ((lse,) if return_lse else ()) + ((skipped,) if return_skipped else ())
+    return res if len(res) > 1 else o
 
 
 class Prefill:
     """A reusable pa_prefill call: workspace and mask buffers allocated once."""
 
     def __init__(self, q, k, v, num_groups: int, mode: int = DYNAMIC, gamma: float = 0.95, frac_permille: int = 0,
-                 score_stride: int = 1):
+                 score_stride: int = 1, skip_threshold: float = 0.0):
         for t, n in ((q, "q"), (k, "k"), (v, "v")):
             _cuda_bf16(t, n)
         self.shape = make_shape(q, k, num_groups)
-        self.budget = make_budget(mode, gamma, frac_permille, score_stride)
+        self.budget = make_budget(mode, gamma, frac_permille, score_stride, skip_threshold)
         self.mask = Mask.empty(self.shape, q.device, mode == DYNAMIC)
         self.ws = torch.empty(workspace_size(self.shape, self.budget), device=q.device, dtype=torch.uint8)
         self._bufs = self.mask.bufs()
@@ -257,9 +272,9 @@ class Prefill:
 
 
 def prefill(q, k, v, num_groups: int, mode: int = DYNAMIC, gamma: float = 0.95, frac_permille: int = 0,
-            score_stride: int = 1):
+            score_stride: int = 1, skip_threshold: float = 0.0):
     """pa_prefill -> (o, Mask)."""
-    call = Prefill(q, k, v, num_groups, mode, gamma, frac_permille, score_stride)
+    call = Prefill(q, k, v, num_groups, mode, gamma, frac_permille, score_stride, skip_threshold)
     o = torch.empty_like(q, memory_format=torch.contiguous_format)
     call(q, k, v, o)
     return o, call.mask

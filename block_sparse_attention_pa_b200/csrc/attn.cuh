@@ -26,6 +26,13 @@
 //              than 2^8 (then O is rescaled in TMEM), final O/l and LSE.
 // TMEM columns: S_0 [0,128)  S_1 [128,256)  O_0 [256,384)  O_1 [384,512);
 // P_t (bf16 pairs) overwrites the first 64 columns of S_t.
+//
+// SKIP = true adds BLASST's running-max block skip (BLASST introduction and
+// 3.1): a visited block after the first whose row maxima all lie below the
+// rows' running maxima (over the blocks visited before, in ascending order)
+// by more than -log2(lambda) is dropped -- no exponentials, no P, no PV.  The
+// four warps of a head take the block-level decision by a bounded vote in
+// shared memory; the MMA warp reads it after the head's p_full barrier.
 #pragma once
 #include "sm100.cuh"
 
@@ -60,6 +67,8 @@ struct AttnParams {
     __nv_bfloat16 *o;
     int64_t osb, oss, osh;
     float *lse;                // [B][H][N] or nullptr
+    float skip_log2;           // SKIP: log2(lambda) (lambda in (0, 1])
+    uint8_t *skipped;          // SKIP: [B][H][T], 1 written for every skipped block, or nullptr
     uint64_t timeout_ns;
     int16_t unit_h0[kMaxHeads];
     int16_t unit_h1[kMaxHeads];  // -1: the unit has one head
@@ -80,6 +89,44 @@ __device__ __forceinline__ int next_block(const uint32_t *a, const uint32_t *b, 
     return (w << 5) + __ffs(static_cast<int>(m)) - 1;
 }
 
+// Block-level vote of the four warps of one head: true when every row of the
+// query block votes yes.  Each warp publishes (tile << 1 | its vote) in its
+// own slot; lanes 0-3 poll the four slots until all carry this tile's tag.
+// The poll is bounded like every other wait: on a timeout (or the CTA's abort
+// flag) `ok` is false for the whole warp.
+__device__ __forceinline__ bool head_vote_all(volatile uint32_t *slots, int q4, uint32_t tile, bool vote,
+                                              const WaitCtl &w, bool &ok) {
+    const uint32_t lane = lane_id();
+    const bool wv = __all_sync(0xffffffffu, vote);
+    if (lane == 0) {
+        slots[q4] = (tile << 1) | (wv ? 1u : 0u);
+        __threadfence_block();
+    }
+    __syncwarp();
+    bool yes = true, good = true;
+    if (lane < 4) {
+        const uint64_t t0 = globaltimer();
+        for (uint32_t it = 0;; ++it) {
+            const uint32_t v = slots[lane];
+            if ((v >> 1) == tile) {
+                yes = (v & 1u) != 0u;
+                break;
+            }
+            if ((it & 31u) == 31u) {
+                if (*w.abort) { good = false; break; }
+                if (globaltimer() - t0 > w.timeout_ns || it > (1u << 30)) {
+                    *w.abort = 1;
+                    flag_status(kStTimeout);
+                    good = false;
+                    break;
+                }
+            }
+        }
+    }
+    ok = __all_sync(0xffffffffu, good);
+    return __all_sync(0xffffffffu, yes);
+}
+
 template <int D>
 struct AttnSmem {
     static constexpr int TB = 128 * D * 2;
@@ -87,7 +134,7 @@ struct AttnSmem {
     static constexpr int BYTES = (2 + 2 * KS) * TB + 1024 + 512 + 1024;  // + two 4096-bit block bitmaps
 };
 
-template <int D>
+template <int D, bool SKIP>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
@@ -114,6 +161,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint64_t *v_empty = bars + 8 + 3 * KS;   // KS
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8 + 4 * KS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile uint32_t *vote = tmem_slot + 4;        // SKIP: [2 heads][4 warps] tagged votes
+    volatile uint32_t *skip_flag = tmem_slot + 12;  // SKIP: [2 heads][2 tile parities]
     uint32_t *bm = reinterpret_cast<uint32_t *>(smem + (2 + 2 * KS) * TB + 512);  // [2][128] block bitmaps
 
     // ------------------------------------------------------------ work item
@@ -179,6 +228,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(&v_empty[s], 1);
         }
         *abort_flag = 0;
+        for (int x = 0; x < 8; ++x) vote[x] = 0xFFFFFFFFu;  // a tag no tile carries
+        for (int x = 0; x < 4; ++x) skip_flag[x] = 0u;
         fence_mbar_init();
     }
     if (warp == kProducerWarp && lane == 0) {
@@ -267,7 +318,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 umma_commit(&o_done[t]);
             };
             auto active = [&](int t, int kb) { return (bm[t * 128 + (kb >> 5)] >> (kb & 31)) & 1u; };
-            int pv_done0 = 0, pv_done1 = 0;
+            int seen0 = 0, seen1 = 0;  // tiles of each head whose P was handed over
+            int pv0 = 0, pv1 = 0;      // SKIP: PV products issued for each head
             bool ok = mbar_wait(q_full, 0, wc) && mbar_wait(&k_full[0], 0, wc);
             if (ok) {
                 tc_fence_after();
@@ -286,11 +338,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 tc_fence_after();
                 for (int t = 0; t < 2; ++t) {
                     if (active(t, kb)) {
-                        int &pv_done = t ? pv_done1 : pv_done0;
-                        if (!mbar_wait(&p_full[t], pv_done & 1, wc)) { ok = false; break; }
+                        int &seen = t ? seen1 : seen0;
+                        int &pv = t ? pv1 : pv0;
+                        if (!mbar_wait(&p_full[t], seen & 1, wc)) { ok = false; break; }
                         tc_fence_after();
-                        issue_pv(t, s, pv_done > 0);
-                        ++pv_done;
+                        if constexpr (SKIP) {
+                            const bool skipped = skip_flag[t * 2 + (seen & 1)] != 0u;
+                            ++seen;
+                            if (!skipped) {
+                                issue_pv(t, s, pv > 0);
+                                ++pv;
+                            }
+                        } else {
+                            issue_pv(t, s, seen > 0);  // without skipping every tile has its PV
+                            ++seen;
+                        }
                     }
                     if (has_next && active(t, kb_next)) issue_qk(t, s1);
                 }
@@ -318,9 +380,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t s_addr = lane_base + t * 128;
         const uint32_t o_addr = lane_base + 256 + t * 128;
         float m = -INFINITY, l = 0.0f;
+        float mtrue = -INFINITY;  // SKIP: exact running max (log2 units) of the tiles visited
+        const long long skip_base = (static_cast<long long>(b) * p.H + h) * T + static_cast<long long>(qb) * (qb + 1) / 2;
         bool ok = true;
         uint32_t s[128];
-        int i = 0;  // tiles of this head so far
+        int i = 0;    // tiles of this head so far
+        int npv = 0;  // of them, tiles whose PV product was issued (o_done phases)
         for (int kb = next_block(bmt, bmt, 0, words); kb >= 0; kb = next_block(bmt, bmt, kb + 1, words), ++i) {
             if (!warp_wait(&s_full[t], i & 1, wc)) { ok = false; break; }
             tc_fence_after();
@@ -343,13 +408,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const float mt = p.scale_log2 *
                 fmax3(fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmax3(mx[6], mx[7], mx[8])),
                       fmax3(mx[9], mx[10], mx[11]), fmax3(mx[12], mx[13], fmaxf(mx[14], mx[15])));
+            if constexpr (SKIP) {
+                bool skip = false;
+                if (i > 0) {
+                    bool vote_ok = true;
+                    skip = head_vote_all(vote + t * 4, q4, static_cast<uint32_t>(i), mt < mtrue + p.skip_log2, wc,
+                                         vote_ok);
+                    if (!vote_ok) { ok = false; break; }
+                }
+                mtrue = fmaxf(mtrue, mt);
+                if (row == 0) skip_flag[t * 2 + (i & 1)] = skip ? 1u : 0u;
+                if (skip) {
+                    // nothing of this tile enters O or l; S is free for the next QK
+                    if (row == 0 && p.skipped) p.skipped[skip_base + kb] = 1;
+                    tc_fence_before();
+                    mbar_arrive(&p_full[t]);
+                    continue;
+                }
+            }
             const float m_new = fmaxf(m, mt);
             if (i > 0) {
                 const bool need = m_new > m + 8.0f;
                 if (__any_sync(0xffffffffu, need)) {
                     // raise the running max: O (in TMEM) and l scale by 2^(m - m_new)
                     const float alpha = (m == -INFINITY) ? 0.0f : ex2(m - m_new);
-                    if (!warp_wait(&o_done[t], (i - 1) & 1, wc)) { ok = false; break; }
+                    if (!warp_wait(&o_done[t], ((SKIP ? npv : i) - 1) & 1, wc)) { ok = false; break; }
                     tc_fence_after();
 #pragma unroll
                     for (int ch = 0; ch < D / 32; ++ch) {
@@ -409,9 +492,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&p_full[t]);
+            if constexpr (SKIP) ++npv;
         }
         // epilogue: O / l -> bf16 -> global; LSE
-        const int ct = i;
+        const int ct = SKIP ? npv : i;
         if (ct > 0 && ok && warp_wait(&o_done[t], (ct - 1) & 1, wc)) {
             tc_fence_after();
             const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;

@@ -89,8 +89,15 @@ pa_status check_stride(int r) {
 // pa_budget.score_stride with 0 (a zero-initialised struct) read as 1.
 int stride_of(const pa_budget *bu) { return (bu && bu->score_stride > 0) ? bu->score_stride : 1; }
 
+pa_status check_skip(float lambda) {
+    if (!(lambda >= 0.0f && lambda <= 1.0f))
+        return fail(PA_ERR_INVALID_ARG, "skip_threshold must be in [0, 1] (got %g)", static_cast<double>(lambda));
+    return PA_OK;
+}
+
 pa_status check_budget(const pa_budget *bu) {
     if (!bu) return fail(PA_ERR_INVALID_ARG, "budget is NULL");
+    if (check_skip(bu->skip_threshold)) return PA_ERR_INVALID_ARG;
     if (bu->score_stride != 0 && check_stride(bu->score_stride)) return PA_ERR_INVALID_ARG;
     if (bu->mode == PA_BUDGET_DYNAMIC) {
         if (!(bu->gamma > 0.0f && bu->gamma <= 1.0f))
@@ -327,10 +334,10 @@ int build_units(const pa_shape *s, int16_t *h0, int16_t *h1) {
     return n;
 }
 
-template <int D>
+template <int D, bool SKIP>
 pa_status launch_attn_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv, const pa::AttnParams &p,
                         cudaStream_t st) {
-    auto kern = pa::attn_kernel<D>;
+    auto kern = pa::attn_kernel<D, SKIP>;
     const int smem = pa::AttnSmem<D>::BYTES;
     PA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     // The kernel's warpgroups re-split the registers it is launched with; the
@@ -346,9 +353,10 @@ pa_status launch_attn_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUte
     return PA_OK;
 }
 
+// skip_threshold: BLASST's lambda in [0, 1] (0: no skipping, the plain kernel)
 pa_status launch_attn(const pa_shape *s, const void *q, pa_strides qs, const void *k, pa_strides ks, const void *v,
                       pa_strides vs, const int32_t *rank, const int32_t *cnt, float scale, void *o, pa_strides os,
-                      float *lse, cudaStream_t st) {
+                      float *lse, float skip_threshold, uint8_t *skipped, cudaStream_t st) {
     const int B = s->batch, H = s->num_q_heads, Hkv = s->num_kv_heads, N = s->seqlen, d = s->head_dim;
     CUtensorMap mq, mk, mv;
     pa_status r = map_bnhd(&mq, q, B, N, H, d, qs, "q");
@@ -373,7 +381,12 @@ pa_status launch_attn(const pa_shape *s, const void *q, pa_strides qs, const voi
     p.osb = os.b; p.oss = os.s; p.osh = os.h;
     p.lse = lse;
     p.timeout_ns = wait_timeout_ns();
-    return d == 128 ? launch_attn_t<128>(mq, mk, mv, p, st) : launch_attn_t<64>(mq, mk, mv, p, st);
+    const bool skip = skip_threshold > 0.0f;
+    p.skip_log2 = skip ? static_cast<float>(std::log2(static_cast<double>(skip_threshold))) : -INFINITY;
+    p.skipped = skip ? skipped : nullptr;
+    if (skip)
+        return d == 128 ? launch_attn_t<128, true>(mq, mk, mv, p, st) : launch_attn_t<64, true>(mq, mk, mv, p, st);
+    return d == 128 ? launch_attn_t<128, false>(mq, mk, mv, p, st) : launch_attn_t<64, false>(mq, mk, mv, p, st);
 }
 
 pa_status check_mask(const pa_mask *m, const pa_budget *bu, bool need_rank_cnt) {
@@ -469,6 +482,25 @@ pa_status pa_build_mask(const pa_shape *shape, const pa_budget *budget, const fl
     return ok();
 }
 
+pa_status pa_block_sparse_attn_skip(const pa_shape *shape, const void *q, pa_strides qs, const void *k,
+                                    pa_strides ks, const void *v, pa_strides vs, const int32_t *rank,
+                                    const int32_t *cnt, float softmax_scale, float skip_threshold, void *o,
+                                    pa_strides os, float *lse, uint8_t *skipped, pa_stream_t stream) {
+    pa_status r;
+    if ((r = check_shape(shape)) || (r = check_skip(skip_threshold))) return r;
+    if ((r = check_tensor(q, qs, "q")) || (r = check_tensor(k, ks, "k")) || (r = check_tensor(v, vs, "v")) ||
+        (r = check_tensor(o, os, "o")))
+        return r;
+    if ((r = check_ptr(rank, "rank", 4)) || (r = check_ptr(cnt, "cnt", 4))) return r;
+    if (lse && (r = check_ptr(lse, "lse", 4))) return r;
+    if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale))
+        return fail(PA_ERR_INVALID_ARG, "softmax_scale must be positive and finite");
+    if ((r = launch_attn(shape, q, qs, k, ks, v, vs, rank, cnt, softmax_scale, o, os, lse, skip_threshold, skipped,
+                         reinterpret_cast<cudaStream_t>(stream))))
+        return r;
+    return ok();
+}
+
 pa_status pa_block_sparse_attn(const pa_shape *shape, const void *q, pa_strides qs, const void *k, pa_strides ks,
                                const void *v, pa_strides vs, const int32_t *rank, const int32_t *cnt,
                                float softmax_scale, void *o, pa_strides os, float *lse, pa_stream_t stream) {
@@ -481,7 +513,7 @@ pa_status pa_block_sparse_attn(const pa_shape *shape, const void *q, pa_strides 
     if (lse && (r = check_ptr(lse, "lse", 4))) return r;
     if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale))
         return fail(PA_ERR_INVALID_ARG, "softmax_scale must be positive and finite");
-    if ((r = launch_attn(shape, q, qs, k, ks, v, vs, rank, cnt, softmax_scale, o, os, lse,
+    if ((r = launch_attn(shape, q, qs, k, ks, v, vs, rank, cnt, softmax_scale, o, os, lse, 0.0f, nullptr,
                          reinterpret_cast<cudaStream_t>(stream))))
         return r;
     return ok();
@@ -515,7 +547,8 @@ pa_status pa_prefill(const pa_shape *shape, const pa_budget *budget, const void 
     if ((r = launch_budget(shape, budget, mask_out->rank, mask_out->mass, mask_out->cnt, mask_out->budget, st)))
         return r;
     const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(shape->head_dim)));
-    if ((r = launch_attn(shape, q, qs, k, ks, v, vs, mask_out->rank, mask_out->cnt, scale, o, os, nullptr, st)))
+    if ((r = launch_attn(shape, q, qs, k, ks, v, vs, mask_out->rank, mask_out->cnt, scale, o, os, nullptr,
+                         budget->skip_threshold, nullptr, st)))
         return r;
     return ok();
 }

@@ -17,6 +17,11 @@ workloads on the ProxyAttn pages, "5. Experiments"; there is no dataset here):
 * ``n_needles`` positions are drawn without replacement from ``[1, N)`` and
   ``K[:, pos, kvh] += 2.0 * u_{dir(kvh)}`` for every KV head.
 * ``K[:, 0] *= 4`` (an attention sink).
+* Optional, for the running-max block skip only (``sink_logit`` > 0, a
+  labelled extra, never one of the five workloads below): ``K[:, 0, kvh] +=
+  (sink_logit * sqrt(d) / 2) * u_{dir(kvh)}``, which lifts the sink's scaled
+  logit of head h by about ``s_h * sink_logit`` above the other keys, the way
+  trained models concentrate attention on their first token.
 * Everything is drawn in fp32 with a seeded ``torch.Generator`` on ``device``
   and cast to bf16 (round to nearest even).  A given (workload, seed, device
   type) always yields the same tensors.
@@ -43,6 +48,7 @@ class Workload:
     per_head_sharpness: bool
     per_group_direction: bool
     seed: int
+    sink_logit: float = 0.0
 
     @property
     def nb(self) -> int:
@@ -60,6 +66,13 @@ WORKLOADS = {
     "llama8b_n128k": Workload("llama8b_n128k", 1, 131072, 32, 8, 128, 1, 0.95, 256, True, False, 1236),
     "qwen7b_n64k": Workload("qwen7b_n64k", 1, 65536, 28, 4, 128, 4, 0.9, 0, True, True, 1237),
     "llama8b_n256k": Workload("llama8b_n256k", 1, 262144, 32, 8, 128, 1, 0.95, 512, True, False, 1238),
+}
+
+# Labelled extra for the running-max block skip: the 128K Llama shape with a
+# strong attention sink (see ``sink_logit`` above).
+EXTRA_WORKLOADS = {
+    "llama8b_n128k_sink": Workload("llama8b_n128k_sink", 1, 131072, 32, 8, 128, 1, 0.95, 256, True, False, 1239,
+                                   sink_logit=4.0),
 }
 
 
@@ -92,6 +105,8 @@ def make_inputs(w: Workload, device="cpu", seed: int | None = None):
     else:
         needles = torch.zeros(0, dtype=torch.long, device=dev)
     k[:, 0] *= 4.0
+    if w.sink_logit > 0.0:
+        k[:, 0] += (w.sink_logit * d ** 0.5 / 2.0 * u[kv_dir])[None]
     return dict(
         q=q.to(torch.bfloat16),
         k=k.to(torch.bfloat16),
@@ -102,8 +117,8 @@ def make_inputs(w: Workload, device="cpu", seed: int | None = None):
 
 
 def small_workload(seqlen=512, heads=4, kv_heads=2, head_dim=64, groups=1, gamma=0.9,
-                   needles=8, batch=1, seed=7, sharp=True, per_group=False) -> Workload:
+                   needles=8, batch=1, seed=7, sharp=True, per_group=False, sink_logit=0.0) -> Workload:
     """A small custom workload for parity tests (sizes the oracle finishes in seconds)."""
     return Workload(f"custom_n{seqlen}_h{heads}_kv{kv_heads}_d{head_dim}_g{groups}",
                     batch, seqlen, heads, kv_heads, head_dim, groups, gamma, needles,
-                    sharp, per_group, seed)
+                    sharp, per_group, seed, sink_logit)

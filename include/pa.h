@@ -95,6 +95,9 @@ typedef struct pa_budget {
                               scores every row; 2, 4 or 8 scores only rows
                               i with i mod r == r-1 (pa_block_scores_strided).
                               Used by pa_prefill and pa_workspace_size. */
+    float skip_threshold;  /* BLASST block skip in the attention of pa_prefill
+                              (pa_block_sparse_attn_skip): lambda in [0, 1],
+                              0 = off */
 } pa_budget;
 
 /* Mask buffers written by pa_build_mask / pa_prefill (device, caller-owned).
@@ -227,9 +230,36 @@ PA_API pa_status pa_block_sparse_attn(const pa_shape *shape,
                                void *o, pa_strides o_strides, float *lse,
                                pa_stream_t stream);
 
+/* pa_block_sparse_attn with BLASST's running-max block skip (BLASST,
+ * introduction and "3.1 pruning attention with the running max": a block
+ * whose scores all lie far below the running maximum contributes almost
+ * nothing after the softmax, so its exponentials and its V product are
+ * skipped).  The rule's own text is cut off on the pages; as implemented:
+ * the blocks of (b, h, qb) are visited in ascending block index; with M_i the
+ * running max of row i's scaled logits over the blocks visited before, a
+ * block after the first is skipped when for every row i of the query block
+ *     max_{j in block, j <= i} softmax_scale * q_i . k_j  <  M_i + ln(lambda)
+ * and the output is the softmax attention over the keys of the blocks kept
+ * (lse likewise).  skip_threshold = lambda in [0, 1]; 0 never skips and runs
+ * exactly pa_block_sparse_attn.  The comparison runs in fp32 on the tensor
+ * core's fp32 logits, so a block within rounding of the threshold may be
+ * decided either way.  skipped (nullable): uint8 [B][H][T]; the kernel writes
+ * 1 at tri(qb)+kb for every block it skips and leaves other entries as they
+ * are (zero it first).  K and V of a skipped block are still loaded: the
+ * loads are issued ahead of the decision. */
+PA_API pa_status pa_block_sparse_attn_skip(const pa_shape *shape,
+                                           const void *q, pa_strides q_strides,
+                                           const void *k, pa_strides k_strides,
+                                           const void *v, pa_strides v_strides,
+                                           const int32_t *rank, const int32_t *cnt,
+                                           float softmax_scale, float skip_threshold,
+                                           void *o, pa_strides o_strides, float *lse,
+                                           uint8_t *skipped, pa_stream_t stream);
+
 /* The whole path: pa_pool_heads -> pa_block_scores -> pa_build_mask ->
  * pa_block_sparse_attn with softmax_scale = 1/sqrt(d) (the strided pooling
- * and scores when budget->score_stride > 1).  The proxies and block
+ * and scores when budget->score_stride > 1; the block skip when
+ * budget->skip_threshold > 0).  The proxies and block
  * scores live in the workspace; the mask is written to *mask_out (all four
  * buffers required in DYNAMIC mode, mass may be NULL otherwise). */
 PA_API pa_status pa_prefill(const pa_shape *shape, const pa_budget *budget,

@@ -129,6 +129,16 @@ def test_budget_and_workspace_errors(L):
                         need, None) == 3
 
 
+@pytest.mark.parametrize("lam", [-0.1, 1.5, float("nan")])
+def test_bad_skip_threshold_rejected(L, lam):
+    s = shape()
+    st = pa.Strides(0, 512, 64)
+    assert L.pa_block_sparse_attn_skip(ctypes.byref(s), 16, st, 16, st, 16, st, 16, 16, ctypes.c_float(0.125),
+                                       ctypes.c_float(lam), 16, st, None, None, None) == 1
+    assert b"skip_threshold" in L.pa_last_error()
+    assert pa.workspace_size(s, pa.make_budget(pa.ALL, 0, 0, 1, lam)) == 0
+
+
 def test_attention_argument_errors(L):
     s = shape()
     st = pa.Strides(0, 512, 64)
