@@ -3,9 +3,9 @@
 // method"; the attention formula of "2. Background").
 //
 // One CTA computes one query block (128 rows) of one or two heads that share
-// a KV head and a proxy group.  The two heads share the group's ranked list;
-// head t visits its first cnt_t entries, so a K/V tile is loaded once for
-// both heads while both still need it.
+// a KV head.  Head t visits the first cnt_t entries of its proxy group's
+// ranked list (two heads of one group share the list); a K/V tile is loaded
+// once for both heads whenever either needs it.
 //
 // Warp roles (384 threads = three warpgroups, one CTA per SM, all 512 TMEM
 // columns).  At the start the third warpgroup hands registers to the two
@@ -180,35 +180,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int unit = p.kv_unit0[kv_of_cta] + j;
     const int h0 = p.unit_h0[unit];
     const int h1 = p.unit_h1[unit];
-    const int g = static_cast<int>(static_cast<long long>(h0) * p.G / p.H);
     const int kvh = static_cast<int>(static_cast<long long>(h0) * p.Hkv / p.H);
     const long long T = static_cast<long long>(p.nb) * (p.nb + 1) / 2;
-    const int32_t *list = p.rank + (static_cast<long long>(b) * p.G + g) * T +
-                          static_cast<long long>(qb) * (qb + 1) / 2;
+    const long long row_off = static_cast<long long>(qb) * (qb + 1) / 2;
+    const int32_t *list0 =
+        p.rank + (static_cast<long long>(b) * p.G + static_cast<long long>(h0) * p.G / p.H) * T + row_off;
+    const int32_t *list1 =
+        p.rank + (static_cast<long long>(b) * p.G + static_cast<long long>(h1 >= 0 ? h1 : h0) * p.G / p.H) * T +
+        row_off;
     int craw[2];
     craw[0] = p.cnt[(static_cast<long long>(b) * p.H + h0) * p.nb + qb];
     craw[1] = (h1 >= 0) ? p.cnt[(static_cast<long long>(b) * p.H + h1) * p.nb + qb] : 0;
     int c[2];
     for (int t = 0; t < 2; ++t) c[t] = min(max(craw[t], 0), qb + 1);
-    const int n = max(c[0], c[1]);
     const int ntiles = (h1 >= 0) ? 2 : 1;
     const int words = (qb + 32) >> 5;  // bitmap words covering blocks 0..qb
 
     // The selected blocks of each head as a bitmap over 0..qb: head t takes the
-    // first c[t] entries of the list.  Every role then visits them in
+    // first c[t] entries of its list.  Every role then visits them in
     // ascending block order (the result does not depend on the order), so the
     // CTAs resident at one time sweep K/V in step.
     for (int w = threadIdx.x; w < 256; w += blockDim.x) bm[w] = 0u;
     __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const int kb = list[i];
+    for (int x = threadIdx.x; x < c[0] + c[1]; x += blockDim.x) {
+        const int t = (x < c[0]) ? 0 : 1;
+        const int kb = t ? list1[x - c[0]] : list0[x];
         if (kb < 0 || kb > qb) {
             flag_status(kStBounds);
             continue;
         }
-        const uint32_t bit = 1u << (kb & 31);
-        if (i < c[0]) atomicOr(&bm[kb >> 5], bit);
-        if (i < c[1]) atomicOr(&bm[128 + (kb >> 5)], bit);
+        atomicOr(&bm[t * 128 + (kb >> 5)], 1u << (kb & 31));
     }
 
     const uint32_t warp = warp_id(), lane = lane_id();

@@ -315,17 +315,15 @@ pa_status launch_budget(const pa_shape *s, const pa_budget *bu, const int32_t *r
 }
 
 // Head units of the attention kernel: pairs of consecutive q heads that share
-// both their KV head and their proxy group (so they share one ranked list and
-// one K/V stream); a head left over forms a unit alone.
+// their KV head (so they share one K/V stream; each follows its own group's
+// ranked list); a head left over forms a unit alone.
 int build_units(const pa_shape *s, int16_t *h0, int16_t *h1) {
-    const int H = s->num_q_heads, Hkv = s->num_kv_heads, G = s->num_groups;
+    const int H = s->num_q_heads, Hkv = s->num_kv_heads;
     int n = 0;
     int h = 0;
     while (h < H) {
         const int kv = static_cast<int>(static_cast<long long>(h) * Hkv / H);
-        const int g = static_cast<int>(static_cast<long long>(h) * G / H);
-        const bool pair = h + 1 < H && static_cast<int>(static_cast<long long>(h + 1) * Hkv / H) == kv &&
-                          static_cast<int>(static_cast<long long>(h + 1) * G / H) == g;
+        const bool pair = h + 1 < H && static_cast<int>(static_cast<long long>(h + 1) * Hkv / H) == kv;
         h0[n] = static_cast<int16_t>(h);
         h1[n] = static_cast<int16_t>(pair ? h + 1 : -1);
         ++n;

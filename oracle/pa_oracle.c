@@ -33,6 +33,8 @@
  *                             the scaled Q.K products (section 2 "Background"),
  *                             restricted to the selected causal keys.
  *   o6 pa_oracle_dense_attn   Plain causal softmax attention, written separately.
+ *   o8 pa_oracle_xattn_mass   XAttention's antidiagonal block estimate (XAttention
+ *      pa_oracle_find_blocks  blog 2.1-2.2) and its threshold selection find_blocks.
  *   o7 pa_oracle_sparse_attn_skip  o5 with BLASST's running-max block skip
  *                             (BLASST introduction, 3.1): a visited block far
  *                             below the running max is left out.
@@ -498,6 +500,94 @@ void pa_oracle_sparse_attn_skip(int N, int H, int Hkv, int d, int G,
         free(use);
         free(row_max);
     }
+}
+
+/* --------------------------------------- o8 XAttention antidiagonal estimate */
+/* XAttention blog, 2.1 "importance prediction" and 2.2 "threshold block
+ * selection" (its block-selection algorithm box).  For head h, query block qb
+ * and stride S (S divides 128): every S x S sub-block of the token-level score
+ * map is scored by the sum along its antidiagonal, i.e. strided row
+ * R = qb*128/S + r (tokens R*S .. R*S+S-1) against strided column c (tokens
+ * c*S .. c*S+S-1) scores
+ *     z[R][c] = sum_{t<S} q[R*S + S-1-t] . k[c*S + t] / (sqrt(d) * S),
+ * the box's reshaped product (query rows taken from S-1 down to 0, key rows
+ * from 0 up).  Readings where the box is silent: the causal mask applies at the
+ * strided level (c <= R: sub-blocks on or below the diagonal); each strided row
+ * is softmax-normalised over its valid columns; the estimate of block kb is the
+ * mean over the query block's 128/S strided rows of the probability falling
+ * in kb's columns, so the estimates of a row sum to one.
+ * mass [B][H][T], entry tri(qb)+kb. */
+void pa_oracle_xattn_mass(int B, int N, int H, int Hkv, int d, int S,
+                          const uint16_t *q, int64_t qsb, int64_t qss, int64_t qsh,
+                          const uint16_t *k, int64_t ksb, int64_t kss, int64_t ksh,
+                          double *mass)
+{
+    int nb = N / BLK, rpb = BLK / S;  /* strided rows (and columns) per block */
+    int64_t T = tri(nb);
+    double scale = 1.0 / (sqrt((double)d) * S);
+    #pragma omp parallel for collapse(3) schedule(dynamic, 1)
+    for (int b = 0; b < B; b++)
+        for (int h = 0; h < H; h++)
+            for (int qb = 0; qb < nb; qb++) {
+                int kvh = kv_of(h, H, Hkv);
+                double *m = mass + ((int64_t)b * H + h) * T + tri(qb);
+                int ncol = (qb + 1) * rpb;
+                double *z = (double *)malloc(sizeof(double) * ncol);
+                for (int kb = 0; kb <= qb; kb++) m[kb] = 0.0;
+                for (int r = 0; r < rpb; r++) {
+                    int R = qb * rpb + r;
+                    double zmax = -INFINITY;
+                    for (int c = 0; c <= R; c++) {
+                        double s = 0.0;
+                        for (int t = 0; t < S; t++)
+                            for (int e = 0; e < d; e++)
+                                s += bf16_to_f64(q[b * qsb + (int64_t)(R * S + S - 1 - t) * qss + h * qsh + e]) *
+                                     bf16_to_f64(k[b * ksb + (int64_t)(c * S + t) * kss + kvh * ksh + e]);
+                        z[c] = s * scale;
+                        if (z[c] > zmax) zmax = z[c];
+                    }
+                    double den = 0.0;
+                    for (int c = 0; c <= R; c++) den += exp(z[c] - zmax);
+                    for (int c = 0; c <= R; c++) m[c / rpb] += exp(z[c] - zmax) / den / rpb;
+                }
+                free(z);
+            }
+}
+
+/* find_blocks (XAttention blog, 2.2 equation): for every (b, h, qb) the
+ * smallest set of blocks whose estimates add up to at least tau, i.e. the
+ * shortest prefix of the blocks ordered by (estimate descending, lower index
+ * first).  Sums run in 2^-40 fixed point as in o4; if no prefix reaches tau
+ * (rounding), every block is kept.  rank [B][H][T] (the ordered blocks),
+ * cnt [B][H][nb] (prefix length). */
+void pa_oracle_find_blocks(int B, int H, int nb, const double *mass, double tau,
+                           int32_t *rank, int32_t *cnt)
+{
+    int64_t T = tri(nb);
+    int64_t tfx = llrint(tau * 1099511627776.0);
+    #pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int b = 0; b < B; b++)
+        for (int h = 0; h < H; h++)
+            for (int qb = 0; qb < nb; qb++) {
+                const double *m = mass + ((int64_t)b * H + h) * T + tri(qb);
+                int32_t *out = rank + ((int64_t)b * H + h) * T + tri(qb);
+                /* insertion sort by (estimate desc, index asc) */
+                for (int t = 0; t <= qb; t++) {
+                    int u = t;
+                    while (u > 0 && (m[out[u - 1]] < m[t] || (m[out[u - 1]] == m[t] && out[u - 1] > t))) {
+                        out[u] = out[u - 1];
+                        u--;
+                    }
+                    out[u] = t;
+                }
+                int64_t cum = 0;
+                int n = qb + 1;
+                for (int t = 0; t <= qb; t++) {
+                    cum += llrint(m[out[t]] * 1099511627776.0);
+                    if (cum >= tfx) { n = t + 1; break; }
+                }
+                cnt[((int64_t)b * H + h) * nb + qb] = n;
+            }
 }
 
 /* ------------------------------------------------------ o6 dense attention */

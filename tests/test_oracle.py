@@ -636,3 +636,86 @@ def test_skip_zero_threshold_and_given_decisions():
     np.testing.assert_allclose(o2, ref, rtol=1e-11, atol=1e-13)
     o3, _, _, _ = oracle.sparse_attn_skip(q, k, v, rank, cnt, 1, items, 0.0, skip_in=s1)
     np.testing.assert_array_equal(o3, o1)
+
+
+# ------------------------------------------- o8 XAttention antidiagonal estimate
+def _antidiag_numpy(q, k, h, S):
+    """numpy: the token-level score map of head h, each S x S sub-block summed
+    along its antidiagonal (row offset S-1-t, column offset t), divided by
+    sqrt(d) * S; strided rows softmax-normalised over sub-blocks on or below
+    the diagonal; block estimates = mean over a block's strided rows."""
+    B, N, H, d = q.shape
+    Hkv = k.shape[2]
+    qf = q[0, :, h].double().numpy()
+    kf = k[0, :, h * Hkv // H].double().numpy()
+    Z = qf @ kf.T
+    n = N // S
+    A = np.zeros((n, n))
+    for t in range(S):
+        A += Z[np.arange(n)[:, None] * S + S - 1 - t, np.arange(n)[None, :] * S + t]
+    A /= math.sqrt(d) * S
+    A[np.triu_indices(n, 1)] = -np.inf
+    P = scipy.special.softmax(A, axis=1)
+    rpb = 128 // S
+    nb = N // 128
+    out = []
+    for qb in range(nb):
+        rows = P[qb * rpb:(qb + 1) * rpb]
+        out.extend(rows[:, kb * rpb:(kb + 1) * rpb].sum() / rpb for kb in range(qb + 1))
+    return np.array(out)
+
+
+@pytest.mark.parametrize("S", [2, 4, 8, 16])
+def test_xattn_mass_is_the_antidiagonal_sum_softmax(S):
+    """o8 against the full score map summed along each sub-block's antidiagonal."""
+    w = synth.small_workload(seqlen=512, heads=4, kv_heads=2, head_dim=32, groups=1)
+    x = synth.make_inputs(w)
+    mass = oracle.xattn_mass(x["q"], x["k"], S)
+    for h in range(4):
+        np.testing.assert_allclose(mass[0, h], _antidiag_numpy(x["q"], x["k"], h, S), rtol=1e-10, atol=1e-13)
+    # every query block's estimates sum to one
+    nb = 4
+    for qb in range(nb):
+        np.testing.assert_allclose(mass[0, :, qb * (qb + 1) // 2: qb * (qb + 1) // 2 + qb + 1].sum(-1), 1.0,
+                                   atol=1e-12)
+
+
+def test_xattn_stride_one_is_the_exact_mass():
+    """S = 1: strided rows are tokens, the antidiagonal is one entry, and the
+    last block's estimates are o3's exact softmax mass."""
+    w = synth.small_workload(seqlen=384, heads=4, kv_heads=2, head_dim=64, groups=1)
+    x = synth.make_inputs(w)
+    mass = oracle.xattn_mass(x["q"], x["k"], 1)
+    exact = oracle.head_mass(x["q"], x["k"])
+    np.testing.assert_allclose(mass[:, :, 3:6], exact, rtol=1e-12, atol=1e-15)
+
+
+def test_find_blocks_brute_force():
+    """The smallest number of blocks whose estimates reach tau (over all
+    subsets) equals the prefix length; the prefix is ordered by (estimate
+    desc, index asc) and reaches tau while one block fewer does not.  A sum
+    that lands exactly on tau counts as reaching it (the equation's >=)."""
+    exact = np.array([[[1.0, 0.25, 0.75, 0.125, 0.5, 0.375]]])  # qb 2: 0.125 + 0.5 + 0.375
+    _, c = oracle.find_blocks(exact, 3, 0.875)
+    assert list(c[0, 0]) == [1, 2, 2]
+    rng = np.random.default_rng(8)
+    nb = 5
+    T = nb * (nb + 1) // 2
+    for trial in range(30):
+        m = np.zeros((1, 2, T))
+        for qb in range(nb):
+            v = rng.dirichlet(np.ones(qb + 1) * 0.5)
+            if trial % 3 == 0 and qb >= 2:
+                v[1] = v[2]  # a tie
+            m[0, :, qb * (qb + 1) // 2: qb * (qb + 1) // 2 + qb + 1] = v
+        tau = float(rng.choice([0.3, 0.5, 0.8, 0.95]))
+        rank, cnt = oracle.find_blocks(m, nb, tau)
+        for h in range(2):
+            for qb in range(nb):
+                v = m[0, h, qb * (qb + 1) // 2: qb * (qb + 1) // 2 + qb + 1]
+                lst = rank[0, h, qb * (qb + 1) // 2: qb * (qb + 1) // 2 + qb + 1]
+                assert sorted(lst) == list(range(qb + 1))
+                assert all((v[a] > v[b_]) or (v[a] == v[b_] and a < b_) for a, b_ in zip(lst, lst[1:]))
+                best = min(len(s) for r in range(1, qb + 2) for s in itertools.combinations(range(qb + 1), r)
+                           if v[list(s)].sum() >= tau - 1e-12) if v.sum() >= tau - 1e-12 else qb + 1
+                assert cnt[0, h, qb] == best

@@ -63,6 +63,17 @@ MUTANTS = [
      "                if (t == 0) row_max[ii] = mt[ii * n + t];"),
     ("skip_block_still_counted", "            use[t] = skip_in ? !skip_in[base + blk[t]] : !own;",
      "            use[t] = skip_in ? !skip_in[base + blk[t]] : 1;"),
+    ("xattn_main_diagonal", "q[b * qsb + (int64_t)(R * S + S - 1 - t) * qss + h * qsh + e]",
+     "q[b * qsb + (int64_t)(R * S + t) * qss + h * qsh + e]"),
+    ("xattn_no_causal", [("for (int c = 0; c <= R; c++) {\n                        double s = 0.0;",
+                          "for (int c = 0; c < ncol; c++) {\n                        double s = 0.0;"),
+                         ("for (int c = 0; c <= R; c++) den += exp(z[c] - zmax);",
+                          "for (int c = 0; c < ncol; c++) den += exp(z[c] - zmax);"),
+                         ("for (int c = 0; c <= R; c++) m[c / rpb] +=", "for (int c = 0; c < ncol; c++) m[c / rpb] +=")],
+     None),
+    ("xattn_scale_without_stride", "double scale = 1.0 / (sqrt((double)d) * S);", "double scale = 1.0 / sqrt((double)d);"),
+    ("find_blocks_strict", "if (cum >= tfx) { n = t + 1; break; }", "if (cum > tfx) { n = t + 1; break; }"),
+    ("find_blocks_ascending", "while (u > 0 && (m[out[u - 1]] < m[t] ||", "while (u > 0 && (m[out[u - 1]] > m[t] ||"),
     ("skip_threshold_log2", "double lnl = (lambda > 0.0) ? log(lambda) : -INFINITY;",
      "double lnl = (lambda > 0.0) ? log2(lambda) : -INFINITY;"),
 ]
@@ -87,6 +98,9 @@ PINS = [
     lambda: T.test_skip_brute_force(0.2),
     T.test_skip_planted_running_max,
     T.test_skip_sweep_skips_some_and_nests,
+    lambda: T.test_xattn_mass_is_the_antidiagonal_sum_softmax(8),
+    T.test_xattn_stride_one_is_the_exact_mass,
+    T.test_find_blocks_brute_force,
     G.test_golden_rank,
     G.test_golden_budget,
 ]

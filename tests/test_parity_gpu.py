@@ -73,6 +73,9 @@ CASES = [
     ("odd_heads_per_grp", 768, 14, 2, 128, 2, pa.DYNAMIC,   0.8,  0,   1),
     ("batch2",            512,  4, 2,  64, 2, pa.DYNAMIC,   0.95, 0,   2),
     ("gamma_one",         512,  4, 2, 128, 1, pa.DYNAMIC,   1.0,  0,   1),
+    # paired heads (one KV head) that follow different lists: G = H under GQA
+    ("gqa_g_eq_h_pairs",  768,  8, 2,  64, 8, pa.DYNAMIC,   0.9,  0,   1),
+    ("gqa_g4_pairs_d128", 640,  8, 2, 128, 4, pa.FIXED_FRACTION, 0, 400, 1),
 ]
 
 
