@@ -62,6 +62,11 @@ def parse_args():
     ap.add_argument("--frac", type=int, default=100, help="fixed budget in per mille of causal blocks")
     ap.add_argument("--score-stride", type=int, default=1, choices=[1, 2, 4, 8],
                     help="query-row stride of the proxy block scores (1: every row)")
+    ap.add_argument("--estimator", choices=["proxy", "xattn"], default="proxy",
+                    help="mask estimator: ProxyAttn (pooled proxy scores + per-head budget) or XAttention "
+                         "(antidiagonal strided scores + find_blocks, one list per head)")
+    ap.add_argument("--xattn-stride", type=int, default=8, choices=[4, 8, 16])
+    ap.add_argument("--tau", type=float, default=0.9, help="XAttention find_blocks threshold")
     ap.add_argument("--skip-threshold", type=float, default=0.0,
                     help="running-max block skip in the attention: lambda in [0, 1] (0: off)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -146,7 +151,7 @@ class Pipeline:
     """Pre-allocated buffers and ctypes arguments for one layer, so that a step is
     four C-ABI calls with CUDA events between them."""
 
-    def __init__(self, q, k, v, G, mode, gamma, frac, stride=1, skip=0.0):
+    def __init__(self, q, k, v, G, mode, gamma, frac, stride=1, skip=0.0, proxies=True):
         import block_sparse_attention_pa_b200 as pa
         self.pa = pa
         self.L = pa.lib()
@@ -161,14 +166,16 @@ class Pipeline:
         self.skip = skip
         self.skipped = None  # uint8 [B, H, T] when counting skipped blocks
         dev = q.device
-        self.qp = torch.empty(B, G, N // stride, d, device=dev, dtype=torch.bfloat16)
-        self.kp = torch.empty(B, G, N, d, device=dev, dtype=torch.bfloat16)
+        pn = N if proxies else 128  # the XAttention pipeline needs no proxies
+        self.qp = torch.empty(B, G, pn // stride, d, device=dev, dtype=torch.bfloat16)
+        self.kp = torch.empty(B, G, pn, d, device=dev, dtype=torch.bfloat16)
         T = self.nb * (self.nb + 1) // 2
         self.T = T
         self.scores = torch.empty(B, G, T, device=dev, dtype=torch.float32)
         self.mask = pa.Mask.empty(self.shape, dev, mode == 0)
         self.bufs = self.mask.bufs()
-        self.ws = torch.empty(max(pa.workspace_size(self.shape, self.budget), 256), device=dev, dtype=torch.uint8)
+        self.ws = torch.empty(max(pa.workspace_size(self.shape, self.budget), 256) if proxies else 256, device=dev,
+                              dtype=torch.uint8)
         self.o = torch.empty_like(q)
         self.qs, self.ks, self.vs, self.os_ = (pa._strides(t) for t in (q, k, v, self.o))
         self.scale = 1.0 / math.sqrt(d)
@@ -187,6 +194,12 @@ class Pipeline:
         pa._check(L.pa_build_mask(sh, bu, self.scores.data_ptr(), self.q.data_ptr(), self.qs, self.k.data_ptr(),
                                   self.ks, ctypes.byref(self.bufs), self.ws.data_ptr(), self.ws.numel(), st))
         if ev: ev[3].record()
+        self.attend(st)
+        if ev: ev[4].record()
+
+    def attend(self, st):
+        pa, L = self.pa, self.L
+        sh = ctypes.byref(self.shape)
         if self.skip > 0.0:
             pa._check(L.pa_block_sparse_attn_skip(sh, self.q.data_ptr(), self.qs, self.k.data_ptr(), self.ks,
                                                   self.v.data_ptr(), self.vs, self.mask.rank.data_ptr(),
@@ -199,7 +212,6 @@ class Pipeline:
                                              self.v.data_ptr(), self.vs, self.mask.rank.data_ptr(),
                                              self.mask.cnt.data_ptr(), self.scale, self.o.data_ptr(), self.os_, None,
                                              st))
-        if ev: ev[4].record()
 
     def visited(self):
         """(visited blocks, algorithmic attention FLOPs with the diagonal tile
@@ -220,6 +232,34 @@ class Pipeline:
         n = int(self.skipped.sum().item())
         self.skipped = None
         return n
+
+
+class XPipeline(Pipeline):
+    """The XAttention estimator in place of the ProxyAttn one: a step is
+    pa_xattn_mask (strided antidiagonal GEMM + selection) then the same
+    attention call with one list per head."""
+
+    def __init__(self, q, k, v, S, tau, skip=0.0):
+        import block_sparse_attention_pa_b200 as pa
+        B, N, H, d = q.shape
+        super().__init__(q, k, v, H, 1, 0.0, 1000, 1, skip, proxies=False)
+        self.S, self.tau = S, tau
+        self.xws = torch.empty(max(int(self.L.pa_xattn_workspace_size(ctypes.byref(self.shape), S)), 256),
+                               device=q.device, dtype=torch.uint8)
+        self.launches_per_step = 3  # xattn gemm, select, attn
+
+    def step(self, ev=None):
+        pa, L, st = self.pa, self.L, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        sh = ctypes.byref(self.shape)
+        if ev: ev[0].record()
+        if ev: ev[1].record()
+        pa._check(L.pa_xattn_mask(sh, self.S, self.tau, self.q.data_ptr(), self.qs, self.k.data_ptr(), self.ks,
+                                  self.mask.rank.data_ptr(), self.mask.cnt.data_ptr(), None, self.xws.data_ptr(),
+                                  self.xws.numel(), st))
+        if ev: ev[2].record()
+        if ev: ev[3].record()
+        self.attend(st)
+        if ev: ev[4].record()
 
 
 def selected_blocks(pipe) -> torch.Tensor:
@@ -431,7 +471,11 @@ def main():
     q, k, v = x["q"], x["k"], x["v"]
     stride = args.score_stride
     skip = args.skip_threshold
-    pipe = Pipeline(q, k, v, G, mode, gamma, frac, stride, skip)
+    xattn = args.estimator == "xattn"
+    if xattn:
+        pipe = XPipeline(q, k, v, args.xattn_stride, args.tau, skip)
+    else:
+        pipe = Pipeline(q, k, v, G, mode, gamma, frac, stride, skip)
     sampler = None if args.no_clocks else ClockSampler(local)
     total_ms, stages, clocks = time_pipeline(pipe, args.steps, args.warmup, dist_on, sampler)
     status = pa.device_status()
@@ -475,12 +519,29 @@ def main():
         "mask": {"ms": float(stages[2])},
         "attn": {"ms": attn_ms, "TFLOP/s": achieved, "frac_tensor": achieved / peak},
     }
+    if xattn:
+        # strided antidiagonal GEMM: executed 128 x 256 tiles; exact causal work beside it
+        S = args.xattn_stride
+        rows = w.seqlen // S
+        tiles = sum(mt // 2 + 1 for mt in range((rows + 127) // 128))
+        x_exec = B * H * tiles * 2 * 128 * 256 * S * d
+        x_exact = B * H * (rows * (rows + 1) // 2) * 2 * S * d
+        stage_roofline = {
+            "xattn_estimate": {"ms": float(stages[1]), "TFLOP/s": x_exec / (stages[1] * 1e-3) / 1e12,
+                               "frac_tensor": x_exec / (stages[1] * 1e-3) / 1e12 / peak,
+                               "flops_executed": x_exec, "flops_exact_causal": x_exact},
+            "attn": {"ms": attn_ms, "TFLOP/s": achieved, "frac_tensor": achieved / peak},
+        }
 
     line = {"metric": METRIC, "value": per_layer(ms_step, world), "unit": "ms/layer", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded needle/sink generator; random inputs, no weights)",
-            "config": config_of(w, G, mode, gamma, frac, stride, skip) | {"parallelism": f"replicas x{world}"},
+            "config": (config_of(w, G, mode, gamma, frac, stride, skip) if not xattn else
+                       config_of(w, H, 1, 0.0, 1000, 1, skip) | {
+                           "groups": H, "budget": f"XAttention find_blocks tau={args.tau}",
+                           "estimator": f"xattn antidiagonal stride {args.xattn_stride}"})
+                      | {"parallelism": f"replicas x{world}"},
             "est_ms": est_ms, "sparse_ms": attn_ms,
             "tflops_effective": flops / (attn_ms * 1e-3) / 1e12, "tflops_exact_causal": flops_exact / (attn_ms * 1e-3) / 1e12,
             "visited_blocks": visited, "density": density, "sparsity": 1.0 - density,
@@ -494,7 +555,7 @@ def main():
 
     # dense baseline: the same kernel with every causal block selected
     if not args.no_dense:
-        dense = Pipeline(q, k, v, G, 2, gamma, frac, stride)
+        dense = Pipeline(q, k, v, w.num_groups, 2, gamma, frac, 1)
         dsteps = max(2, min(5, args.steps))
         _, dstages, _ = time_pipeline(dense, dsteps, 1, dist_on)
         dense_attn = float(dstages[3])
@@ -530,12 +591,12 @@ def main():
         del every, a, b
 
     # end to end through the public API with pinned host buffers
-    if not args.no_e2e:
+    if not args.no_e2e and not xattn:
         e2e = run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world, stride, skip)
         line["e2e"] = e2e
 
     # the CPU oracle on a bounded sample (rank 0, one GPU only)
-    if not args.no_cpu_baseline and world == 1 and rank == 0:
+    if not args.no_cpu_baseline and world == 1 and rank == 0 and not xattn:
         import oracle
         xc = {n: x[n].cpu() for n in ("q", "k", "v")}
         ms, det, sample = oracle_estimate(xc, w, G, mode, gamma, frac, size="baseline", stride=stride, skip=skip)

@@ -32,8 +32,9 @@ STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_E
 ENTRY_POINTS = ("pa_workspace_size", "pa_pool_heads", "pa_block_scores", "pa_build_mask",
                 "pa_block_sparse_attn", "pa_prefill", "pa_get_device_status", "pa_status_string",
                 "pa_last_error", "pa_abi_version", "pa_build_mask_noalloc", "pa_selftest_wait_timeout",
-                "pa_pool_heads_strided", "pa_block_scores_strided", "pa_block_sparse_attn_skip")
+                "pa_pool_heads_strided", "pa_block_scores_strided", "pa_block_sparse_attn_skip", "pa_xattn_workspace_size", "pa_xattn_mask")
 
+XATTN_STRIDES = (4, 8, 16)
 SCORE_STRIDES = (1, 2, 4, 8)
 
 
@@ -89,6 +90,10 @@ def lib() -> ctypes.CDLL:
         L.pa_prefill.argtypes = [P(Shape), P(Budget), vp, st, vp, st, vp, st, vp, st, P(MaskBufs), vp,
                                  ctypes.c_size_t, vp]
         L.pa_get_device_status.argtypes = [vp, ctypes.c_int]
+        L.pa_xattn_workspace_size.restype = ctypes.c_size_t
+        L.pa_xattn_workspace_size.argtypes = [P(Shape), ctypes.c_int32]
+        L.pa_xattn_mask.argtypes = [P(Shape), ctypes.c_int32, ctypes.c_float, vp, st, vp, st, vp, vp, vp, vp,
+                                    ctypes.c_size_t, vp]
         L.pa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp]
         L.pa_status_string.restype = ctypes.c_char_p
         L.pa_status_string.argtypes = [ctypes.c_int]
@@ -96,7 +101,7 @@ def lib() -> ctypes.CDLL:
         L.pa_abi_version.restype = ctypes.c_int32
         for name in ("pa_pool_heads", "pa_block_scores", "pa_build_mask", "pa_block_sparse_attn", "pa_prefill",
                      "pa_get_device_status", "pa_selftest_wait_timeout", "pa_pool_heads_strided",
-                     "pa_block_scores_strided", "pa_block_sparse_attn_skip"):
+                     "pa_block_scores_strided", "pa_block_sparse_attn_skip", "pa_xattn_mask"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -219,6 +224,29 @@ def build_mask(scores: torch.Tensor, q: torch.Tensor, k: torch.Tensor, num_group
                                _strides(q), k.data_ptr(), _strides(k), ctypes.byref(bufs), workspace.data_ptr(),
                                workspace.numel(), _stream(q.device)))
     return mask
+
+
+def xattn_mask(q: torch.Tensor, k: torch.Tensor, stride: int = 8, tau: float = 0.9,
+               workspace: torch.Tensor | None = None):
+    """pa_xattn_mask -> (rank int32 [B, H, T], cnt int32 [B, H, nb], mass fp32
+    [B, H, T]); feed rank/cnt to block_sparse_attn with num_groups = H."""
+    _cuda_bf16(q, "q")
+    _cuda_bf16(k, "k")
+    B, N, H, d = q.shape
+    shape = make_shape(q, k, H)
+    nb = N // 128
+    T = nb * (nb + 1) // 2
+    i32 = dict(device=q.device, dtype=torch.int32)
+    rank = torch.empty(B, H, T, **i32)
+    cnt = torch.empty(B, H, nb, **i32)
+    mass = torch.empty(B, H, T, device=q.device, dtype=torch.float32)
+    if workspace is None:
+        need = int(lib().pa_xattn_workspace_size(ctypes.byref(shape), int(stride)))
+        workspace = torch.empty(max(need, 256), device=q.device, dtype=torch.uint8)
+    _check(lib().pa_xattn_mask(ctypes.byref(shape), int(stride), float(tau), q.data_ptr(), _strides(q), k.data_ptr(),
+                               _strides(k), rank.data_ptr(), cnt.data_ptr(), mass.data_ptr(), workspace.data_ptr(),
+                               workspace.numel(), _stream(q.device)))
+    return rank, cnt, mass
 
 
 def block_sparse_attn(q, k, v, rank, cnt, num_groups: int, softmax_scale: float | None = None,

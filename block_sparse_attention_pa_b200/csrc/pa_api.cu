@@ -19,6 +19,7 @@
 #include "mask.cuh"
 #include "pool.cuh"
 #include "tile_gemm.cuh"
+#include "xattn.cuh"
 
 namespace {
 
@@ -176,6 +177,27 @@ pa_status map_proxy(CUtensorMap *m, const void *base, int B, int G, int N, int d
     return make_map(m, base, dims, strides, 128, 1, name);
 }
 
+// [B][N][heads][d] with element strides, the token axis split as (token mod S,
+// token / S) -> dims (d, heads, S, N/S, B), box 64 x 1 x 1 x rows x 1.
+pa_status map_bnhd_split(CUtensorMap *m, const void *base, int B, int N, int heads, int d, int S, pa_strides st,
+                         cuuint32_t rows, const char *name) {
+    auto fn = encode_fn();
+    if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    const int64_t sb = (B == 1) ? st.s * N : st.b;
+    const cuuint64_t dims[5] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(heads),
+                                static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(N / S),
+                                static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[4] = {static_cast<cuuint64_t>(st.h) * 2, static_cast<cuuint64_t>(st.s) * 2,
+                                   static_cast<cuuint64_t>(st.s) * S * 2, static_cast<cuuint64_t>(sb) * 2};
+    const cuuint32_t box[5] = {64, 1, 1, rows, 1};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed: %d", name, static_cast<int>(r));
+    return PA_OK;
+}
+
 int num_sms() {
     int dev = 0, n = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -204,6 +226,26 @@ WsLayout ws_layout(const pa_shape *s, const pa_budget *bu) {
 
 size_t mask_ws_bytes(const pa_shape *s, const pa_budget *bu) {
     return ws_layout(s, bu).qp;  // the partial-softmax statistics come first
+}
+
+// XAttention partials: part_s [B][H][nb][N/S] then part_m [B][H][nchunk][N/S].
+struct XWsLayout {
+    size_t part_s, part_m, total;
+};
+
+XWsLayout xattn_ws_layout(const pa_shape *s, int S) {
+    const size_t B = s->batch, H = s->num_q_heads, N = s->seqlen, nb = N / kBlk;
+    const size_t rows = N / S, nchunk = (rows + 127) / 128;
+    XWsLayout w;
+    w.part_s = 0;
+    w.part_m = align256(B * H * nb * rows * sizeof(float));
+    w.total = w.part_m + align256(B * H * nchunk * rows * sizeof(float));
+    return w;
+}
+
+pa_status check_xstride(int S) {
+    if (S != 4 && S != 8 && S != 16) return fail(PA_ERR_INVALID_ARG, "stride must be 4, 8 or 16 (got %d)", S);
+    return PA_OK;
 }
 
 // ------------------------------------------------------------- launches
@@ -310,6 +352,68 @@ pa_status launch_budget(const pa_shape *s, const pa_budget *bu, const int32_t *r
     p.mode = bu->mode; p.gamma = bu->gamma; p.frac_permille = bu->frac_permille;
     p.rank = rank; p.mass = mass; p.cnt = cnt; p.budget = budget;
     pa::budget_kernel<<<s->batch * s->num_q_heads, 1024, 0, st>>>(p);
+    PA_CUDA(cudaGetLastError());
+    return PA_OK;
+}
+
+template <int D, int S>
+pa_status launch_xattn_gemm_t(const CUtensorMap &mq, const CUtensorMap &mk, const pa::XattnParams &p,
+                              cudaStream_t st) {
+    auto kern = pa::xattn_gemm_kernel<D, S>;
+    const int smem = pa::XattnSmem<D, S>::BYTES;
+    PA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    const long long grid = std::min<long long>(p.num_units, num_sms());
+    if (grid <= 0) return PA_OK;
+    kern<<<static_cast<unsigned>(grid), 192, smem, st>>>(mq, mk, p);
+    PA_CUDA(cudaGetLastError());
+    return PA_OK;
+}
+
+template <int D>
+pa_status launch_xattn_gemm_d(int S, const CUtensorMap &mq, const CUtensorMap &mk, const pa::XattnParams &p,
+                              cudaStream_t st) {
+    if (S == 4) return launch_xattn_gemm_t<D, 4>(mq, mk, p, st);
+    if (S == 8) return launch_xattn_gemm_t<D, 8>(mq, mk, p, st);
+    return launch_xattn_gemm_t<D, 16>(mq, mk, p, st);
+}
+
+pa_status launch_xattn(const pa_shape *s, int S, float tau, const void *q, pa_strides qs, const void *k,
+                       pa_strides ks, int32_t *rank, int32_t *cnt, float *mass, void *ws, cudaStream_t st) {
+    const int B = s->batch, H = s->num_q_heads, Hkv = s->num_kv_heads, N = s->seqlen, d = s->head_dim;
+    const int nb = N / kBlk, rows = N / S;
+    CUtensorMap mq, mk;
+    pa_status r = map_bnhd_split(&mq, q, B, N, H, d, S, qs, 128, "q");
+    if (r) return r;
+    if ((r = map_bnhd_split(&mk, k, B, N, Hkv, d, S, ks, 256, "k"))) return r;
+    const XWsLayout w = xattn_ws_layout(s, S);
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    pa::XattnParams p{};
+    p.B = B; p.H = H; p.Hkv = Hkv; p.nb = nb;
+    p.rows = rows;
+    p.nchunk = (rows + 127) / 128;
+    const int mtiles = (rows + 127) / 128;
+    long long per = 0;
+    for (int mt = 0; mt < mtiles; ++mt) per += mt / 2 + 1;
+    p.units_per_bh = per;
+    p.num_units = per * B * H;
+    p.c2 = static_cast<float>(1.4426950408889634 / (std::sqrt(static_cast<double>(d)) * S));
+    p.part_s = reinterpret_cast<float *>(base + w.part_s);
+    p.part_m = reinterpret_cast<float *>(base + w.part_m);
+    p.timeout_ns = wait_timeout_ns();
+    r = d == 128 ? launch_xattn_gemm_d<128>(S, mq, mk, p, st) : launch_xattn_gemm_d<64>(S, mq, mk, p, st);
+    if (r) return r;
+    pa::XselParams sp{};
+    sp.B = B; sp.H = H; sp.nb = nb; sp.rows = rows; sp.nchunk = p.nchunk; sp.S = S;
+    sp.tau = tau;
+    sp.part_s = p.part_s;
+    sp.part_m = p.part_m;
+    sp.mass = mass;
+    sp.rank = rank;
+    sp.cnt = cnt;
+    int P = 1;
+    while (P < nb) P <<= 1;
+    const long long grid = static_cast<long long>(B) * H * nb;
+    pa::xattn_select_kernel<<<static_cast<unsigned>(grid), 256, P * 8, st>>>(sp);
     PA_CUDA(cudaGetLastError());
     return PA_OK;
 }
@@ -561,6 +665,36 @@ pa_status pa_get_device_status(pa_stream_t stream, int clear) {
     }
     g_last_error.clear();
     return static_cast<pa_status>(v);
+}
+
+}  // extern "C"
+
+// ================================================================ XAttention
+extern "C" {
+
+size_t pa_xattn_workspace_size(const pa_shape *shape, int32_t stride) {
+    if (check_shape(shape) || check_xstride(stride)) return 0;
+    return xattn_ws_layout(shape, stride).total;
+}
+
+pa_status pa_xattn_mask(const pa_shape *shape, int32_t stride, float tau, const void *q, pa_strides qs,
+                        const void *k, pa_strides ks, int32_t *rank, int32_t *cnt, float *mass, void *ws,
+                        size_t ws_bytes, pa_stream_t stream) {
+    pa_status r;
+    if ((r = check_shape(shape)) || (r = check_xstride(stride))) return r;
+    if (!(tau > 0.0f && tau <= 1.0f))
+        return fail(PA_ERR_INVALID_ARG, "tau must be in (0, 1] (got %g)", static_cast<double>(tau));
+    if ((r = check_tensor(q, qs, "q")) || (r = check_tensor(k, ks, "k"))) return r;
+    if ((r = check_ptr(rank, "rank", 4)) || (r = check_ptr(cnt, "cnt", 4))) return r;
+    if (mass && (r = check_ptr(mass, "mass", 4))) return r;
+    const size_t need = xattn_ws_layout(shape, stride).total;
+    if (!ws || ws_bytes < need)
+        return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, need);
+    if ((r = check_ptr(ws, "workspace", 256))) return r;
+    if ((r = launch_xattn(shape, stride, tau, q, qs, k, ks, rank, cnt, mass, ws,
+                          reinterpret_cast<cudaStream_t>(stream))))
+        return r;
+    return ok();
 }
 
 }  // extern "C"

@@ -256,6 +256,33 @@ PA_API pa_status pa_block_sparse_attn_skip(const pa_shape *shape,
                                            void *o, pa_strides o_strides, float *lse,
                                            uint8_t *skipped, pa_stream_t stream);
 
+/* XAttention's estimator (XAttention blog, 2.1 "importance prediction",
+ * 2.2 "threshold block selection" and its block-selection algorithm), a second
+ * way to build the mask that pa_block_sparse_attn consumes.  Per head h (one
+ * list per head: pass the result to pa_block_sparse_attn with a shape whose
+ * num_groups = num_q_heads), stride S in {4, 8, 16}:
+ *   z[R][c] = sum_{t<S} q[R*S + S-1-t] . k[c*S + t] / (sqrt(d) * S)
+ * for strided rows R and columns c (the antidiagonal sum of each S x S
+ * sub-block of the score map); each row R is softmax-normalised over c <= R
+ * (the causal mask at the sub-block level, a reading: the box shows none);
+ *   mass[b][h][tri(qb)+kb] = (S/128) * sum over the 128/S rows R of block qb
+ *                            of the probability in block kb's 128/S columns;
+ *   rank[b][h][tri(qb) ..]  = blocks 0..qb by (mass desc, lower index first);
+ *   cnt[b][h][qb]           = find_blocks: the shortest prefix of that list
+ *                            whose masses sum to >= tau (sums in 2^-40 fixed
+ *                            point, tau taken as the fp32 value), else qb+1.
+ * No block is forced into the set.  bf16 tensor-core products with fp32
+ * accumulation; mass (nullable) fp32.  ws: device workspace of
+ * ws_bytes >= pa_xattn_workspace_size(shape, S); tau in (0, 1].  The shape's
+ * num_groups is not used. */
+PA_API size_t pa_xattn_workspace_size(const pa_shape *shape, int32_t stride);
+
+PA_API pa_status pa_xattn_mask(const pa_shape *shape, int32_t stride, float tau,
+                               const void *q, pa_strides q_strides,
+                               const void *k, pa_strides k_strides,
+                               int32_t *rank, int32_t *cnt, float *mass,
+                               void *ws, size_t ws_bytes, pa_stream_t stream);
+
 /* The whole path: pa_pool_heads -> pa_block_scores -> pa_build_mask ->
  * pa_block_sparse_attn with softmax_scale = 1/sqrt(d) (the strided pooling
  * and scores when budget->score_stride > 1; the block skip when

@@ -139,6 +139,21 @@ def test_bad_skip_threshold_rejected(L, lam):
     assert pa.workspace_size(s, pa.make_budget(pa.ALL, 0, 0, 1, lam)) == 0
 
 
+def test_xattn_workspace_and_argument_errors(L):
+    s = shape(N=1024, H=8)
+    for S in (4, 8, 16):
+        rows = 1024 // S
+        a256 = lambda x: (x + 255) // 256 * 256
+        assert L.pa_xattn_workspace_size(ctypes.byref(s), S) == a256(8 * 8 * rows * 4) + a256(8 * ((rows + 127) // 128) * rows * 4)
+    assert L.pa_xattn_workspace_size(ctypes.byref(s), 2) == 0
+    st = pa.Strides(0, 512, 64)
+    for S, tau in ((3, 0.9), (32, 0.9), (8, 0.0), (8, 1.5)):
+        assert L.pa_xattn_mask(ctypes.byref(s), S, ctypes.c_float(tau), 16, st, 16, st, 16, 16, None, 256, 1 << 30,
+                               None) == 1
+    assert L.pa_xattn_mask(ctypes.byref(s), 8, ctypes.c_float(0.9), 16, st, 16, st, 16, 16, None, 256, 16,
+                           None) == 3
+
+
 def test_attention_argument_errors(L):
     s = shape()
     st = pa.Strides(0, 512, 64)

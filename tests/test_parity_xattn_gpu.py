@@ -1,0 +1,111 @@
+"""GPU parity of the XAttention estimator (pa_xattn_mask: antidiagonal
+strided scores, softmax block estimates, find_blocks) against the oracle's
+o8 on the same seeded inputs, and of the block-sparse attention it drives.
+
+Acceptance:
+  block estimates  |gpu - ref| <= 2e-5 + 2e-3 * ref (fp32 logits of bf16
+                   products over S*d terms, exp2 on the MUFU; as for the head
+                   mass of the ProxyAttn budget); every query block's
+                   estimates sum to one within 1e-4
+  rank, cnt        bit-exact with the oracle's find_blocks fed the GPU's fp32
+                   estimates (ties to the lower index)
+  O                max-abs <= 2e-2, mean-abs <= 2e-3 against o5 with the
+                   GPU's lists (one list per head: num_groups = num_q_heads)
+Cases span several 128-row x 256-column output tiles, ragged last tiles
+(N/S not a multiple of 128), S = 4, 8, 16, d = 64 and 128, GQA, batch 2.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import block_sparse_attention_pa_b200 as pa
+from block_sparse_attention_pa_b200 import build, synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    pa.lib()
+    assert pa.device_status() == 0
+
+
+CASES = [
+    # name,              N,    H, Hkv, d,   S,  tau,  B
+    ("s8_d64",           1024, 4, 2,  64,  8,  0.9,  1),
+    ("s4_d128_tiles",    4096, 2, 1,  128, 4,  0.95, 1),
+    ("s16_ragged_d128",  1152, 4, 2,  128, 16, 0.8,  1),
+    ("s8_ragged_gqa",    2944, 6, 2,  64,  8,  0.9,  1),
+    ("s4_batch2",        640,  4, 4,  64,  4,  0.7,  2),
+    ("s8_single_block",  128,  2, 1,  128, 8,  0.9,  1),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_xattn_parity(case):
+    name, N, H, Hkv, d, S, tau, B = case
+    w = synth.small_workload(seqlen=N, heads=H, kv_heads=Hkv, head_dim=d, groups=H, batch=B, needles=8,
+                             seed=700 + CASES.index(case))
+    x = synth.make_inputs(w)
+    qc, kc, vc = x["q"], x["k"], x["v"]
+    q, k, v = qc.cuda(), kc.cuda(), vc.cuda()
+    nb = N // 128
+    rank, cnt, mass = pa.xattn_mask(q, k, S, tau)
+    o = pa.block_sparse_attn(q, k, v, rank, cnt, H)
+    torch.cuda.synchronize()
+    assert pa.device_status() == 0
+
+    mg = mass.double().cpu().numpy()
+    ref = oracle.xattn_mass(qc, kc, S)
+    err = np.abs(mg - ref)
+    assert np.all(err <= 2e-5 + 2e-3 * ref), err.max()
+    for qb in range(nb):
+        sl = slice(qb * (qb + 1) // 2, qb * (qb + 1) // 2 + qb + 1)
+        np.testing.assert_allclose(mg[:, :, sl].sum(-1), 1.0, atol=1e-4)
+
+    rank_ref, cnt_ref = oracle.find_blocks(mass.cpu().numpy(), nb, float(np.float32(tau)))
+    assert np.array_equal(rank.cpu().numpy(), rank_ref)
+    assert np.array_equal(cnt.cpu().numpy(), cnt_ref)
+    if nb > 2:
+        assert cnt_ref.min() < cnt_ref.max()  # the threshold selects, not everything
+
+    items = [(b, h, qb) for b in range(B) for h in range(H) for qb in range(nb)]
+    if len(items) > 48:
+        rng = np.random.default_rng(1)
+        items = [items[i] for i in sorted(rng.choice(len(items), 48, replace=False))] + [(0, H - 1, nb - 1)]
+    oref, _ = oracle.sparse_attn(qc, kc, vc, rank.cpu().numpy(), cnt.cpu().numpy(), H, items)
+    og = o.float().cpu().numpy()
+    ogi = np.stack([og[b, qb * 128:(qb + 1) * 128, h] for (b, h, qb) in items])
+    diff = np.abs(ogi - oref)
+    assert diff.max() <= 2e-2 and diff.mean() <= 2e-3, (diff.max(), diff.mean())
+
+
+def test_xattn_full_size_sampled():
+    """The 32K Llama shape at S = 8: estimates of sampled (head, query block)
+    rows against the oracle on the matching token range, lists complete and
+    bit-exact given the GPU's estimates."""
+    w = synth.WORKLOADS["llama8b_n32k"]
+    x = synth.make_inputs(w, device="cuda")
+    q, k = x["q"], x["k"]
+    B, N, H, d = q.shape
+    nb = N // 128
+    rank, cnt, mass = pa.xattn_mask(q, k, 8, 0.9)
+    torch.cuda.synchronize()
+    assert pa.device_status() == 0
+    mg = mass.cpu().numpy()
+    rank_ref, cnt_ref = oracle.find_blocks(mg, nb, float(np.float32(0.9)))
+    assert np.array_equal(rank.cpu().numpy(), rank_ref)
+    assert np.array_equal(cnt.cpu().numpy(), cnt_ref)
+    # the estimates of query blocks qb depend only on tokens < (qb+1)*128:
+    # run the oracle on the prefix and compare its rows
+    qc, kc = q.cpu(), k.cpu()
+    for qb in (0, 5, 40):
+        n_tok = (qb + 1) * 128
+        heads = [0, H - 1]
+        kvs = [h * w.num_kv_heads // H for h in heads]
+        ref = oracle.xattn_mass(qc[:, :n_tok, heads].contiguous(), kc[:, :n_tok, kvs].contiguous(), 8)
+        sl = slice(qb * (qb + 1) // 2, qb * (qb + 1) // 2 + qb + 1)
+        got = mg[:, heads, sl].astype(np.float64)
+        assert np.all(np.abs(got - ref[:, :, sl]) <= 2e-5 + 2e-3 * ref[:, :, sl])
