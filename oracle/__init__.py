@@ -100,22 +100,32 @@ def _proxy_bits(t: torch.Tensor) -> np.ndarray:
     return t.view(torch.int16).numpy().view(np.uint16)
 
 
+def rows_total(nb: int, causal: bool = True) -> int:
+    """Entries of one (b, g) row set of scores or lists: T = nb(nb+1)/2
+    causal (row qb at qb(qb+1)/2), nb*nb non-causal (row qb at qb*nb)."""
+    return nb * (nb + 1) // 2 if causal else nb * nb
+
+
+def row_at(nb: int, qb: int, causal: bool = True) -> int:
+    return qb * (qb + 1) // 2 if causal else qb * nb
+
+
 def block_scores(qp_bf16: torch.Tensor, kp_bf16: torch.Tensor, scale: float | None = None,
-                 stride: int = 1) -> np.ndarray:
+                 stride: int = 1, causal: bool = True) -> np.ndarray:
     """o2: scores [B, G, T] fp64 from the bf16 proxies [B, G, N, d]; with
     stride r only the query rows i = r-1 (mod r) are scored."""
     B, G, N, d = qp_bf16.shape
     nb = N // BLK
     scale = 1.0 / np.sqrt(d) if scale is None else scale
     assert stride >= 1 and BLK % stride == 0
-    out = np.empty((B, G, nb * (nb + 1) // 2), np.float64)
+    out = np.empty((B, G, rows_total(nb, causal)), np.float64)
     lib().pa_oracle_block_scores(_i(B), _i(N), _i(G), _i(d), _p(_proxy_bits(qp_bf16)),
-                                 _p(_proxy_bits(kp_bf16)), _d(scale), _i(stride), _p(out))
+                                 _p(_proxy_bits(kp_bf16)), _d(scale), _i(stride), _i(int(causal)), _p(out))
     return out
 
 
 def block_score_tiles(qp_bf16: torch.Tensor, kp_bf16: torch.Tensor, tiles, scale: float | None = None,
-                      stride: int = 1) -> np.ndarray:
+                      stride: int = 1, causal: bool = True) -> np.ndarray:
     """o2 on a sample: tiles is an int array [n, 4] of (b, g, qb, kb)."""
     B, G, N, d = qp_bf16.shape
     scale = 1.0 / np.sqrt(d) if scale is None else scale
@@ -123,12 +133,14 @@ def block_score_tiles(qp_bf16: torch.Tensor, kp_bf16: torch.Tensor, tiles, scale
     tiles = np.ascontiguousarray(np.asarray(tiles, np.int32).reshape(-1, 4))
     out = np.empty(len(tiles), np.float64)
     lib().pa_oracle_block_score_tiles(_i(N), _i(G), _i(d), _p(_proxy_bits(qp_bf16)),
-                                      _p(_proxy_bits(kp_bf16)), _d(scale), _i(stride), _i(len(tiles)),
+                                      _p(_proxy_bits(kp_bf16)), _d(scale), _i(stride), _i(int(causal)),
+                                      _i(len(tiles)),
                                       _p(tiles), _p(out))
     return out
 
 
-def head_mass(q: torch.Tensor, k: torch.Tensor, scale: float | None = None, with_rowsum=False):
+def head_mass(q: torch.Tensor, k: torch.Tensor, scale: float | None = None, with_rowsum=False,
+              causal: bool = True):
     """o3: mass [B, H, nb] fp64 (and, optionally, max |row sum - 1| per (b, h))."""
     B, N, H, d = q.shape
     Hkv = k.shape[2]
@@ -141,23 +153,23 @@ def head_mass(q: torch.Tensor, k: torch.Tensor, scale: float | None = None, with
     lib().pa_oracle_head_mass(_i(B), _i(N), _i(H), _i(Hkv), _i(d),
                               _p(qa), _i64(qs[0]), _i64(qs[1]), _i64(qs[2]),
                               _p(ka), _i64(ks[0]), _i64(ks[1]), _i64(ks[2]),
-                              _d(scale), _p(mass), _p(dev))
+                              _d(scale), _i(int(causal)), _p(mass), _p(dev))
     return (mass, dev) if with_rowsum else mass
 
 
-def rank(scores: np.ndarray, nb: int) -> np.ndarray:
+def rank(scores: np.ndarray, nb: int, causal: bool = True) -> np.ndarray:
     """o4a: ranked lists [B, G, T] int32 from block scores [B, G, T] (any float dtype;
     converted exactly to fp64)."""
     s = np.ascontiguousarray(np.asarray(scores, dtype=np.float64))
     B, G, T = s.shape
-    assert T == nb * (nb + 1) // 2
+    assert T == rows_total(nb, causal)
     out = np.empty((B, G, T), np.int32)
-    lib().pa_oracle_rank(_i(B), _i(G), _i(nb), _p(s), _p(out))
+    lib().pa_oracle_rank(_i(B), _i(G), _i(nb), _p(s), _i(int(causal)), _p(out))
     return out
 
 
 def budget(rank_lists: np.ndarray, mass, H: int, G: int, nb: int, mode: int = DYNAMIC,
-           gamma: float = 0.95, frac_permille: int = 0):
+           gamma: float = 0.95, frac_permille: int = 0, causal: bool = True):
     """o4b: (budget [B, H] int32, cnt [B, H, nb] int32)."""
     r = np.ascontiguousarray(np.asarray(rank_lists, np.int32))
     B = r.shape[0]
@@ -168,11 +180,11 @@ def budget(rank_lists: np.ndarray, mass, H: int, G: int, nb: int, mode: int = DY
     bud = np.empty((B, H), np.int32)
     cnt = np.empty((B, H, nb), np.int32)
     lib().pa_oracle_budget(_i(B), _i(H), _i(G), _i(nb), _i(mode), _d(gamma), _i(frac_permille),
-                           _p(r), _p(m), _p(bud), _p(cnt))
+                           _p(r), _p(m), _i(int(causal)), _p(bud), _p(cnt))
     return bud, cnt
 
 
-def sparse_attn(q, k, v, rank_lists, cnt, G: int, items, scale: float | None = None):
+def sparse_attn(q, k, v, rank_lists, cnt, G: int, items, scale: float | None = None, causal: bool = True):
     """o5: for items [n, 3] of (b, h, qb) returns (O [n, 128, d], lse [n, 128]) fp64."""
     B, N, H, d = q.shape
     Hkv = k.shape[2]
@@ -189,12 +201,13 @@ def sparse_attn(q, k, v, rank_lists, cnt, G: int, items, scale: float | None = N
                                 _p(qa), _i64(qs[0]), _i64(qs[1]), _i64(qs[2]),
                                 _p(ka), _i64(ks[0]), _i64(ks[1]), _i64(ks[2]),
                                 _p(va), _i64(vs[0]), _i64(vs[1]), _i64(vs[2]),
-                                _p(r), _p(c), _d(scale), _i(len(items)), _p(items), _p(out), _p(lse))
+                                _p(r), _p(c), _d(scale), _i(int(causal)), _i(len(items)), _p(items), _p(out),
+                                _p(lse))
     return out, lse
 
 
 def sparse_attn_skip(q, k, v, rank_lists, cnt, G: int, items, lam: float, skip_in=None,
-                     scale: float | None = None):
+                     scale: float | None = None, causal: bool = True):
     """o7: o5 with the running-max block skip at threshold lam.  Returns
     (O [n, 128, d], lse [n, 128], skip [B, H, T] uint8, gap [B, H, T] fp64):
     skip and gap hold the oracle's own decision and its margin (log2 units)
@@ -204,7 +217,7 @@ def sparse_attn_skip(q, k, v, rank_lists, cnt, G: int, items, lam: float, skip_i
     B, N, H, d = q.shape
     Hkv = k.shape[2]
     nb = N // BLK
-    T = nb * (nb + 1) // 2
+    T = rows_total(nb, causal)
     scale = 1.0 / np.sqrt(d) if scale is None else scale
     qa, qs = _bits(q)
     ka, ks = _bits(k)
@@ -221,7 +234,7 @@ def sparse_attn_skip(q, k, v, rank_lists, cnt, G: int, items, lam: float, skip_i
                                      _p(qa), _i64(qs[0]), _i64(qs[1]), _i64(qs[2]),
                                      _p(ka), _i64(ks[0]), _i64(ks[1]), _i64(ks[2]),
                                      _p(va), _i64(vs[0]), _i64(vs[1]), _i64(vs[2]),
-                                     _p(r), _p(c), _d(scale), _d(lam), _i(len(items)), _p(items),
+                                     _p(r), _p(c), _d(scale), _d(lam), _i(int(causal)), _i(len(items)), _p(items),
                                      _p(sin) if sin is not None else None, _p(skip), _p(gap), _p(out), _p(lse))
     return out, lse, skip, gap
 
@@ -252,7 +265,7 @@ def find_blocks(mass, nb: int, tau: float):
     return rank, cnt
 
 
-def dense_attn(q, k, v, rows, scale: float | None = None):
+def dense_attn(q, k, v, rows, scale: float | None = None, causal: bool = True):
     """o6: for rows [n, 3] of (b, h, i) returns (O [n, d], lse [n]) fp64."""
     B, N, H, d = q.shape
     Hkv = k.shape[2]
@@ -267,18 +280,18 @@ def dense_attn(q, k, v, rows, scale: float | None = None):
                                _p(qa), _i64(qs[0]), _i64(qs[1]), _i64(qs[2]),
                                _p(ka), _i64(ks[0]), _i64(ks[1]), _i64(ks[2]),
                                _p(va), _i64(vs[0]), _i64(vs[1]), _i64(vs[2]),
-                               _d(scale), _i(len(rows)), _p(rows), _p(out), _p(lse))
+                               _d(scale), _i(int(causal)), _i(len(rows)), _p(rows), _p(out), _p(lse))
     return out, lse
 
 
-def prefill_masks(q, k, G: int, mode=DYNAMIC, gamma=0.95, frac_permille=0, stride=1):
+def prefill_masks(q, k, G: int, mode=DYNAMIC, gamma=0.95, frac_permille=0, stride=1, causal=True):
     """o1-o4 end to end on the oracle's own fp64 scores and masses:
     dict(qp, kp, scores, mass, rank, budget, cnt)."""
     B, N, H, d = q.shape
     nb = N // BLK
     _, _, qpb, kpb = pool(q, k, G)
-    scores = block_scores(qpb, kpb, stride=stride)
-    mass = head_mass(q, k) if mode == DYNAMIC else None
-    r = rank(scores, nb)
-    bud, cnt = budget(r, mass, H, G, nb, mode, gamma, frac_permille)
+    scores = block_scores(qpb, kpb, stride=stride, causal=causal)
+    mass = head_mass(q, k, causal=causal) if mode == DYNAMIC else None
+    r = rank(scores, nb, causal)
+    bud, cnt = budget(r, mass, H, G, nb, mode, gamma, frac_permille, causal)
     return dict(qp=qpb, kp=kpb, scores=scores, mass=mass, rank=r, budget=bud, cnt=cnt)

@@ -93,6 +93,14 @@ uint16_t pa_oracle_f64_to_bf16(double x)
 
 static inline int64_t tri(int64_t qb) { return qb * (qb + 1) / 2; }
 
+/* Per-(b, g) arrays of block scores and ranked lists.  Causal: row qb holds
+ * the blocks 0..qb at offset tri(qb) (T = tri(nb) entries).  Non-causal
+ * (every query attends to every key; the pages' DiT use, XAttention blog
+ * "video generation"): row qb holds all nb blocks at offset qb*nb. */
+static inline int64_t row_at(int causal, int nb, int qb) { return causal ? tri(qb) : (int64_t)qb * nb; }
+static inline int64_t rows_total(int causal, int nb) { return causal ? tri(nb) : (int64_t)nb * nb; }
+static inline int row_len(int causal, int nb, int qb) { return causal ? qb + 1 : nb; }
+
 /* q head h -> its KV head (GQA) and its proxy group. */
 static inline int kv_of(int h, int H, int Hkv) { return (int)((int64_t)h * Hkv / H); }
 static inline int grp_of(int h, int H, int G) { return (int)((int64_t)h * G / H); }
@@ -141,14 +149,14 @@ void pa_oracle_pool(int B, int N, int H, int Hkv, int d, int G,
  * rows, the one whose causal key range covers the others'.  r = 1 scores
  * every row. */
 static double tile_score(const uint16_t *qp, const uint16_t *kp, int d, int qb, int kb, double scale,
-                         int stride)
+                         int stride, int causal)
 {
     double best = -INFINITY;
     for (int ii = stride - 1; ii < BLK; ii += stride) {
         int i = qb * BLK + ii;
         for (int jj = 0; jj < BLK; jj++) {
             int j = kb * BLK + jj;
-            if (j > i) continue;
+            if (causal && j > i) continue;
             double s = 0.0;
             for (int c = 0; c < d; c++)
                 s += bf16_to_f64(qp[(int64_t)i * d + c]) * bf16_to_f64(kp[(int64_t)j * d + c]);
@@ -161,33 +169,33 @@ static double tile_score(const uint16_t *qp, const uint16_t *kp, int d, int qb, 
 
 void pa_oracle_block_scores(int B, int N, int G, int d,
                             const uint16_t *qp, const uint16_t *kp, double scale,
-                            int stride, double *scores)
+                            int stride, int causal, double *scores)
 {
     int nb = N / BLK;
-    int64_t T = tri(nb);
+    int64_t T = rows_total(causal, nb);
     #pragma omp parallel for collapse(3) schedule(dynamic, 1)
     for (int b = 0; b < B; b++)
         for (int g = 0; g < G; g++)
             for (int qb = 0; qb < nb; qb++) {
                 const uint16_t *qpg = qp + ((int64_t)b * G + g) * N * d;
                 const uint16_t *kpg = kp + ((int64_t)b * G + g) * N * d;
-                for (int kb = 0; kb <= qb; kb++)
-                    scores[((int64_t)b * G + g) * T + tri(qb) + kb] =
-                        tile_score(qpg, kpg, d, qb, kb, scale, stride);
+                for (int kb = 0; kb < row_len(causal, nb, qb); kb++)
+                    scores[((int64_t)b * G + g) * T + row_at(causal, nb, qb) + kb] =
+                        tile_score(qpg, kpg, d, qb, kb, scale, stride, causal);
             }
 }
 
 /* Score of a list of single tiles (b, g, qb, kb): used to sample large sizes. */
 void pa_oracle_block_score_tiles(int N, int G, int d, const uint16_t *qp, const uint16_t *kp,
-                                 double scale, int stride, int n_tiles, const int32_t *tiles /* [n][4] */,
-                                 double *out)
+                                 double scale, int stride, int causal, int n_tiles,
+                                 const int32_t *tiles /* [n][4] */, double *out)
 {
     #pragma omp parallel for schedule(dynamic, 1)
     for (int t = 0; t < n_tiles; t++) {
         int b = tiles[4 * t], g = tiles[4 * t + 1], qb = tiles[4 * t + 2], kb = tiles[4 * t + 3];
         const uint16_t *qpg = qp + ((int64_t)b * G + g) * N * d;
         const uint16_t *kpg = kp + ((int64_t)b * G + g) * N * d;
-        out[t] = tile_score(qpg, kpg, d, qb, kb, scale, stride);
+        out[t] = tile_score(qpg, kpg, d, qb, kb, scale, stride, causal);
     }
 }
 
@@ -200,7 +208,7 @@ void pa_oracle_block_score_tiles(int N, int G, int d, const uint16_t *qp, const 
 void pa_oracle_head_mass(int B, int N, int H, int Hkv, int d,
                          const uint16_t *q, int64_t qsb, int64_t qss, int64_t qsh,
                          const uint16_t *k, int64_t ksb, int64_t kss, int64_t ksh,
-                         double scale, double *mass, double *rowsum_dev)
+                         double scale, int causal, double *mass, double *rowsum_dev)
 {
     int nb = N / BLK;
     #pragma omp parallel for collapse(2) schedule(dynamic, 1)
@@ -212,8 +220,9 @@ void pa_oracle_head_mass(int B, int N, int H, int Hkv, int d,
             double dev = 0.0;
             for (int kb = 0; kb < nb; kb++) m[kb] = 0.0;
             for (int i = N - BLK; i < N; i++) {
+                int jhi = causal ? i + 1 : N;  /* keys j < jhi */
                 double zmax = -INFINITY;
-                for (int j = 0; j <= i; j++) {
+                for (int j = 0; j < jhi; j++) {
                     double s = 0.0;
                     for (int c = 0; c < d; c++)
                         s += bf16_to_f64(q[b * qsb + (int64_t)i * qss + h * qsh + c]) *
@@ -222,9 +231,9 @@ void pa_oracle_head_mass(int B, int N, int H, int Hkv, int d,
                     if (z[j] > zmax) zmax = z[j];
                 }
                 double den = 0.0;
-                for (int j = 0; j <= i; j++) den += exp(z[j] - zmax);
+                for (int j = 0; j < jhi; j++) den += exp(z[j] - zmax);
                 double rs = 0.0;
-                for (int j = 0; j <= i; j++) {
+                for (int j = 0; j < jhi; j++) {
                     double p = exp(z[j] - zmax) / den;
                     m[j / BLK] += p / BLK;
                     rs += p;
@@ -248,27 +257,31 @@ static int by_score_desc_then_index(const void *pa, const void *pb)
     return (a->kb < b->kb) ? -1 : (a->kb > b->kb);
 }
 
-/* Ranked list of query block qb of every (b, g): [0, qb, then the blocks
- * 1..qb-1 in (score desc, index asc) order]; [0] alone at qb = 0.
- * rank[b][g][tri(qb)+t]. */
-void pa_oracle_rank(int B, int G, int nb, const double *scores, int32_t *rank)
+/* Ranked list of query block qb of every (b, g): [0, qb, then the other
+ * blocks of the row (1..qb-1 causal, all but 0 and qb non-causal) in (score
+ * desc, index asc) order]; at qb = 0 the sink is the diagonal and leads
+ * alone.  rank[b][g][row_at(qb)+t]. */
+void pa_oracle_rank(int B, int G, int nb, const double *scores, int causal, int32_t *rank)
 {
-    int64_t T = tri(nb);
+    int64_t T = rows_total(causal, nb);
     #pragma omp parallel for collapse(3) schedule(dynamic, 4)
     for (int b = 0; b < B; b++)
         for (int g = 0; g < G; g++)
             for (int qb = 0; qb < nb; qb++) {
-                const double *row = scores + ((int64_t)b * G + g) * T + tri(qb);
-                int32_t *out = rank + ((int64_t)b * G + g) * T + tri(qb);
+                const double *row = scores + ((int64_t)b * G + g) * T + row_at(causal, nb, qb);
+                int32_t *out = rank + ((int64_t)b * G + g) * T + row_at(causal, nb, qb);
+                int len = row_len(causal, nb, qb);
                 out[0] = 0;
-                if (qb == 0) continue;
-                out[1] = qb;
-                int n = qb - 1;
+                if (qb > 0) out[1] = qb;
+                int lead = qb > 0 ? 2 : 1;
+                int n = len - lead;
                 if (n == 0) continue;
                 keyed *tmp = (keyed *)malloc(sizeof(keyed) * n);
-                for (int t = 0; t < n; t++) { tmp[t].s = row[t + 1]; tmp[t].kb = t + 1; }
+                int m = 0;
+                for (int kb = 1; kb < len; kb++)
+                    if (kb != qb) { tmp[m].s = row[kb]; tmp[m].kb = kb; m++; }
                 qsort(tmp, n, sizeof(keyed), by_score_desc_then_index);
-                for (int t = 0; t < n; t++) out[2 + t] = tmp[t].kb;
+                for (int t = 0; t < n; t++) out[lead + t] = tmp[t].kb;
                 free(tmp);
             }
 }
@@ -284,19 +297,21 @@ static inline int clampi(int64_t x, int lo, int hi) { return (int)(x < lo ? lo :
  * DYNAMIC: fixed-point masses m_fx = rint(mass * 2^40), gamma_fx = rint(gamma *
  *   2^40); k_h = the smallest k >= |F_last| whose prefix of the last row's list
  *   (group grp(h)) carries sum m_fx >= gamma_fx, or nb if none does;
- *   cnt = clamp(ceil(k_h (qb+1) / nb), |F_qb|, qb+1).
- * FIXED_FRACTION: cnt = clamp(ceil(p (qb+1) / 1000), |F_qb|, qb+1), p per mille.
- * ALL: cnt = qb+1.  budget[b][h] = cnt at the last row. */
+ *   cnt = clamp(ceil(k_h (qb+1) / nb), |F_qb|, qb+1) causal; non-causal every
+ *   row has nb blocks, so cnt = clamp(k_h, |F_qb|, nb).
+ * FIXED_FRACTION: cnt = clamp(ceil(p (qb+1) / 1000), |F_qb|, qb+1), p per mille
+ *   (non-causal: ceil(p nb / 1000), up to nb).
+ * ALL: cnt = the row's length.  budget[b][h] = cnt at the last row. */
 void pa_oracle_budget(int B, int H, int G, int nb, int mode, double gamma, int frac_permille,
-                      const int32_t *rank, const double *mass, int32_t *budget, int32_t *cnt)
+                      const int32_t *rank, const double *mass, int causal, int32_t *budget, int32_t *cnt)
 {
-    int64_t T = tri(nb);
+    int64_t T = rows_total(causal, nb);
     for (int b = 0; b < B; b++)
         for (int h = 0; h < H; h++) {
             int g = grp_of(h, H, G);
             int32_t *c = cnt + ((int64_t)b * H + h) * nb;
             if (mode == ORACLE_DYNAMIC) {
-                const int32_t *last = rank + ((int64_t)b * G + g) * T + tri(nb - 1);
+                const int32_t *last = rank + ((int64_t)b * G + g) * T + row_at(causal, nb, nb - 1);
                 const double *m = mass + ((int64_t)b * H + h) * nb;
                 int64_t gfx = llrint(gamma * 1099511627776.0);
                 int64_t cum = 0;
@@ -307,13 +322,15 @@ void pa_oracle_budget(int B, int H, int G, int nb, int mode, double gamma, int f
                 }
                 budget[(int64_t)b * H + h] = kh;
                 for (int qb = 0; qb < nb; qb++)
-                    c[qb] = clampi(((int64_t)kh * (qb + 1) + nb - 1) / nb, forced(qb), qb + 1);
+                    c[qb] = causal ? clampi(((int64_t)kh * (qb + 1) + nb - 1) / nb, forced(qb), qb + 1)
+                                   : clampi(kh, forced(qb), nb);
             } else if (mode == ORACLE_FIXED_FRACTION) {
                 for (int qb = 0; qb < nb; qb++)
-                    c[qb] = clampi(((int64_t)frac_permille * (qb + 1) + 999) / 1000, forced(qb), qb + 1);
+                    c[qb] = causal ? clampi(((int64_t)frac_permille * (qb + 1) + 999) / 1000, forced(qb), qb + 1)
+                                   : clampi(((int64_t)frac_permille * nb + 999) / 1000, forced(qb), nb);
                 budget[(int64_t)b * H + h] = c[nb - 1];
             } else {
-                for (int qb = 0; qb < nb; qb++) c[qb] = qb + 1;
+                for (int qb = 0; qb < nb; qb++) c[qb] = row_len(causal, nb, qb);
                 budget[(int64_t)b * H + h] = nb;
             }
         }
@@ -329,17 +346,17 @@ void pa_oracle_sparse_attn(int N, int H, int Hkv, int d, int G,
                            const uint16_t *q, int64_t qsb, int64_t qss, int64_t qsh,
                            const uint16_t *k, int64_t ksb, int64_t kss, int64_t ksh,
                            const uint16_t *v, int64_t vsb, int64_t vss, int64_t vsh,
-                           const int32_t *rank, const int32_t *cnt, double scale,
+                           const int32_t *rank, const int32_t *cnt, double scale, int causal,
                            int n_items, const int32_t *items /* [n][3] = b,h,qb */,
                            double *out, double *lse)
 {
     int nb = N / BLK;
-    int64_t T = tri(nb);
+    int64_t T = rows_total(causal, nb);
     #pragma omp parallel for schedule(dynamic, 1)
     for (int it = 0; it < n_items; it++) {
         int b = items[3 * it], h = items[3 * it + 1], qb = items[3 * it + 2];
         int g = grp_of(h, H, G), kvh = kv_of(h, H, Hkv);
-        const int32_t *list = rank + ((int64_t)b * G + g) * T + tri(qb);
+        const int32_t *list = rank + ((int64_t)b * G + g) * T + row_at(causal, nb, qb);
         int n = cnt[((int64_t)b * H + h) * nb + qb];
         double *z = (double *)malloc(sizeof(double) * n * BLK);
         for (int ii = 0; ii < BLK; ii++) {
@@ -349,7 +366,7 @@ void pa_oracle_sparse_attn(int N, int H, int Hkv, int d, int G,
                 for (int jj = 0; jj < BLK; jj++) {
                     int j = list[t] * BLK + jj;
                     double s = -INFINITY;
-                    if (j <= i) {
+                    if (!causal || j <= i) {
                         s = 0.0;
                         for (int c = 0; c < d; c++)
                             s += bf16_to_f64(q[b * qsb + (int64_t)i * qss + h * qsh + c]) *
@@ -402,20 +419,20 @@ void pa_oracle_sparse_attn_skip(int N, int H, int Hkv, int d, int G,
                                 const uint16_t *k, int64_t ksb, int64_t kss, int64_t ksh,
                                 const uint16_t *v, int64_t vsb, int64_t vss, int64_t vsh,
                                 const int32_t *rank, const int32_t *cnt, double scale, double lambda,
-                                int n_items, const int32_t *items /* [n][3] = b,h,qb */,
+                                int causal, int n_items, const int32_t *items /* [n][3] = b,h,qb */,
                                 const uint8_t *skip_in, uint8_t *skip_out, double *gap,
                                 double *out, double *lse)
 {
     int nb = N / BLK;
-    int64_t T = tri(nb);
+    int64_t T = rows_total(causal, nb);
     double lnl = (lambda > 0.0) ? log(lambda) : -INFINITY;
     #pragma omp parallel for schedule(dynamic, 1)
     for (int it = 0; it < n_items; it++) {
         int b = items[3 * it], h = items[3 * it + 1], qb = items[3 * it + 2];
         int g = grp_of(h, H, G), kvh = kv_of(h, H, Hkv);
-        const int32_t *list = rank + ((int64_t)b * G + g) * T + tri(qb);
+        const int32_t *list = rank + ((int64_t)b * G + g) * T + row_at(causal, nb, qb);
         int n = cnt[((int64_t)b * H + h) * nb + qb];
-        int64_t base = ((int64_t)b * H + h) * T + tri(qb);
+        int64_t base = ((int64_t)b * H + h) * T + row_at(causal, nb, qb);
         int *blk = (int *)malloc(sizeof(int) * (n > 0 ? n : 1));
         double *mt = (double *)malloc(sizeof(double) * BLK * (n > 0 ? n : 1));
         unsigned char *use = (unsigned char *)malloc(n > 0 ? n : 1);
@@ -433,7 +450,7 @@ void pa_oracle_sparse_attn_skip(int N, int H, int Hkv, int d, int G,
                 double best = -INFINITY;
                 for (int jj = 0; jj < BLK; jj++) {
                     int j = blk[t] * BLK + jj;
-                    if (j > i) continue;
+                    if (causal && j > i) continue;
                     double s = 0.0;
                     for (int c = 0; c < d; c++)
                         s += bf16_to_f64(q[b * qsb + (int64_t)i * qss + h * qsh + c]) *
@@ -478,7 +495,7 @@ void pa_oracle_sparse_attn_skip(int N, int H, int Hkv, int d, int G,
                     if (!use[t]) continue;
                     for (int jj = 0; jj < BLK; jj++) {
                         int j = blk[t] * BLK + jj;
-                        if (j > i) continue;
+                        if (causal && j > i) continue;
                         double s = 0.0;
                         for (int c = 0; c < d; c++)
                             s += bf16_to_f64(q[b * qsb + (int64_t)i * qss + h * qsh + c]) *
@@ -597,17 +614,17 @@ void pa_oracle_dense_attn(int N, int H, int Hkv, int d,
                           const uint16_t *q, int64_t qsb, int64_t qss, int64_t qsh,
                           const uint16_t *k, int64_t ksb, int64_t kss, int64_t ksh,
                           const uint16_t *v, int64_t vsb, int64_t vss, int64_t vsh,
-                          double scale, int n_rows, const int32_t *rows /* [n][3] = b,h,i */,
+                          double scale, int causal, int n_rows, const int32_t *rows /* [n][3] = b,h,i */,
                           double *out, double *lse)
 {
-    (void)N;
     #pragma omp parallel for schedule(dynamic, 4)
     for (int r = 0; r < n_rows; r++) {
         int b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
         int kvh = kv_of(h, H, Hkv);
-        double *z = (double *)malloc(sizeof(double) * (i + 1));
+        int nkeys = causal ? i + 1 : N;  /* keys 0 .. nkeys-1 */
+        double *z = (double *)malloc(sizeof(double) * nkeys);
         double zmax = -INFINITY;
-        for (int j = 0; j <= i; j++) {
+        for (int j = 0; j < nkeys; j++) {
             double s = 0.0;
             for (int c = 0; c < d; c++)
                 s += bf16_to_f64(q[b * qsb + (int64_t)i * qss + h * qsh + c]) *
@@ -616,10 +633,10 @@ void pa_oracle_dense_attn(int N, int H, int Hkv, int d,
             if (z[j] > zmax) zmax = z[j];
         }
         double den = 0.0;
-        for (int j = 0; j <= i; j++) den += exp(z[j] - zmax);
+        for (int j = 0; j < nkeys; j++) den += exp(z[j] - zmax);
         double *o = out + (int64_t)r * d;
         for (int c = 0; c < d; c++) o[c] = 0.0;
-        for (int j = 0; j <= i; j++) {
+        for (int j = 0; j < nkeys; j++) {
             double p = exp(z[j] - zmax) / den;
             for (int c = 0; c < d; c++)
                 o[c] += p * bf16_to_f64(v[b * vsb + (int64_t)j * vss + kvh * vsh + c]);

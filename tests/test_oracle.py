@@ -719,3 +719,86 @@ def test_find_blocks_brute_force():
                 best = min(len(s) for r in range(1, qb + 2) for s in itertools.combinations(range(qb + 1), r)
                            if v[list(s)].sum() >= tau - 1e-12) if v.sum() >= tau - 1e-12 else qb + 1
                 assert cnt[0, h, qb] == best
+
+
+# --------------------------------------------------------- non-causal mode
+def test_noncausal_dense_and_sparse_all_match_sdpa():
+    """Non-causal: o6 equals torch SDPA without a mask (fp64, GQA), and o5 with
+    every block selected equals o6."""
+    w = synth.small_workload(seqlen=384, heads=4, kv_heads=2, head_dim=64)
+    x = synth.make_inputs(w)
+    q, k, v = x["q"], x["k"], x["v"]
+    N = 384
+    ref = sdpa_reference(q, k, v, mask=torch.ones(N, N, dtype=torch.bool))
+    rows = [(0, h, i) for h in range(4) for i in (0, 5, 127, 200, 383)]
+    od, lsed = oracle.dense_attn(q, k, v, rows, causal=False)
+    for (b, h, i), oo in zip(rows, od):
+        np.testing.assert_allclose(oo, ref[b, i, h].numpy(), rtol=1e-12, atol=1e-12)
+    for (b, h, i), l in zip(rows, lsed):
+        z = (q[b, i, h].double() @ k[b, :, h * 2 // 4].double().T) / 8.0
+        assert l == pytest.approx(torch.logsumexp(z, 0).item(), abs=1e-12)
+    m = oracle.prefill_masks(q, k, 1, mode=oracle.ALL, causal=False)
+    assert list(m["cnt"][0, 0]) == [3, 3, 3]
+    items = [(0, h, qb) for h in range(4) for qb in range(3)]
+    o, lse = oracle.sparse_attn(q, k, v, m["rank"], m["cnt"], 1, items, causal=False)
+    rows2 = [(0, h, qb * 128 + i) for (_, h, qb) in items for i in range(128)]
+    od2, lsed2 = oracle.dense_attn(q, k, v, rows2, causal=False)
+    np.testing.assert_allclose(o.reshape(-1, 64), od2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse.reshape(-1), lsed2, rtol=0, atol=1e-12)
+
+
+def test_noncausal_sparse_matches_sdpa_with_block_mask():
+    w = synth.small_workload(seqlen=512, heads=4, kv_heads=2, head_dim=64, groups=2)
+    x = synth.make_inputs(w)
+    q, k, v = x["q"], x["k"], x["v"]
+    m = oracle.prefill_masks(q, k, 2, mode=oracle.FIXED_FRACTION, frac_permille=500, causal=False)
+    nb = 4
+    assert (m["cnt"] == 2).all()  # ceil(0.5 * 4)
+    mask = torch.zeros(4, 512, 512, dtype=torch.bool)
+    for h in range(4):
+        g = h * 2 // 4
+        for qb in range(nb):
+            for kb in m["rank"][0, g, qb * nb: qb * nb + m["cnt"][0, h, qb]]:
+                mask[h, qb * 128:(qb + 1) * 128, kb * 128:(kb + 1) * 128] = True
+    ref = sdpa_reference(q, k, v, mask=mask[None])
+    items = [(0, h, qb) for h in range(4) for qb in range(nb)]
+    o, _ = oracle.sparse_attn(q, k, v, m["rank"], m["cnt"], 2, items, causal=False)
+    for (b, h, qb), oo in zip(items, o):
+        np.testing.assert_allclose(oo, ref[0, qb * 128:(qb + 1) * 128, h].numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_noncausal_scores_mass_rank_budget():
+    """Non-causal scores equal per-head unmasked numpy block maxima (G = H);
+    head mass rows equal scipy softmax over all keys; lists are [0, qb, rest by
+    score] over all nb blocks; counts are clamp(k_h, |F|, nb) and the fixed
+    fraction ceil(p nb / 1000)."""
+    w = synth.small_workload(seqlen=512, heads=3, kv_heads=3, head_dim=64, groups=3)
+    x = synth.make_inputs(w)
+    q, k = x["q"], x["k"]
+    nb = 4
+    _, _, qpb, kpb = oracle.pool(q, k, 3)
+    sc = oracle.block_scores(qpb, kpb, causal=False)
+    for h in range(3):
+        s = (q[0, :, h].double().numpy() @ k[0, :, h].double().numpy().T) / 8.0
+        ref = [s[a * 128:(a + 1) * 128, c * 128:(c + 1) * 128].max() for a in range(nb) for c in range(nb)]
+        np.testing.assert_allclose(sc[0, h], ref, rtol=1e-13, atol=1e-13)
+    mass = oracle.head_mass(q, k, causal=False)
+    for h in range(3):
+        z = (q[0, 384:, h].double().numpy() @ k[0, :, h].double().numpy().T) / 8.0
+        p = scipy.special.softmax(z, axis=1)
+        np.testing.assert_allclose(mass[0, h], p.reshape(128, nb, 128).sum(2).mean(0), rtol=1e-12, atol=1e-15)
+    r = oracle.rank(sc, nb, causal=False)
+    for h in range(3):
+        for qb in range(nb):
+            lst = list(r[0, h, qb * nb:(qb + 1) * nb])
+            rest = sorted((kb for kb in range(1, nb) if kb != qb), key=lambda kb: (-sc[0, h, qb * nb + kb], kb))
+            assert lst == ([0] + ([qb] if qb else []) + rest)
+    bud, cnt = oracle.budget(r, mass, 3, 3, nb, oracle.DYNAMIC, 0.9, causal=False)
+    for h in range(3):
+        lst = r[0, h, (nb - 1) * nb:]
+        cum = np.cumsum([int(np.rint(mass[0, h, kb] * 2.0 ** 40)) for kb in lst])
+        kh = next(t + 1 for t in range(nb) if t + 1 >= 2 and cum[t] >= int(np.rint(0.9 * 2.0 ** 40)))
+        assert bud[0, h] == kh
+        assert list(cnt[0, h]) == [max(kh, 1)] + [max(kh, 2)] * (nb - 1)
+    _, cf = oracle.budget(r, None, 3, 3, nb, oracle.FIXED_FRACTION, 0, 300, causal=False)
+    assert (cf == 2).all()  # ceil(0.3 * 4) = 2

@@ -24,32 +24,27 @@ MUTANTS = [
     ("pool_no_rounding", "if (qp_bf16) qp_bf16[o] = pa_oracle_f64_to_bf16(mq);",
      "if (qp_bf16) qp_bf16[o] = pa_oracle_f64_to_bf16(mq * 1.001);"),
     ("rne_ties_away", "double r = nearbyint(x / q) * q;", "double r = round(x / q) * q;"),
-    ("scores_no_causal_mask", "            if (j > i) continue;\n            double s = 0.0;",
+    ("scores_no_causal_mask", "            if (causal && j > i) continue;\n            double s = 0.0;",
      "            double s = 0.0;"),
     ("scores_min_not_max", "\n            if (s > best) best = s;", "\n            if (best == -INFINITY || s < best) best = s;"),
     ("scores_no_scale", "            s *= scale;\n            if (s > best) best = s;", "            if (s > best) best = s;"),
     ("mass_not_mean_over_rows", "m[j / BLK] += p / BLK;", "m[j / BLK] += p;"),
-    ("mass_no_causal", [("for (int j = 0; j <= i; j++) {\n                    double s = 0.0;",
-                         "for (int j = 0; j < N; j++) {\n                    double s = 0.0;"),
-                        ("for (int j = 0; j <= i; j++) den += exp(z[j] - zmax);\n                double rs = 0.0;",
-                         "for (int j = 0; j < N; j++) den += exp(z[j] - zmax);\n                double rs = 0.0;"),
-                        ("for (int j = 0; j <= i; j++) {\n                    double p = exp(z[j] - zmax) / den;",
-                         "for (int j = 0; j < N; j++) {\n                    double p = exp(z[j] - zmax) / den;")], None),
+    ("mass_no_causal", "int jhi = causal ? i + 1 : N;", "int jhi = N;"),
     ("rank_ascending", "    if (a->s > b->s) return -1;\n    if (a->s < b->s) return 1;",
      "    if (a->s < b->s) return -1;\n    if (a->s > b->s) return 1;"),
     ("rank_ties_high_index_first", "return (a->kb < b->kb) ? -1 : (a->kb > b->kb);",
      "return (a->kb > b->kb) ? -1 : (a->kb < b->kb);"),
-    ("rank_no_forced_diagonal", "                out[1] = qb;\n                int n = qb - 1;",
-     "                out[1] = qb - 1 > 0 ? qb - 1 : qb;\n                int n = qb - 1;"),
+    ("rank_no_forced_diagonal", "if (qb > 0) out[1] = qb;", "if (qb > 0) out[1] = qb - 1 > 0 ? qb - 1 : qb;"),
     ("budget_off_by_one", "if (t + 1 >= forced(nb - 1) && cum >= gfx) { kh = t + 1; break; }",
      "if (t + 1 >= forced(nb - 1) && cum >= gfx) { kh = t + 2 > nb ? nb : t + 2; break; }"),
     ("budget_strict", "cum >= gfx) { kh = t + 1; break; }", "cum > gfx) { kh = t + 1; break; }"),
-    ("budget_floor_not_ceil", "c[qb] = clampi(((int64_t)kh * (qb + 1) + nb - 1) / nb, forced(qb), qb + 1);",
-     "c[qb] = clampi(((int64_t)kh * (qb + 1)) / nb, forced(qb), qb + 1);"),
-    ("fixed_floor_not_ceil", "c[qb] = clampi(((int64_t)frac_permille * (qb + 1) + 999) / 1000, forced(qb), qb + 1);",
-     "c[qb] = clampi(((int64_t)frac_permille * (qb + 1)) / 1000, forced(qb), qb + 1);"),
+    ("budget_floor_not_ceil", "clampi(((int64_t)kh * (qb + 1) + nb - 1) / nb, forced(qb), qb + 1)",
+     "clampi(((int64_t)kh * (qb + 1)) / nb, forced(qb), qb + 1)"),
+    ("fixed_floor_not_ceil", "clampi(((int64_t)frac_permille * (qb + 1) + 999) / 1000, forced(qb), qb + 1)",
+     "clampi(((int64_t)frac_permille * (qb + 1)) / 1000, forced(qb), qb + 1)"),
     ("sparse_unnormalised", "                    double p = exp(zz - zmax) / den;", "                    double p = exp(zz - zmax);"),
-    ("sparse_no_causal", "                    if (j <= i) {\n                        s = 0.0;", "                    if (1) {\n                        s = 0.0;"),
+    ("sparse_no_causal", "                    if (!causal || j <= i) {\n                        s = 0.0;",
+     "                    if (1) {\n                        s = 0.0;"),
     ("sparse_v_from_q_head", "o[c] += p * bf16_to_f64(v[b * vsb + (int64_t)j * vss + kvh * vsh + c]);\n                }\n            if (lse)",
      "o[c] += p * bf16_to_f64(v[b * vsb + (int64_t)j * vss + (h % Hkv) * vsh + c]);\n                }\n            if (lse)"),
     ("dense_wrong_scale", "            z[j] = scale * s;", "            z[j] = s;"),
@@ -74,6 +69,10 @@ MUTANTS = [
     ("xattn_scale_without_stride", "double scale = 1.0 / (sqrt((double)d) * S);", "double scale = 1.0 / sqrt((double)d);"),
     ("find_blocks_strict", "if (cum >= tfx) { n = t + 1; break; }", "if (cum > tfx) { n = t + 1; break; }"),
     ("find_blocks_ascending", "while (u > 0 && (m[out[u - 1]] < m[t] ||", "while (u > 0 && (m[out[u - 1]] > m[t] ||"),
+    ("noncausal_budget_row_scaled", ": clampi(kh, forced(qb), nb);",
+     ": clampi(((int64_t)kh * (qb + 1) + nb - 1) / nb, forced(qb), nb);"),
+    ("noncausal_dense_still_causal", "int nkeys = causal ? i + 1 : N;", "int nkeys = i + 1;"),
+    ("noncausal_rank_keeps_only_lower_blocks", "int len = row_len(causal, nb, qb);", "int len = qb + 1;"),
     ("skip_threshold_log2", "double lnl = (lambda > 0.0) ? log(lambda) : -INFINITY;",
      "double lnl = (lambda > 0.0) ? log2(lambda) : -INFINITY;"),
 ]
@@ -101,6 +100,8 @@ PINS = [
     lambda: T.test_xattn_mass_is_the_antidiagonal_sum_softmax(8),
     T.test_xattn_stride_one_is_the_exact_mass,
     T.test_find_blocks_brute_force,
+    T.test_noncausal_dense_and_sparse_all_match_sdpa,
+    T.test_noncausal_scores_mass_rank_budget,
     G.test_golden_rank,
     G.test_golden_budget,
 ]
