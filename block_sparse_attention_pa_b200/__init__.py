@@ -47,7 +47,7 @@ class PaError(RuntimeError):
 class Shape(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("seqlen", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("block", ctypes.c_int32),
-                ("num_groups", ctypes.c_int32)]
+                ("num_groups", ctypes.c_int32), ("non_causal", ctypes.c_int32)]
 
 
 class Strides(ctypes.Structure):
@@ -128,9 +128,14 @@ def _cuda_bf16(t: torch.Tensor, name: str):
         raise ValueError(f"{name} must be bf16 [B, N, heads, d] with a contiguous last dimension")
 
 
-def make_shape(q: torch.Tensor, k: torch.Tensor, num_groups: int) -> Shape:
+def make_shape(q: torch.Tensor, k: torch.Tensor, num_groups: int, causal: bool = True) -> Shape:
     B, N, H, d = q.shape
-    return Shape(B, N, H, k.shape[2], d, 128, num_groups)
+    return Shape(B, N, H, k.shape[2], d, 128, num_groups, 0 if causal else 1)
+
+
+def rows_total(nb: int, causal: bool = True) -> int:
+    """Entries of one (b, g) set of block scores or ranked lists."""
+    return nb * (nb + 1) // 2 if causal else nb * nb
 
 
 def make_budget(mode: int = DYNAMIC, gamma: float = 0.95, frac_permille: int = 0, score_stride: int = 1,
@@ -153,7 +158,7 @@ class Mask:
     @staticmethod
     def empty(shape: Shape, device, with_mass: bool) -> "Mask":
         nb = shape.seqlen // 128
-        T = nb * (nb + 1) // 2
+        T = rows_total(nb, not shape.non_causal)
         i32 = dict(device=device, dtype=torch.int32)
         return Mask(torch.empty(shape.batch, shape.num_groups, T, **i32),
                     torch.empty(shape.batch, shape.num_q_heads, nb, **i32),
@@ -166,12 +171,12 @@ class Mask:
                         self.mass.data_ptr() if self.mass is not None else None)
 
 
-def pool_heads(q: torch.Tensor, k: torch.Tensor, num_groups: int, score_stride: int = 1):
+def pool_heads(q: torch.Tensor, k: torch.Tensor, num_groups: int, score_stride: int = 1, causal: bool = True):
     """pa_pool_heads (score_stride 1) or pa_pool_heads_strided -> (q_proxy,
     k_proxy): q_proxy bf16 [B, G, N/score_stride, d], k_proxy [B, G, N, d]."""
     _cuda_bf16(q, "q")
     _cuda_bf16(k, "k")
-    shape = make_shape(q, k, num_groups)
+    shape = make_shape(q, k, num_groups, causal)
     B, N, H, d = q.shape
     r = int(score_stride)
     qp = torch.empty(B, num_groups, N // r if r in SCORE_STRIDES else N, d, device=q.device, dtype=torch.bfloat16)
@@ -186,7 +191,7 @@ def pool_heads(q: torch.Tensor, k: torch.Tensor, num_groups: int, score_stride: 
 
 
 def block_scores(q_proxy: torch.Tensor, k_proxy: torch.Tensor, num_q_heads: int = 1, num_kv_heads: int = 1,
-                 score_stride: int = 1):
+                 score_stride: int = 1, causal: bool = True):
     """pa_block_scores (score_stride 1) or pa_block_scores_strided -> fp32
     [B, G, T].  k_proxy is [B, G, N, d]; q_proxy [B, G, N/score_stride, d]."""
     for t, n in ((q_proxy, "q_proxy"), (k_proxy, "k_proxy")):
@@ -197,9 +202,9 @@ def block_scores(q_proxy: torch.Tensor, k_proxy: torch.Tensor, num_q_heads: int 
     if tuple(q_proxy.shape) != (B, G, N // max(r, 1), d):
         raise ValueError(f"q_proxy must be [B, G, N/{r}, d] = {(B, G, N // max(r, 1), d)}, got {tuple(q_proxy.shape)}")
     H = max(num_q_heads, G)
-    shape = Shape(B, N, H, min(num_kv_heads, H), d, 128, G)
+    shape = Shape(B, N, H, min(num_kv_heads, H), d, 128, G, 0 if causal else 1)
     nb = N // 128
-    scores = torch.empty(B, G, nb * (nb + 1) // 2, device=q_proxy.device, dtype=torch.float32)
+    scores = torch.empty(B, G, rows_total(nb, causal), device=q_proxy.device, dtype=torch.float32)
     if r == 1:
         _check(lib().pa_block_scores(ctypes.byref(shape), q_proxy.data_ptr(), k_proxy.data_ptr(), scores.data_ptr(),
                                      _stream(q_proxy.device)))
@@ -210,11 +215,12 @@ def block_scores(q_proxy: torch.Tensor, k_proxy: torch.Tensor, num_q_heads: int 
 
 
 def build_mask(scores: torch.Tensor, q: torch.Tensor, k: torch.Tensor, num_groups: int, mode: int = DYNAMIC,
-               gamma: float = 0.95, frac_permille: int = 0, workspace: torch.Tensor | None = None) -> Mask:
+               gamma: float = 0.95, frac_permille: int = 0, workspace: torch.Tensor | None = None,
+               causal: bool = True) -> Mask:
     """pa_build_mask -> Mask."""
     _cuda_bf16(q, "q")
     _cuda_bf16(k, "k")
-    shape = make_shape(q, k, num_groups)
+    shape = make_shape(q, k, num_groups, causal)
     budget = make_budget(mode, gamma, frac_permille)
     mask = Mask.empty(shape, q.device, mode == DYNAMIC)
     if workspace is None:
@@ -251,18 +257,18 @@ def xattn_mask(q: torch.Tensor, k: torch.Tensor, stride: int = 8, tau: float = 0
 
 def block_sparse_attn(q, k, v, rank, cnt, num_groups: int, softmax_scale: float | None = None,
                       out: torch.Tensor | None = None, return_lse: bool = False, skip_threshold: float = 0.0,
-                      return_skipped: bool = False):
+                      return_skipped: bool = False, causal: bool = True):
     """pa_block_sparse_attn (skip_threshold 0) or pa_block_sparse_attn_skip ->
     o (bf16 [B, N, H, d]) [, lse fp32 [B, H, N]] [, skipped uint8 [B, H, T]]."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _cuda_bf16(t, n)
-    shape = make_shape(q, k, num_groups)
+    shape = make_shape(q, k, num_groups, causal)
     B, N, H, d = q.shape
     nb = N // 128
     scale = 1.0 / math.sqrt(d) if softmax_scale is None else softmax_scale
     o = torch.empty_like(q, memory_format=torch.contiguous_format) if out is None else out
     lse = torch.empty(B, H, N, device=q.device, dtype=torch.float32) if return_lse else None
-    skipped = torch.zeros(B, H, nb * (nb + 1) // 2, device=q.device, dtype=torch.uint8) if return_skipped else None
+    skipped = torch.zeros(B, H, rows_total(nb, causal), device=q.device, dtype=torch.uint8) if return_skipped else None
     lse_p = lse.data_ptr() if lse is not None else None
     if skip_threshold == 0.0 and not return_skipped:
         _check(lib().pa_block_sparse_attn(ctypes.byref(shape), q.data_ptr(), _strides(q), k.data_ptr(), _strides(k),
@@ -282,10 +288,10 @@ class Prefill:
     """A reusable pa_prefill call: workspace and mask buffers allocated once."""
 
     def __init__(self, q, k, v, num_groups: int, mode: int = DYNAMIC, gamma: float = 0.95, frac_permille: int = 0,
-                 score_stride: int = 1, skip_threshold: float = 0.0):
+                 score_stride: int = 1, skip_threshold: float = 0.0, causal: bool = True):
         for t, n in ((q, "q"), (k, "k"), (v, "v")):
             _cuda_bf16(t, n)
-        self.shape = make_shape(q, k, num_groups)
+        self.shape = make_shape(q, k, num_groups, causal)
         self.budget = make_budget(mode, gamma, frac_permille, score_stride, skip_threshold)
         self.mask = Mask.empty(self.shape, q.device, mode == DYNAMIC)
         self.ws = torch.empty(workspace_size(self.shape, self.budget), device=q.device, dtype=torch.uint8)
@@ -300,9 +306,9 @@ class Prefill:
 
 
 def prefill(q, k, v, num_groups: int, mode: int = DYNAMIC, gamma: float = 0.95, frac_permille: int = 0,
-            score_stride: int = 1, skip_threshold: float = 0.0):
+            score_stride: int = 1, skip_threshold: float = 0.0, causal: bool = True):
     """pa_prefill -> (o, Mask)."""
-    call = Prefill(q, k, v, num_groups, mode, gamma, frac_permille, score_stride, skip_threshold)
+    call = Prefill(q, k, v, num_groups, mode, gamma, frac_permille, score_stride, skip_threshold, causal)
     o = torch.empty_like(q, memory_format=torch.contiguous_format)
     call(q, k, v, o)
     return o, call.mask

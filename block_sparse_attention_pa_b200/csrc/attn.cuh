@@ -67,6 +67,7 @@ struct AttnParams {
     __nv_bfloat16 *o;
     int64_t osb, oss, osh;
     float *lse;                // [B][H][N] or nullptr
+    int causal;                // 1: keys j <= i, rows at qb(qb+1)/2; 0: every key, rows at qb*nb
     float skip_log2;           // SKIP: log2(lambda) (lambda in (0, 1])
     uint8_t *skipped;          // SKIP: [B][H][T], 1 written for every skipped block, or nullptr
     uint64_t timeout_ns;
@@ -181,8 +182,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int h0 = p.unit_h0[unit];
     const int h1 = p.unit_h1[unit];
     const int kvh = static_cast<int>(static_cast<long long>(h0) * p.Hkv / p.H);
-    const long long T = static_cast<long long>(p.nb) * (p.nb + 1) / 2;
-    const long long row_off = static_cast<long long>(qb) * (qb + 1) / 2;
+    const long long T = p.causal ? static_cast<long long>(p.nb) * (p.nb + 1) / 2 : static_cast<long long>(p.nb) * p.nb;
+    const long long row_off = p.causal ? static_cast<long long>(qb) * (qb + 1) / 2 : static_cast<long long>(qb) * p.nb;
+    const int row_len = p.causal ? qb + 1 : p.nb;  // blocks in this query block's list
     const int32_t *list0 =
         p.rank + (static_cast<long long>(b) * p.G + static_cast<long long>(h0) * p.G / p.H) * T + row_off;
     const int32_t *list1 =
@@ -192,9 +194,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     craw[0] = p.cnt[(static_cast<long long>(b) * p.H + h0) * p.nb + qb];
     craw[1] = (h1 >= 0) ? p.cnt[(static_cast<long long>(b) * p.H + h1) * p.nb + qb] : 0;
     int c[2];
-    for (int t = 0; t < 2; ++t) c[t] = min(max(craw[t], 0), qb + 1);
+    for (int t = 0; t < 2; ++t) c[t] = min(max(craw[t], 0), row_len);
     const int ntiles = (h1 >= 0) ? 2 : 1;
-    const int words = (qb + 32) >> 5;  // bitmap words covering blocks 0..qb
+    const int words = (row_len + 31) >> 5;  // bitmap words covering the row's blocks
 
     // The selected blocks of each head as a bitmap over 0..qb: head t takes the
     // first c[t] entries of its list.  Every role then visits them in
@@ -205,7 +207,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int x = threadIdx.x; x < c[0] + c[1]; x += blockDim.x) {
         const int t = (x < c[0]) ? 0 : 1;
         const int kb = t ? list1[x - c[0]] : list0[x];
-        if (kb < 0 || kb > qb) {
+        if (kb < 0 || kb >= row_len) {
             flag_status(kStBounds);
             continue;
         }
@@ -382,7 +384,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t o_addr = lane_base + 256 + t * 128;
         float m = -INFINITY, l = 0.0f;
         float mtrue = -INFINITY;  // SKIP: exact running max (log2 units) of the tiles visited
-        const long long skip_base = (static_cast<long long>(b) * p.H + h) * T + static_cast<long long>(qb) * (qb + 1) / 2;
+        const long long skip_base = (static_cast<long long>(b) * p.H + h) * T + row_off;
         bool ok = true;
         uint32_t s[128];
         int i = 0;    // tiles of this head so far
@@ -390,7 +392,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int kb = next_block(bmt, bmt, 0, words); kb >= 0; kb = next_block(bmt, bmt, kb + 1, words), ++i) {
             if (!warp_wait(&s_full[t], i & 1, wc)) { ok = false; break; }
             tc_fence_after();
-            const bool masked = (kb == qb);  // the diagonal tile: same for the whole CTA
+            const bool masked = p.causal && kb == qb;  // the causal diagonal tile: same for the whole CTA
             tmem_ld128(s_addr, s);
             if (masked) {
 #pragma unroll

@@ -75,28 +75,33 @@ __device__ __forceinline__ uint32_t score_desc_key(float f) {
     return ~ord;  // larger score -> smaller key
 }
 
-// One CTA per (b, g, qb); dynamic smem holds P = pow2 >= qb-1 keys.
+// One CTA per (b, g, qb); dynamic smem holds P = pow2 >= n keys.  Causal
+// rows hold blocks 0..qb at qb(qb+1)/2; non-causal rows all nb blocks at
+// qb*nb.  The sorted blocks are the row's blocks other than 0 and qb: the
+// i-th of them is i+1, or i+2 once i+1 reaches qb.
 __global__ void __launch_bounds__(256) rank_kernel(const float *__restrict__ scores, int32_t *__restrict__ rank,
-                                                   int nb) {
+                                                   int nb, int causal) {
     extern __shared__ unsigned long long keys[];
     const long long bg = blockIdx.x / nb;
     const int qb = nb - 1 - static_cast<int>(blockIdx.x % nb);  // long rows first
-    const long long T = static_cast<long long>(nb) * (nb + 1) / 2;
-    const long long row0 = bg * T + static_cast<long long>(qb) * (qb + 1) / 2;
+    const long long T = causal ? static_cast<long long>(nb) * (nb + 1) / 2 : static_cast<long long>(nb) * nb;
+    const long long row0 = bg * T + (causal ? static_cast<long long>(qb) * (qb + 1) / 2 : static_cast<long long>(qb) * nb);
     const float *srow = scores + row0;
     int32_t *out = rank + row0;
-    const int n = qb >= 2 ? qb - 1 : 0;
+    const int lead = qb > 0 ? 2 : 1;
+    const int n = (causal ? qb + 1 : nb) - lead;
     int P = 1;
     while (P < n) P <<= 1;
     for (int i = threadIdx.x; i < P; i += blockDim.x) {
         unsigned long long key = ~0ull;
         if (i < n) {
-            float s = srow[i + 1];
+            const int kb = i + 1 + ((qb > 0 && i + 1 >= qb) ? 1 : 0);
+            float s = srow[kb];
             if (!isfinite(s)) {
                 flag_status(kStNonFinite);
                 s = -INFINITY;
             }
-            key = (static_cast<unsigned long long>(score_desc_key(s)) << 32) | static_cast<uint32_t>(i + 1);
+            key = (static_cast<unsigned long long>(score_desc_key(s)) << 32) | static_cast<uint32_t>(kb);
         }
         keys[i] = key;
     }
@@ -121,13 +126,14 @@ __global__ void __launch_bounds__(256) rank_kernel(const float *__restrict__ sco
         out[0] = 0;
         if (qb > 0) out[1] = qb;
     }
-    for (int i = threadIdx.x; i < n; i += blockDim.x) out[2 + i] = static_cast<int32_t>(keys[i] & 0xFFFFFFFFu);
+    for (int i = threadIdx.x; i < n; i += blockDim.x) out[lead + i] = static_cast<int32_t>(keys[i] & 0xFFFFFFFFu);
 }
 
 // ----------------------------------------------------------------- budget
 struct BudgetParams {
     int B, H, G, nb;
     int mode;            // 0 dynamic, 1 fixed fraction, 2 all
+    int causal;          // 0: every row holds all nb blocks
     float gamma;
     int frac_permille;
     const int32_t *rank;
@@ -148,9 +154,9 @@ __global__ void __launch_bounds__(1024) budget_kernel(BudgetParams p) {
     int k = nb;
     if (p.mode == 0) {
         const int g = static_cast<int>(static_cast<long long>(h) * p.G / p.H);
-        const long long T = static_cast<long long>(nb) * (nb + 1) / 2;
+        const long long T = p.causal ? static_cast<long long>(nb) * (nb + 1) / 2 : static_cast<long long>(nb) * nb;
         const int32_t *last = p.rank + (static_cast<long long>(b) * p.G + g) * T +
-                              static_cast<long long>(nb - 1) * nb / 2;
+                              (p.causal ? static_cast<long long>(nb - 1) * nb / 2 : static_cast<long long>(nb - 1) * nb);
         const float *m = p.mass + static_cast<long long>(bh) * nb;
         const long long gfx = __double2ll_rn(static_cast<double>(p.gamma) * 1099511627776.0);
         const int F = forced_blocks(nb - 1);
@@ -212,14 +218,17 @@ __global__ void __launch_bounds__(1024) budget_kernel(BudgetParams p) {
     }
     int32_t *c = p.cnt + static_cast<long long>(bh) * nb;
     for (int qb = threadIdx.x; qb < nb; qb += blockDim.x) {
+        // a causal row holds qb+1 blocks and takes its share of the last row's
+        // budget; a non-causal row holds nb blocks and takes the budget itself
+        const long long len = p.causal ? qb + 1 : nb;
         long long want;
         if (p.mode == 0)
-            want = (static_cast<long long>(k) * (qb + 1) + nb - 1) / nb;
+            want = p.causal ? (static_cast<long long>(k) * (qb + 1) + nb - 1) / nb : k;
         else if (p.mode == 1)
-            want = (static_cast<long long>(p.frac_permille) * (qb + 1) + 999) / 1000;
+            want = (static_cast<long long>(p.frac_permille) * len + 999) / 1000;
         else
-            want = qb + 1;
-        const long long lo = forced_blocks(qb), hi = qb + 1;
+            want = len;
+        const long long lo = forced_blocks(qb), hi = len;
         const int val = static_cast<int>(want < lo ? lo : (want > hi ? hi : want));
         c[qb] = val;
         if (qb == nb - 1) p.budget[bh] = val;

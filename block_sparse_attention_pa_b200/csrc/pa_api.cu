@@ -77,7 +77,17 @@ pa_status check_shape(const pa_shape *s) {
     if (s->num_q_heads % s->num_groups)
         return fail(PA_ERR_UNSUPPORTED, "num_q_heads %d not a multiple of num_groups %d", s->num_q_heads,
                     s->num_groups);
+    if (s->non_causal != 0 && s->non_causal != 1)
+        return fail(PA_ERR_INVALID_ARG, "non_causal must be 0 or 1 (got %d)", s->non_causal);
     return PA_OK;
+}
+
+bool causal_of(const pa_shape *s) { return s->non_causal == 0; }
+
+// Entries of one (b, g) set of block scores or ranked lists.
+size_t rows_total(const pa_shape *s) {
+    const size_t nb = s->seqlen / kBlk;
+    return causal_of(s) ? nb * (nb + 1) / 2 : nb * nb;
 }
 
 // Query-row stride of the block scores: 1, 2, 4 or 8.
@@ -213,7 +223,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 WsLayout ws_layout(const pa_shape *s, const pa_budget *bu) {
     const size_t B = s->batch, G = s->num_groups, N = s->seqlen, d = s->head_dim, H = s->num_q_heads;
-    const size_t nb = N / kBlk, T = nb * (nb + 1) / 2;
+    const size_t nb = N / kBlk, T = rows_total(s);
     WsLayout w;
     w.partial = 0;
     const size_t part = (bu && bu->mode == PA_BUDGET_DYNAMIC) ? align256(B * H * nb * 128 * sizeof(float2)) : 0;
@@ -292,11 +302,16 @@ pa_status launch_scores(const pa_shape *s, int stride, const void *qp, const voi
     p.B = B; p.nb = nb; p.NH = G; p.H = s->num_q_heads; p.Hkv = s->num_kv_heads;
     p.chunk = kScoreChunk;
     p.stride = stride;
-    // A tile m (query blocks m*r .. m*r+r-1) owns ceil((m+1) / (chunk/r)) units
+    p.causal = causal_of(s) ? 1 : 0;
+    // causal: A tile m (query blocks m*r .. m*r+r-1) owns ceil((m+1) / (chunk/r))
+    // units; non-causal: every A tile owns ceil(nb / chunk)
     const int cr = kScoreChunk / stride;
     const int a_tiles = (nb + stride - 1) / stride;
     long long per = 0;
-    for (int m = 0; m < a_tiles; ++m) per += (m + cr) / cr;
+    if (p.causal)
+        for (int m = 0; m < a_tiles; ++m) per += (m + cr) / cr;
+    else
+        per = static_cast<long long>(a_tiles) * ((nb + kScoreChunk - 1) / kScoreChunk);
     p.units_per_bh = per;
     p.num_units = per * B * G;
     p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
@@ -319,6 +334,7 @@ pa_status launch_mass(const pa_shape *s, const void *q, pa_strides qs, const voi
     p.B = B; p.nb = nb; p.NH = H; p.H = H; p.Hkv = Hkv;
     p.chunk = kScoreChunk;
     p.stride = 1;
+    p.causal = causal_of(s) ? 1 : 0;
     p.units_per_bh = (nb + kScoreChunk - 1) / kScoreChunk;
     p.num_units = p.units_per_bh * B * H;
     p.scale = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
@@ -340,7 +356,7 @@ pa_status launch_rank(const pa_shape *s, const float *scores, int32_t *rank, cud
     const int smem = P * 8;
     PA_CUDA(cudaFuncSetAttribute(pa::rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, std::max(smem, 1)));
     const long long grid = static_cast<long long>(s->batch) * s->num_groups * nb;
-    pa::rank_kernel<<<static_cast<unsigned>(grid), 256, smem, st>>>(scores, rank, nb);
+    pa::rank_kernel<<<static_cast<unsigned>(grid), 256, smem, st>>>(scores, rank, nb, causal_of(s) ? 1 : 0);
     PA_CUDA(cudaGetLastError());
     return PA_OK;
 }
@@ -350,6 +366,7 @@ pa_status launch_budget(const pa_shape *s, const pa_budget *bu, const int32_t *r
     pa::BudgetParams p;
     p.B = s->batch; p.H = s->num_q_heads; p.G = s->num_groups; p.nb = s->seqlen / kBlk;
     p.mode = bu->mode; p.gamma = bu->gamma; p.frac_permille = bu->frac_permille;
+    p.causal = causal_of(s) ? 1 : 0;
     p.rank = rank; p.mass = mass; p.cnt = cnt; p.budget = budget;
     pa::budget_kernel<<<s->batch * s->num_q_heads, 1024, 0, st>>>(p);
     PA_CUDA(cudaGetLastError());
@@ -482,6 +499,7 @@ pa_status launch_attn(const pa_shape *s, const void *q, pa_strides qs, const voi
     p.o = static_cast<__nv_bfloat16 *>(o);
     p.osb = os.b; p.oss = os.s; p.osh = os.h;
     p.lse = lse;
+    p.causal = causal_of(s) ? 1 : 0;
     p.timeout_ns = wait_timeout_ns();
     const bool skip = skip_threshold > 0.0f;
     p.skip_log2 = skip ? static_cast<float>(std::log2(static_cast<double>(skip_threshold))) : -INFINITY;
@@ -682,6 +700,7 @@ pa_status pa_xattn_mask(const pa_shape *shape, int32_t stride, float tau, const 
                         size_t ws_bytes, pa_stream_t stream) {
     pa_status r;
     if ((r = check_shape(shape)) || (r = check_xstride(stride))) return r;
+    if (!causal_of(shape)) return fail(PA_ERR_UNSUPPORTED, "the XAttention estimator is causal only");
     if (!(tau > 0.0f && tau <= 1.0f))
         return fail(PA_ERR_INVALID_ARG, "tau must be in (0, 1] (got %g)", static_cast<double>(tau));
     if ((r = check_tensor(q, qs, "q")) || (r = check_tensor(k, ks, "k"))) return r;

@@ -37,6 +37,7 @@ struct TileParams {
     int H, Hkv;            // mass: q head -> KV head
     int chunk;             // tiles per unit (a multiple of stride)
     int stride;            // scores: query-row stride r in {1,2,4,8}; mass: 1
+    int causal;            // 1: keys j <= i only (triangular rows); 0: every key (square rows)
     long long units_per_bh;
     long long num_units;
     float scale;           // scores: 1/sqrt(d); mass: scale*log2(e)
@@ -60,7 +61,13 @@ __device__ __forceinline__ Unit decode_unit(const TileParams &p, long long u, in
     r.b = static_cast<int>(bh / p.NH);
     r.bh_head = static_cast<int>(bh % p.NH);
     const int C = p.chunk;
-    if (mode == MODE_SCORES) {
+    if (mode == MODE_SCORES && !p.causal) {
+        // non-causal: every A tile owns ceil(nb / C) units over all key tiles
+        const long long upr = (p.nb + C - 1) / C;
+        r.qb = static_cast<int>(w / upr);
+        r.kb0 = static_cast<int>(w % upr) * C;
+        r.kb1 = min(r.kb0 + C, p.nb);
+    } else if (mode == MODE_SCORES) {
         const int Cr = C / p.stride;
         long long a = static_cast<long long>((sqrt(1.0 + 8.0 * static_cast<double>(w) / Cr) - 1.0) * 0.5);
         while (a > 0 && static_cast<long long>(Cr) * a * (a + 1) / 2 > w) --a;
@@ -267,7 +274,7 @@ __global__ void __launch_bounds__(192, 1)
                 float lsum[2];
                 for (int j = 0; j < nt; ++j, ++tile) {
                     const int kb = kb0 + j;
-                    const bool diag = (kb == qbw);
+                    const bool diag = p.causal && (kb == qbw);
                     uint32_t r[128];
                     tmem_ld128(lane_base + acc * 256 + j * 128, r);
                     if (j == nt - 1) {
@@ -311,11 +318,13 @@ __global__ void __launch_bounds__(192, 1)
                             if (o < span) w = fmaxf(w, __shfl_xor_sync(0xffffffffu, w, o));
                         // tiles above this query block's diagonal, and A rows past the last
                         // block (zero-filled), give no score
-                        const bool valid = kb <= qbw && qbw < p.nb;
+                        const bool valid = (!p.causal || kb <= qbw) && qbw < p.nb;
                         if (valid && (static_cast<int>(lane) & (span - 1)) == 0) {
-                            const long long T = static_cast<long long>(p.nb) * (p.nb + 1) / 2;
+                            const long long T = p.causal ? static_cast<long long>(p.nb) * (p.nb + 1) / 2
+                                                         : static_cast<long long>(p.nb) * p.nb;
                             const long long idx = (static_cast<long long>(un.b) * p.NH + un.bh_head) * T +
-                                                  static_cast<long long>(qbw) * (qbw + 1) / 2 + kb;
+                                                  (p.causal ? static_cast<long long>(qbw) * (qbw + 1) / 2
+                                                            : static_cast<long long>(qbw) * p.nb) + kb;
                             if (wpq <= 1) {
                                 p.scores[idx] = w;
                             } else {

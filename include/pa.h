@@ -21,7 +21,9 @@
  *   the scored rows, [B][G][N/r][d].
  *   Block scores and ranked lists are [B][G][T] with nb = N/128,
  *   T = nb(nb+1)/2 and query block qb's row starting at tri(qb) = qb(qb+1)/2
- *   (entries tri(qb)+0 .. tri(qb)+qb).
+ *   (entries tri(qb)+0 .. tri(qb)+qb).  With shape->non_causal = 1 every row
+ *   holds all nb blocks: T = nb*nb, row qb at qb*nb ("tri(qb)" below then
+ *   reads qb*nb, "j <= i" holds for every key and "qb+1" blocks read nb).
  * Heads.  kv(h) = floor(h*Hkv/H) (GQA), grp(h) = floor(h*G/H) (proxy group).
  * Memory.  Every pointer is a device pointer owned by the caller unless a
  *   comment says otherwise.  The library allocates no device memory; calls
@@ -46,7 +48,7 @@
 extern "C" {
 #endif
 
-#define PA_ABI_VERSION 2
+#define PA_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define PA_API __attribute__((visibility("default")))
@@ -75,6 +77,12 @@ typedef struct pa_shape {
     int32_t head_dim;     /* d: 64 or 128 */
     int32_t block;        /* must be 128 */
     int32_t num_groups;   /* G proxy groups, divides H */
+    int32_t non_causal;   /* 0: causal prefill (query i attends keys j <= i);
+                             1: every query attends every key (bidirectional,
+                             e.g. diffusion transformers; XAttention blog,
+                             video generation).  Non-causal block scores and
+                             ranked lists hold all nb blocks per query block:
+                             [B][G][nb*nb], row qb at qb*nb. */
 } pa_shape;
 
 typedef struct pa_strides {
@@ -176,8 +184,10 @@ PA_API pa_status pa_block_scores_strided(const pa_shape *shape, int32_t score_st
  *  - budget: DYNAMIC: with m_fx = rint(mass * 2^40), g_fx = rint(gamma * 2^40),
  *    k_h = smallest k >= |F| (|F| = 2, or 1 when nb = 1) such that the first k
  *    entries of the last row's list carry sum m_fx >= g_fx, else nb;
- *    cnt[b][h][qb] = clamp(ceil(k_h (qb+1) / nb), |F_qb|, qb+1).
- *    FIXED_FRACTION: cnt = clamp(ceil(p (qb+1) / 1000), |F_qb|, qb+1).
+ *    cnt[b][h][qb] = clamp(ceil(k_h (qb+1) / nb), |F_qb|, qb+1)
+ *    (non-causal: every row has nb blocks, cnt = clamp(k_h, |F_qb|, nb)).
+ *    FIXED_FRACTION: cnt = clamp(ceil(p (qb+1) / 1000), |F_qb|, qb+1)
+ *    (non-causal: ceil(p nb / 1000)).
  *    ALL: cnt = qb+1.  budget = cnt at qb = nb-1.
  * q and k are only read in DYNAMIC mode (may be NULL otherwise).  ws: device
  * workspace of ws_bytes >= pa_workspace_size(shape, budget). */
@@ -274,7 +284,8 @@ PA_API pa_status pa_block_sparse_attn_skip(const pa_shape *shape,
  * No block is forced into the set.  bf16 tensor-core products with fp32
  * accumulation; mass (nullable) fp32.  ws: device workspace of
  * ws_bytes >= pa_xattn_workspace_size(shape, S); tau in (0, 1].  The shape's
- * num_groups is not used. */
+ * num_groups is not used; the shape must be causal (PA_ERR_UNSUPPORTED
+ * otherwise). */
 PA_API size_t pa_xattn_workspace_size(const pa_shape *shape, int32_t stride);
 
 PA_API pa_status pa_xattn_mask(const pa_shape *shape, int32_t stride, float tau,

@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_version_and_status_strings(L):
-    assert L.pa_abi_version() == 2
+    assert L.pa_abi_version() == 3
     for code in range(8):
         assert L.pa_status_string(code).decode() not in ("", "unknown status")
     assert L.pa_status_string(99).decode() == "unknown status"
@@ -152,6 +152,22 @@ def test_xattn_workspace_and_argument_errors(L):
                                None) == 1
     assert L.pa_xattn_mask(ctypes.byref(s), 8, ctypes.c_float(0.9), 16, st, 16, st, 16, 16, None, 256, 16,
                            None) == 3
+
+
+def test_noncausal_shape_sizes_and_errors(L):
+    s = shape(N=1024, H=8, Hkv=2, d=64, G=2)
+    s.non_causal = 1
+    nb = 8
+    a256 = lambda x: (x + 255) // 256 * 256
+    fixed = pa.workspace_size(s, pa.make_budget(pa.FIXED_FRACTION, 0, 100))
+    assert fixed == 2 * a256(2 * 1024 * 64 * 2) + a256(2 * nb * nb * 4)
+    s.non_causal = 2
+    assert pa.workspace_size(s, pa.make_budget(pa.FIXED_FRACTION, 0, 100)) == 0
+    st = pa.Strides(0, 512, 64)
+    assert L.pa_pool_heads(ctypes.byref(s), 16, st, 16, st, 16, 16, None) == 1
+    s.non_causal = 1
+    assert L.pa_xattn_mask(ctypes.byref(s), 8, ctypes.c_float(0.9), 16, st, 16, st, 16, 16, None, 256, 1 << 30,
+                           None) == 2
 
 
 def test_attention_argument_errors(L):
