@@ -62,6 +62,8 @@ def parse_args():
     ap.add_argument("--frac", type=int, default=100, help="fixed budget in per mille of causal blocks")
     ap.add_argument("--score-stride", type=int, default=1, choices=[1, 2, 4, 8],
                     help="query-row stride of the proxy block scores (1: every row)")
+    ap.add_argument("--non-causal", action="store_true",
+                    help="every query attends every key (bidirectional attention)")
     ap.add_argument("--estimator", choices=["proxy", "xattn"], default="proxy",
                     help="mask estimator: ProxyAttn (pooled proxy scores + per-head budget) or XAttention "
                          "(antidiagonal strided scores + find_blocks, one list per head)")
@@ -151,7 +153,7 @@ class Pipeline:
     """Pre-allocated buffers and ctypes arguments for one layer, so that a step is
     four C-ABI calls with CUDA events between them."""
 
-    def __init__(self, q, k, v, G, mode, gamma, frac, stride=1, skip=0.0, proxies=True):
+    def __init__(self, q, k, v, G, mode, gamma, frac, stride=1, skip=0.0, proxies=True, causal=True):
         import block_sparse_attention_pa_b200 as pa
         self.pa = pa
         self.L = pa.lib()
@@ -159,7 +161,8 @@ class Pipeline:
         B, N, H, d = q.shape
         self.B, self.N, self.H, self.d, self.G = B, N, H, d, G
         self.nb = N // 128
-        self.shape = pa.make_shape(q, k, G)
+        self.shape = pa.make_shape(q, k, G, causal)
+        self.causal = causal
         self.budget = pa.make_budget(mode, gamma, frac, stride, skip)
         self.mode = mode
         self.stride = stride
@@ -169,7 +172,7 @@ class Pipeline:
         pn = N if proxies else 128  # the XAttention pipeline needs no proxies
         self.qp = torch.empty(B, G, pn // stride, d, device=dev, dtype=torch.bfloat16)
         self.kp = torch.empty(B, G, pn, d, device=dev, dtype=torch.bfloat16)
-        T = self.nb * (self.nb + 1) // 2
+        T = pa.rows_total(self.nb, causal)
         self.T = T
         self.scores = torch.empty(B, G, T, device=dev, dtype=torch.float32)
         self.mask = pa.Mask.empty(self.shape, dev, mode == 0)
@@ -219,6 +222,8 @@ class Pipeline:
         v = int(self.mask.cnt.sum().item())
         ndiag = self.B * self.H * self.nb
         per = 4 * 128 * 128 * self.d
+        if not self.causal:
+            return v, v * per, v * per
         exact = (v - ndiag) * per + ndiag * 4 * self.d * (128 * 129 // 2)
         return v, v * per, exact
 
@@ -475,7 +480,7 @@ def main():
     if xattn:
         pipe = XPipeline(q, k, v, args.xattn_stride, args.tau, skip)
     else:
-        pipe = Pipeline(q, k, v, G, mode, gamma, frac, stride, skip)
+        pipe = Pipeline(q, k, v, G, mode, gamma, frac, stride, skip, causal=not args.non_causal)
     sampler = None if args.no_clocks else ClockSampler(local)
     total_ms, stages, clocks = time_pipeline(pipe, args.steps, args.warmup, dist_on, sampler)
     status = pa.device_status()
@@ -485,7 +490,7 @@ def main():
     ms_step = total_ms / args.steps
     visited, flops, flops_exact = pipe.visited()
     B, H, nb = w.batch, w.num_q_heads, pipe.nb
-    T = nb * (nb + 1) // 2
+    T = pipe.T
     density = visited / (B * H * T)
     est_ms = float(stages[:3].sum())
     attn_ms = float(stages[3])
@@ -541,7 +546,7 @@ def main():
                        config_of(w, H, 1, 0.0, 1000, 1, skip) | {
                            "groups": H, "budget": f"XAttention find_blocks tau={args.tau}",
                            "estimator": f"xattn antidiagonal stride {args.xattn_stride}"})
-                      | {"parallelism": f"replicas x{world}"},
+                      | {"parallelism": f"replicas x{world}", "causal": not args.non_causal},
             "est_ms": est_ms, "sparse_ms": attn_ms,
             "tflops_effective": flops / (attn_ms * 1e-3) / 1e12, "tflops_exact_causal": flops_exact / (attn_ms * 1e-3) / 1e12,
             "visited_blocks": visited, "density": density, "sparsity": 1.0 - density,
@@ -555,7 +560,7 @@ def main():
 
     # dense baseline: the same kernel with every causal block selected
     if not args.no_dense:
-        dense = Pipeline(q, k, v, w.num_groups, 2, gamma, frac, 1)
+        dense = Pipeline(q, k, v, w.num_groups, 2, gamma, frac, 1, causal=not args.non_causal)
         dsteps = max(2, min(5, args.steps))
         _, dstages, _ = time_pipeline(dense, dsteps, 1, dist_on)
         dense_attn = float(dstages[3])
@@ -592,11 +597,11 @@ def main():
 
     # end to end through the public API with pinned host buffers
     if not args.no_e2e and not xattn:
-        e2e = run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world, stride, skip)
+        e2e = run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world, stride, skip, not args.non_causal)
         line["e2e"] = e2e
 
     # the CPU oracle on a bounded sample (rank 0, one GPU only)
-    if not args.no_cpu_baseline and world == 1 and rank == 0 and not xattn:
+    if not args.no_cpu_baseline and world == 1 and rank == 0 and not xattn and not args.non_causal:
         import oracle
         xc = {n: x[n].cpu() for n in ("q", "k", "v")}
         ms, det, sample = oracle_estimate(xc, w, G, mode, gamma, frac, size="baseline", stride=stride, skip=skip)
@@ -610,7 +615,7 @@ def main():
         torch.distributed.destroy_process_group()
 
 
-def run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world, stride=1, skip=0.0):
+def run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world, stride=1, skip=0.0, causal=True):
     """The metric through the public API with host buffers, as a user runs
     consecutive layers: every step copies its q, k, v from pinned host memory
     and reads its o back.  Two device buffer sets and two copy streams let the
@@ -619,7 +624,7 @@ def run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world, stride=1, skip
     q, k, v = x["q"], x["k"], x["v"]
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
     bufs = [tuple(torch.empty_like(t) for t in (q, k, v, q)) for _ in range(2)]
-    call = pa.Prefill(bufs[0][0], bufs[0][1], bufs[0][2], G, mode, gamma, frac, stride, skip)
+    call = pa.Prefill(bufs[0][0], bufs[0][1], bufs[0][2], G, mode, gamma, frac, stride, skip, causal)
     ho = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(2)]
     ms = torch.cuda.current_stream()
     hs, ds = torch.cuda.Stream(), torch.cuda.Stream()
