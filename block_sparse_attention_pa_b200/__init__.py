@@ -32,7 +32,8 @@ STATUS = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED", 3: "PA_E
 ENTRY_POINTS = ("pa_workspace_size", "pa_pool_heads", "pa_block_scores", "pa_build_mask",
                 "pa_block_sparse_attn", "pa_prefill", "pa_get_device_status", "pa_status_string",
                 "pa_last_error", "pa_abi_version", "pa_build_mask_noalloc", "pa_selftest_wait_timeout",
-                "pa_pool_heads_strided", "pa_block_scores_strided", "pa_block_sparse_attn_skip", "pa_xattn_workspace_size", "pa_xattn_mask")
+                "pa_pool_heads_strided", "pa_block_scores_strided", "pa_block_sparse_attn_skip", "pa_xattn_workspace_size", "pa_xattn_mask",
+                "pa_workspace_size_varlen", "pa_prefill_varlen")
 
 XATTN_STRIDES = (4, 8, 16)
 SCORE_STRIDES = (1, 2, 4, 8)
@@ -90,6 +91,10 @@ def lib() -> ctypes.CDLL:
         L.pa_prefill.argtypes = [P(Shape), P(Budget), vp, st, vp, st, vp, st, vp, st, P(MaskBufs), vp,
                                  ctypes.c_size_t, vp]
         L.pa_get_device_status.argtypes = [vp, ctypes.c_int]
+        L.pa_workspace_size_varlen.restype = ctypes.c_size_t
+        L.pa_workspace_size_varlen.argtypes = [P(Shape), P(Budget), ctypes.c_int32, vp]
+        L.pa_prefill_varlen.argtypes = [P(Shape), P(Budget), ctypes.c_int32, vp, vp, st, vp, st, vp, st, vp, st,
+                                        P(MaskBufs), vp, ctypes.c_size_t, vp]
         L.pa_xattn_workspace_size.restype = ctypes.c_size_t
         L.pa_xattn_workspace_size.argtypes = [P(Shape), ctypes.c_int32]
         L.pa_xattn_mask.argtypes = [P(Shape), ctypes.c_int32, ctypes.c_float, vp, st, vp, st, vp, vp, vp, vp,
@@ -101,7 +106,7 @@ def lib() -> ctypes.CDLL:
         L.pa_abi_version.restype = ctypes.c_int32
         for name in ("pa_pool_heads", "pa_block_scores", "pa_build_mask", "pa_block_sparse_attn", "pa_prefill",
                      "pa_get_device_status", "pa_selftest_wait_timeout", "pa_pool_heads_strided",
-                     "pa_block_scores_strided", "pa_block_sparse_attn_skip", "pa_xattn_mask"):
+                     "pa_block_scores_strided", "pa_block_sparse_attn_skip", "pa_xattn_mask", "pa_prefill_varlen"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -322,3 +327,51 @@ def device_status(clear: bool = True, device=None) -> int:
 def selftest_wait_timeout(timeout_us: int = 1000, device=None) -> None:
     """pa_selftest_wait_timeout: a bounded device wait that is made to run out."""
     _check(lib().pa_selftest_wait_timeout(int(timeout_us), _stream(device)))
+
+
+@dataclass
+class VarlenMask:
+    """Packed mask buffers of pa_prefill_varlen and each sequence's views."""
+    rank: torch.Tensor     # int32, sequences' [G, T_s] blocks back to back
+    cnt: torch.Tensor      # int32, sequences' [H, nb_s] blocks back to back
+    budget: torch.Tensor   # int32 [num_seqs, H]
+    mass: torch.Tensor | None
+    views: list            # per sequence: Mask of views into the packed buffers
+
+
+def prefill_varlen(q, k, v, cu_seqlens, num_groups: int, mode: int = DYNAMIC, gamma: float = 0.95,
+                   frac_permille: int = 0, score_stride: int = 1, skip_threshold: float = 0.0, causal: bool = True):
+    """pa_prefill_varlen: q, k, v are [1, total, heads, d]; cu_seqlens a list of
+    num_seqs+1 token offsets -> (o, VarlenMask)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _cuda_bf16(t, n)
+    cu = [int(x) for x in cu_seqlens]
+    nseq = len(cu) - 1
+    shape = make_shape(q, k, num_groups, causal)
+    budget = make_budget(mode, gamma, frac_permille, score_stride, skip_threshold)
+    H, G = shape.num_q_heads, num_groups
+    nbs = [(cu[s + 1] - cu[s]) // 128 for s in range(nseq)]
+    Ts = [rows_total(nb, causal) for nb in nbs]
+    dev = q.device
+    i32 = dict(device=dev, dtype=torch.int32)
+    rank = torch.empty(G * sum(Ts), **i32)
+    cnt = torch.empty(H * sum(nbs), **i32)
+    bud = torch.empty(nseq, H, **i32)
+    mass = torch.empty(H * sum(nbs), device=dev, dtype=torch.float32) if mode == DYNAMIC else None
+    cu_arr = (ctypes.c_int32 * len(cu))(*cu)
+    need = int(lib().pa_workspace_size_varlen(ctypes.byref(shape), ctypes.byref(budget), nseq, cu_arr))
+    ws = torch.empty(max(need, 256), device=dev, dtype=torch.uint8)
+    o = torch.empty_like(q, memory_format=torch.contiguous_format)
+    bufs = MaskBufs(rank.data_ptr(), cnt.data_ptr(), bud.data_ptr(), mass.data_ptr() if mass is not None else None)
+    _check(lib().pa_prefill_varlen(ctypes.byref(shape), ctypes.byref(budget), nseq, cu_arr, q.data_ptr(),
+                                   _strides(q), k.data_ptr(), _strides(k), v.data_ptr(), _strides(v), o.data_ptr(),
+                                   _strides(o), ctypes.byref(bufs), ws.data_ptr(), ws.numel(), _stream(dev)))
+    views, ro, bo = [], 0, 0
+    for s in range(nseq):
+        views.append(Mask(rank[G * ro: G * (ro + Ts[s])].view(1, G, Ts[s]),
+                          cnt[H * bo: H * (bo + nbs[s])].view(1, H, nbs[s]),
+                          bud[s].view(1, H),
+                          mass[H * bo: H * (bo + nbs[s])].view(1, H, nbs[s]) if mass is not None else None))
+        ro += Ts[s]
+        bo += nbs[s]
+    return o, VarlenMask(rank, cnt, bud, mass, views)

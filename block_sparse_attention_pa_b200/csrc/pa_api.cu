@@ -639,20 +639,16 @@ pa_status pa_block_sparse_attn(const pa_shape *shape, const void *q, pa_strides 
     return ok();
 }
 
-pa_status pa_prefill(const pa_shape *shape, const pa_budget *budget, const void *q, pa_strides qs, const void *k,
-                     pa_strides ks, const void *v, pa_strides vs, void *o, pa_strides os, const pa_mask *mask_out,
-                     void *ws, size_t ws_bytes, pa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The launches of pa_prefill for one already-validated problem.
+pa_status run_prefill(const pa_shape *shape, const pa_budget *budget, const void *q, pa_strides qs, const void *k,
+                      pa_strides ks, const void *v, pa_strides vs, void *o, pa_strides os, const pa_mask *mask_out,
+                      void *ws, cudaStream_t st) {
     pa_status r;
-    if ((r = check_shape(shape)) || (r = check_budget(budget))) return r;
-    if ((r = check_tensor(q, qs, "q")) || (r = check_tensor(k, ks, "k")) || (r = check_tensor(v, vs, "v")) ||
-        (r = check_tensor(o, os, "o")))
-        return r;
-    if ((r = check_mask(mask_out, budget, true))) return r;
     const WsLayout w = ws_layout(shape, budget);
-    if (!ws || ws_bytes < w.total)
-        return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, w.total);
-    if ((r = check_ptr(ws, "workspace", 256))) return r;
-    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *base = static_cast<uint8_t *>(ws);
     void *qp = base + w.qp;
     void *kp = base + w.kp;
@@ -670,6 +666,106 @@ pa_status pa_prefill(const pa_shape *shape, const pa_budget *budget, const void 
     if ((r = launch_attn(shape, q, qs, k, ks, v, vs, mask_out->rank, mask_out->cnt, scale, o, os, nullptr,
                          budget->skip_threshold, nullptr, st)))
         return r;
+    return PA_OK;
+}
+
+// Validates a packed variable-length batch; fills the longest sequence.
+pa_status check_varlen(const pa_shape *shape, int32_t num_seqs, const int32_t *cu, int32_t *max_len) {
+    pa_status r;
+    if ((r = check_shape(shape))) return r;
+    if (shape->batch != 1) return fail(PA_ERR_INVALID_ARG, "a packed batch needs shape->batch = 1 (got %d)", shape->batch);
+    if (num_seqs < 1) return fail(PA_ERR_INVALID_ARG, "num_seqs must be >= 1 (got %d)", num_seqs);
+    if (!cu) return fail(PA_ERR_INVALID_ARG, "cu_seqlens is NULL");
+    if (cu[0] != 0) return fail(PA_ERR_INVALID_ARG, "cu_seqlens[0] must be 0 (got %d)", cu[0]);
+    int32_t mx = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+        const int64_t len = static_cast<int64_t>(cu[s + 1]) - cu[s];
+        if (len <= 0 || len % kBlk)
+            return fail(PA_ERR_UNSUPPORTED, "sequence %d has %lld tokens: lengths must be positive multiples of 128", s,
+                        static_cast<long long>(len));
+        if (len / kBlk > kMaxNb)
+            return fail(PA_ERR_UNSUPPORTED, "sequence %d has %lld tokens, more than %d", s, static_cast<long long>(len),
+                        kMaxNb * kBlk);
+        mx = std::max<int32_t>(mx, static_cast<int32_t>(len));
+    }
+    if (cu[num_seqs] != shape->seqlen)
+        return fail(PA_ERR_INVALID_ARG, "cu_seqlens[num_seqs] = %d differs from shape->seqlen = %d", cu[num_seqs],
+                    shape->seqlen);
+    *max_len = mx;
+    return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_prefill(const pa_shape *shape, const pa_budget *budget, const void *q, pa_strides qs, const void *k,
+                     pa_strides ks, const void *v, pa_strides vs, void *o, pa_strides os, const pa_mask *mask_out,
+                     void *ws, size_t ws_bytes, pa_stream_t stream) {
+    pa_status r;
+    if ((r = check_shape(shape)) || (r = check_budget(budget))) return r;
+    if ((r = check_tensor(q, qs, "q")) || (r = check_tensor(k, ks, "k")) || (r = check_tensor(v, vs, "v")) ||
+        (r = check_tensor(o, os, "o")))
+        return r;
+    if ((r = check_mask(mask_out, budget, true))) return r;
+    const WsLayout w = ws_layout(shape, budget);
+    if (!ws || ws_bytes < w.total)
+        return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, w.total);
+    if ((r = check_ptr(ws, "workspace", 256))) return r;
+    if ((r = run_prefill(shape, budget, q, qs, k, ks, v, vs, o, os, mask_out, ws,
+                         reinterpret_cast<cudaStream_t>(stream))))
+        return r;
+    return ok();
+}
+
+size_t pa_workspace_size_varlen(const pa_shape *shape, const pa_budget *budget, int32_t num_seqs,
+                                const int32_t *cu_seqlens) {
+    int32_t mx = 0;
+    if (check_varlen(shape, num_seqs, cu_seqlens, &mx) || check_budget(budget)) return 0;
+    pa_shape one = *shape;
+    one.seqlen = mx;
+    return ws_layout(&one, budget).total;
+}
+
+pa_status pa_prefill_varlen(const pa_shape *shape, const pa_budget *budget, int32_t num_seqs,
+                            const int32_t *cu_seqlens, const void *q, pa_strides qs, const void *k, pa_strides ks,
+                            const void *v, pa_strides vs, void *o, pa_strides os, const pa_mask *mask_out, void *ws,
+                            size_t ws_bytes, pa_stream_t stream) {
+    pa_status r;
+    int32_t mx = 0;
+    if ((r = check_varlen(shape, num_seqs, cu_seqlens, &mx)) || (r = check_budget(budget))) return r;
+    if ((r = check_tensor(q, qs, "q")) || (r = check_tensor(k, ks, "k")) || (r = check_tensor(v, vs, "v")) ||
+        (r = check_tensor(o, os, "o")))
+        return r;
+    if ((r = check_mask(mask_out, budget, true))) return r;
+    pa_shape longest = *shape;
+    longest.seqlen = mx;
+    const size_t need = ws_layout(&longest, budget).total;
+    if (!ws || ws_bytes < need)
+        return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, need);
+    if ((r = check_ptr(ws, "workspace", 256))) return r;
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int G = shape->num_groups, H = shape->num_q_heads;
+    int64_t rows_off = 0, blk_off = 0;  // sums of T_s and nb_s over the sequences before
+    for (int s = 0; s < num_seqs; ++s) {
+        pa_shape one = *shape;
+        one.seqlen = cu_seqlens[s + 1] - cu_seqlens[s];
+        const int64_t nb = one.seqlen / kBlk;
+        const int64_t T = static_cast<int64_t>(rows_total(&one));
+        const int64_t t0 = cu_seqlens[s];
+        pa_mask m;
+        m.rank = mask_out->rank + G * rows_off;
+        m.cnt = mask_out->cnt + H * blk_off;
+        m.budget = mask_out->budget + static_cast<int64_t>(H) * s;
+        m.mass = mask_out->mass ? mask_out->mass + H * blk_off : nullptr;
+        const auto *qb = static_cast<const __nv_bfloat16 *>(q) + t0 * qs.s;
+        const auto *kb = static_cast<const __nv_bfloat16 *>(k) + t0 * ks.s;
+        const auto *vb = static_cast<const __nv_bfloat16 *>(v) + t0 * vs.s;
+        auto *ob = static_cast<__nv_bfloat16 *>(o) + t0 * os.s;
+        if ((r = run_prefill(&one, budget, qb, qs, kb, ks, vb, vs, ob, os, &m, ws, st))) return r;
+        rows_off += T;
+        blk_off += nb;
+    }
     return ok();
 }
 

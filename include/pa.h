@@ -308,6 +308,36 @@ PA_API pa_status pa_prefill(const pa_shape *shape, const pa_budget *budget,
                      const pa_mask *mask_out, void *ws, size_t ws_bytes,
                      pa_stream_t stream);
 
+/* Variable-length batch (the pages' workloads are one sequence per layer
+ * call; this is the packed form serving frameworks use): num_seqs sequences
+ * packed along the token axis of q, k, v, o ([1][total][heads][d] with the
+ * usual strides).  cu_seqlens is a HOST array of num_seqs+1 token offsets:
+ * cu_seqlens[0] = 0, every length cu_seqlens[s+1] - cu_seqlens[s] a positive
+ * multiple of 128 (at most 4096 blocks), cu_seqlens[num_seqs] =
+ * shape->seqlen; shape->batch must be 1.  Sequence s is exactly the
+ * single-sequence problem of pa_prefill on its tokens (no attention across
+ * sequences), run in order on `stream`, all sequences reusing one workspace of
+ * pa_workspace_size_varlen bytes (the longest sequence's).  The mask buffers
+ * are packed by sequence, with nb_s = len_s/128 and T_s the entries of one
+ * (b, g) row set (nb_s(nb_s+1)/2, or nb_s^2 non-causal):
+ *   rank   sequence s at element offset G * sum_{s'<s} T_s', laid out [G][T_s]
+ *   cnt    at H * sum_{s'<s} nb_s', [H][nb_s];  mass likewise (DYNAMIC)
+ *   budget at H * s, [H]
+ * Errors as pa_prefill; a malformed cu_seqlens is PA_ERR_INVALID_ARG (or
+ * PA_ERR_UNSUPPORTED for a length outside the supported set).  0 from
+ * pa_workspace_size_varlen means invalid arguments. */
+PA_API size_t pa_workspace_size_varlen(const pa_shape *shape, const pa_budget *budget,
+                                       int32_t num_seqs, const int32_t *cu_seqlens);
+
+PA_API pa_status pa_prefill_varlen(const pa_shape *shape, const pa_budget *budget,
+                                   int32_t num_seqs, const int32_t *cu_seqlens,
+                                   const void *q, pa_strides q_strides,
+                                   const void *k, pa_strides k_strides,
+                                   const void *v, pa_strides v_strides,
+                                   void *o, pa_strides o_strides,
+                                   const pa_mask *mask_out, void *ws, size_t ws_bytes,
+                                   pa_stream_t stream);
+
 /* Synchronises `stream`, then returns the device status word of the current
  * device (PA_OK, PA_ERR_TIMEOUT, PA_ERR_DEVICE_BOUNDS or PA_ERR_DEVICE_NONFINITE:
  * the first problem any

@@ -170,6 +170,27 @@ def test_noncausal_shape_sizes_and_errors(L):
                            None) == 2
 
 
+def test_varlen_validation_and_workspace(L):
+    s = shape(N=2560, H=8, Hkv=2, d=64, G=2)
+    b = pa.make_budget(pa.DYNAMIC, 0.9)
+    cu = (ctypes.c_int32 * 5)(0, 384, 1408, 1536, 2560)
+    longest = shape(N=1024, H=8, Hkv=2, d=64, G=2)
+    assert L.pa_workspace_size_varlen(ctypes.byref(s), ctypes.byref(b), 4, cu) == pa.workspace_size(longest, b)
+    st = pa.Strides(0, 512, 64)
+    m = pa.MaskBufs(16, 16, 16, 16)
+    for bad, code in (((0, 384, 1400, 1536, 2560), 2), ((128, 384, 1408, 1536, 2560), 1),
+                      ((0, 384, 1408, 1536, 2432), 1), ((0, 384, 384, 1536, 2560), 2)):
+        c = (ctypes.c_int32 * 5)(*bad)
+        assert L.pa_workspace_size_varlen(ctypes.byref(s), ctypes.byref(b), 4, c) == 0
+        assert L.pa_prefill_varlen(ctypes.byref(s), ctypes.byref(b), 4, c, 16, st, 16, st, 16, st, 16, st,
+                                   ctypes.byref(m), 256, 1 << 30, None) == code
+    s2 = shape(B=2, N=2560, H=8, Hkv=2, d=64, G=2)
+    assert L.pa_prefill_varlen(ctypes.byref(s2), ctypes.byref(b), 4, cu, 16, st, 16, st, 16, st, 16, st,
+                               ctypes.byref(m), 256, 1 << 30, None) == 1
+    assert L.pa_prefill_varlen(ctypes.byref(s), ctypes.byref(b), 4, None, 16, st, 16, st, 16, st, 16, st,
+                               ctypes.byref(m), 256, 1 << 30, None) == 1
+
+
 def test_attention_argument_errors(L):
     s = shape()
     st = pa.Strides(0, 512, 64)
