@@ -417,6 +417,18 @@ def oracle_estimate(x, w: synth.Workload, G, mode, gamma, frac, size="baseline",
     return sum(det.values()) * 1e3, det, sample
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (for the oracle baseline's record)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def run_reference(args, w, G, mode, gamma, frac):
     """The reference arm: the CPU oracle, timed on the host cores."""
     if int(os.environ.get("RANK", "0")) != 0:
@@ -435,7 +447,8 @@ def run_reference(args, w, G, mode, gamma, frac):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": v, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(w, G, mode, gamma, frac, args.score_stride, args.skip_threshold),
-            "cpu_baseline": {"value": v, "unit": "ms/layer", "cores": cores, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": v, "unit": "ms/layer", "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
+                             "sample": sample},
             "e2e": {"value": v, "unit": "ms/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -516,12 +529,21 @@ def main():
     # strided scores read and pool only the scored q rows (1/stride of them)
     pool_bytes = B * w.seqlen * d * 2 * ((H + G) / stride + Hkv + G)
     score_flops = B * G * T * 2 * 128 * 128 * d / stride
+    mask_bytes = B * G * T * 4 * 2 + B * H * nb * 4 * 2 + B * H * 4
+    if mode == 0:
+        mask_bytes += B * 128 * H * d * 2 + B * w.seqlen * Hkv * d * 2 + B * H * nb * 128 * 8 * 2 + B * H * nb * 4
     stage_roofline = {
         "pool": {"ms": float(stages[0]), "GB/s": pool_bytes / (stages[0] * 1e-3) / 1e9,
                  "frac_hbm": pool_bytes / (stages[0] * 1e-3) / 1e9 / peaks["hbm_gbs"]},
         "scores": {"ms": float(stages[1]), "TFLOP/s": score_flops / (stages[1] * 1e-3) / 1e12,
                    "frac_tensor": score_flops / (stages[1] * 1e-3) / 1e12 / peak},
-        "mask": {"ms": float(stages[2])},
+        # algorithmic bytes of pa_build_mask: block scores read and ranked lists
+        # written; DYNAMIC also the last query block of q and all of k read by
+        # the head-mass GEMM, its (m, l) partials written and read back, and the
+        # masses; counts and budgets.  Latency-bound (sorts and scans of <= 4096
+        # entries), so this fraction of HBM cannot approach 1.
+        "mask": {"ms": float(stages[2]), "bytes": mask_bytes, "GB/s": mask_bytes / (stages[2] * 1e-3) / 1e9,
+                 "frac_hbm": mask_bytes / (stages[2] * 1e-3) / 1e9 / peaks["hbm_gbs"]},
         "attn": {"ms": attn_ms, "TFLOP/s": achieved, "frac_tensor": achieved / peak},
     }
     if xattn:
@@ -606,7 +628,7 @@ def main():
         xc = {n: x[n].cpu() for n in ("q", "k", "v")}
         ms, det, sample = oracle_estimate(xc, w, G, mode, gamma, frac, size="baseline", stride=stride, skip=skip)
         line["cpu_baseline"] = {"value": ms, "unit": "ms/layer", "cores": oracle.num_threads(), "kind": "oracle",
-                                "sample": sample, "stage_s": det}
+                                "cpu_model": cpu_model(), "sample": sample, "stage_s": det}
 
     if rank == 0:
         print(json.dumps(line), flush=True)
