@@ -653,7 +653,7 @@ def run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world, stride=1, skip
     h2d_done = [torch.cuda.Event() for _ in range(2)]
     comp_done = [torch.cuda.Event() for _ in range(2)]
     d2h_done = [torch.cuda.Event() for _ in range(2)]
-    steps = max(2, min(5, args.steps))
+    steps = max(2, min(20, args.steps))  # a stream of layers: the first upload and the last read-back do not overlap compute
 
     def run(n, start_event=None):
         if start_event is not None:
