@@ -239,7 +239,7 @@ def sparse_attn_skip(q, k, v, rank_lists, cnt, G: int, items, lam: float, skip_i
     return out, lse, skip, gap
 
 
-def xattn_mass(q, k, S: int) -> np.ndarray:
+def xattn_mass(q, k, S: int, causal: bool = True) -> np.ndarray:
     """o8: XAttention antidiagonal block estimates [B, H, T] at stride S."""
     B, N, H, d = q.shape
     Hkv = k.shape[2]
@@ -247,21 +247,22 @@ def xattn_mass(q, k, S: int) -> np.ndarray:
     assert BLK % S == 0
     qa, qs = _bits(q)
     ka, ks = _bits(k)
-    out = np.empty((B, H, nb * (nb + 1) // 2), np.float64)
+    out = np.empty((B, H, rows_total(nb, causal)), np.float64)
     lib().pa_oracle_xattn_mass(_i(B), _i(N), _i(H), _i(Hkv), _i(d), _i(S),
                                _p(qa), _i64(qs[0]), _i64(qs[1]), _i64(qs[2]),
-                               _p(ka), _i64(ks[0]), _i64(ks[1]), _i64(ks[2]), _p(out))
+                               _p(ka), _i64(ks[0]), _i64(ks[1]), _i64(ks[2]), _i(int(causal)), _p(out))
     return out
 
 
-def find_blocks(mass, nb: int, tau: float):
+def find_blocks(mass, nb: int, tau: float, causal: bool = True):
     """o8 selection: (rank [B, H, T] int32, cnt [B, H, nb] int32) from block
     estimates [B, H, T] (any float type; compared as float64)."""
     m = np.ascontiguousarray(np.asarray(mass, np.float64))
     B, H, T = m.shape
+    assert T == rows_total(nb, causal)
     rank = np.empty((B, H, T), np.int32)
     cnt = np.empty((B, H, nb), np.int32)
-    lib().pa_oracle_find_blocks(_i(B), _i(H), _i(nb), _p(m), _d(tau), _p(rank), _p(cnt))
+    lib().pa_oracle_find_blocks(_i(B), _i(H), _i(nb), _p(m), _d(tau), _i(int(causal)), _p(rank), _p(cnt))
     return rank, cnt
 
 

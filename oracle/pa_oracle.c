@@ -529,32 +529,34 @@ void pa_oracle_sparse_attn_skip(int N, int H, int Hkv, int d, int G,
  *     z[R][c] = sum_{t<S} q[R*S + S-1-t] . k[c*S + t] / (sqrt(d) * S),
  * the box's reshaped product (query rows taken from S-1 down to 0, key rows
  * from 0 up).  Readings where the box is silent: the causal mask applies at the
- * strided level (c <= R: sub-blocks on or below the diagonal); each strided row
+ * strided level (c <= R: sub-blocks on or below the diagonal; non-causal: every
+ * column, the pages' video-generation use); each strided row
  * is softmax-normalised over its valid columns; the estimate of block kb is the
  * mean over the query block's 128/S strided rows of the probability falling
  * in kb's columns, so the estimates of a row sum to one.
- * mass [B][H][T], entry tri(qb)+kb. */
+ * mass [B][H][T], entry row_at(qb)+kb. */
 void pa_oracle_xattn_mass(int B, int N, int H, int Hkv, int d, int S,
                           const uint16_t *q, int64_t qsb, int64_t qss, int64_t qsh,
                           const uint16_t *k, int64_t ksb, int64_t kss, int64_t ksh,
-                          double *mass)
+                          int causal, double *mass)
 {
     int nb = N / BLK, rpb = BLK / S;  /* strided rows (and columns) per block */
-    int64_t T = tri(nb);
+    int64_t T = rows_total(causal, nb);
     double scale = 1.0 / (sqrt((double)d) * S);
     #pragma omp parallel for collapse(3) schedule(dynamic, 1)
     for (int b = 0; b < B; b++)
         for (int h = 0; h < H; h++)
             for (int qb = 0; qb < nb; qb++) {
                 int kvh = kv_of(h, H, Hkv);
-                double *m = mass + ((int64_t)b * H + h) * T + tri(qb);
-                int ncol = (qb + 1) * rpb;
+                double *m = mass + ((int64_t)b * H + h) * T + row_at(causal, nb, qb);
+                int ncol = row_len(causal, nb, qb) * rpb;
                 double *z = (double *)malloc(sizeof(double) * ncol);
-                for (int kb = 0; kb <= qb; kb++) m[kb] = 0.0;
+                for (int kb = 0; kb < row_len(causal, nb, qb); kb++) m[kb] = 0.0;
                 for (int r = 0; r < rpb; r++) {
                     int R = qb * rpb + r;
+                    int cend = causal ? R + 1 : ncol;  /* strided columns c < cend */
                     double zmax = -INFINITY;
-                    for (int c = 0; c <= R; c++) {
+                    for (int c = 0; c < cend; c++) {
                         double s = 0.0;
                         for (int t = 0; t < S; t++)
                             for (int e = 0; e < d; e++)
@@ -564,8 +566,8 @@ void pa_oracle_xattn_mass(int B, int N, int H, int Hkv, int d, int S,
                         if (z[c] > zmax) zmax = z[c];
                     }
                     double den = 0.0;
-                    for (int c = 0; c <= R; c++) den += exp(z[c] - zmax);
-                    for (int c = 0; c <= R; c++) m[c / rpb] += exp(z[c] - zmax) / den / rpb;
+                    for (int c = 0; c < cend; c++) den += exp(z[c] - zmax);
+                    for (int c = 0; c < cend; c++) m[c / rpb] += exp(z[c] - zmax) / den / rpb;
                 }
                 free(z);
             }
@@ -577,19 +579,20 @@ void pa_oracle_xattn_mass(int B, int N, int H, int Hkv, int d, int S,
  * first).  Sums run in 2^-40 fixed point as in o4; if no prefix reaches tau
  * (rounding), every block is kept.  rank [B][H][T] (the ordered blocks),
  * cnt [B][H][nb] (prefix length). */
-void pa_oracle_find_blocks(int B, int H, int nb, const double *mass, double tau,
+void pa_oracle_find_blocks(int B, int H, int nb, const double *mass, double tau, int causal,
                            int32_t *rank, int32_t *cnt)
 {
-    int64_t T = tri(nb);
+    int64_t T = rows_total(causal, nb);
     int64_t tfx = llrint(tau * 1099511627776.0);
     #pragma omp parallel for collapse(2) schedule(dynamic, 1)
     for (int b = 0; b < B; b++)
         for (int h = 0; h < H; h++)
             for (int qb = 0; qb < nb; qb++) {
-                const double *m = mass + ((int64_t)b * H + h) * T + tri(qb);
-                int32_t *out = rank + ((int64_t)b * H + h) * T + tri(qb);
+                const double *m = mass + ((int64_t)b * H + h) * T + row_at(causal, nb, qb);
+                int32_t *out = rank + ((int64_t)b * H + h) * T + row_at(causal, nb, qb);
+                int len = row_len(causal, nb, qb);
                 /* insertion sort by (estimate desc, index asc) */
-                for (int t = 0; t <= qb; t++) {
+                for (int t = 0; t < len; t++) {
                     int u = t;
                     while (u > 0 && (m[out[u - 1]] < m[t] || (m[out[u - 1]] == m[t] && out[u - 1] > t))) {
                         out[u] = out[u - 1];
@@ -598,8 +601,8 @@ void pa_oracle_find_blocks(int B, int H, int nb, const double *mass, double tau,
                     out[u] = t;
                 }
                 int64_t cum = 0;
-                int n = qb + 1;
-                for (int t = 0; t <= qb; t++) {
+                int n = len;
+                for (int t = 0; t < len; t++) {
                     cum += llrint(m[out[t]] * 1099511627776.0);
                     if (cum >= tfx) { n = t + 1; break; }
                 }

@@ -639,7 +639,7 @@ def test_skip_zero_threshold_and_given_decisions():
 
 
 # ------------------------------------------- o8 XAttention antidiagonal estimate
-def _antidiag_numpy(q, k, h, S):
+def _antidiag_numpy(q, k, h, S, causal=True):
     """numpy: the token-level score map of head h, each S x S sub-block summed
     along its antidiagonal (row offset S-1-t, column offset t), divided by
     sqrt(d) * S; strided rows softmax-normalised over sub-blocks on or below
@@ -654,14 +654,15 @@ def _antidiag_numpy(q, k, h, S):
     for t in range(S):
         A += Z[np.arange(n)[:, None] * S + S - 1 - t, np.arange(n)[None, :] * S + t]
     A /= math.sqrt(d) * S
-    A[np.triu_indices(n, 1)] = -np.inf
+    if causal:
+        A[np.triu_indices(n, 1)] = -np.inf
     P = scipy.special.softmax(A, axis=1)
     rpb = 128 // S
     nb = N // 128
     out = []
     for qb in range(nb):
         rows = P[qb * rpb:(qb + 1) * rpb]
-        out.extend(rows[:, kb * rpb:(kb + 1) * rpb].sum() / rpb for kb in range(qb + 1))
+        out.extend(rows[:, kb * rpb:(kb + 1) * rpb].sum() / rpb for kb in range(qb + 1 if causal else nb))
     return np.array(out)
 
 
@@ -678,6 +679,27 @@ def test_xattn_mass_is_the_antidiagonal_sum_softmax(S):
     for qb in range(nb):
         np.testing.assert_allclose(mass[0, :, qb * (qb + 1) // 2: qb * (qb + 1) // 2 + qb + 1].sum(-1), 1.0,
                                    atol=1e-12)
+
+
+@pytest.mark.parametrize("S", [4, 16])
+def test_xattn_noncausal_is_the_unmasked_antidiagonal_softmax(S):
+    """Non-causal o8: every strided column, rows of all nb blocks summing to one;
+    S = 1 on the last block equals o3's non-causal mass."""
+    w = synth.small_workload(seqlen=384, heads=2, kv_heads=1, head_dim=32, groups=1)
+    x = synth.make_inputs(w)
+    mass = oracle.xattn_mass(x["q"], x["k"], S, causal=False)
+    for h in range(2):
+        np.testing.assert_allclose(mass[0, h], _antidiag_numpy(x["q"], x["k"], h, S, causal=False),
+                                   rtol=1e-10, atol=1e-13)
+    np.testing.assert_allclose(mass.reshape(1, 2, 3, 3).sum(-1), 1.0, atol=1e-12)
+    m1 = oracle.xattn_mass(x["q"], x["k"], 1, causal=False)
+    np.testing.assert_allclose(m1[:, :, 6:9], oracle.head_mass(x["q"], x["k"], causal=False), rtol=1e-12,
+                               atol=1e-15)
+    rank, cnt = oracle.find_blocks(mass, 3, 0.99, causal=False)
+    for h in range(2):
+        for qb in range(3):
+            v = mass[0, h, qb * 3:(qb + 1) * 3]
+            assert list(rank[0, h, qb * 3:(qb + 1) * 3]) == sorted(range(3), key=lambda kb: (-v[kb], kb))
 
 
 def test_xattn_stride_one_is_the_exact_mass():

@@ -60,12 +60,7 @@ MUTANTS = [
      "            use[t] = skip_in ? !skip_in[base + blk[t]] : 1;"),
     ("xattn_main_diagonal", "q[b * qsb + (int64_t)(R * S + S - 1 - t) * qss + h * qsh + e]",
      "q[b * qsb + (int64_t)(R * S + t) * qss + h * qsh + e]"),
-    ("xattn_no_causal", [("for (int c = 0; c <= R; c++) {\n                        double s = 0.0;",
-                          "for (int c = 0; c < ncol; c++) {\n                        double s = 0.0;"),
-                         ("for (int c = 0; c <= R; c++) den += exp(z[c] - zmax);",
-                          "for (int c = 0; c < ncol; c++) den += exp(z[c] - zmax);"),
-                         ("for (int c = 0; c <= R; c++) m[c / rpb] +=", "for (int c = 0; c < ncol; c++) m[c / rpb] +=")],
-     None),
+    ("xattn_no_causal", "int cend = causal ? R + 1 : ncol;", "int cend = ncol;"),
     ("xattn_scale_without_stride", "double scale = 1.0 / (sqrt((double)d) * S);", "double scale = 1.0 / sqrt((double)d);"),
     ("find_blocks_strict", "if (cum >= tfx) { n = t + 1; break; }", "if (cum > tfx) { n = t + 1; break; }"),
     ("find_blocks_ascending", "while (u > 0 && (m[out[u - 1]] < m[t] ||", "while (u > 0 && (m[out[u - 1]] > m[t] ||"),
