@@ -238,15 +238,15 @@ def build_mask(scores: torch.Tensor, q: torch.Tensor, k: torch.Tensor, num_group
 
 
 def xattn_mask(q: torch.Tensor, k: torch.Tensor, stride: int = 8, tau: float = 0.9,
-               workspace: torch.Tensor | None = None):
+               workspace: torch.Tensor | None = None, causal: bool = True):
     """pa_xattn_mask -> (rank int32 [B, H, T], cnt int32 [B, H, nb], mass fp32
     [B, H, T]); feed rank/cnt to block_sparse_attn with num_groups = H."""
     _cuda_bf16(q, "q")
     _cuda_bf16(k, "k")
     B, N, H, d = q.shape
-    shape = make_shape(q, k, H)
+    shape = make_shape(q, k, H, causal)
     nb = N // 128
-    T = nb * (nb + 1) // 2
+    T = rows_total(nb, causal)
     i32 = dict(device=q.device, dtype=torch.int32)
     rank = torch.empty(B, H, T, **i32)
     cnt = torch.empty(B, H, nb, **i32)

@@ -409,8 +409,12 @@ pa_status launch_xattn(const pa_shape *s, int S, float tau, const void *q, pa_st
     p.rows = rows;
     p.nchunk = (rows + 127) / 128;
     const int mtiles = (rows + 127) / 128;
+    p.causal = causal_of(s) ? 1 : 0;
     long long per = 0;
-    for (int mt = 0; mt < mtiles; ++mt) per += mt / 2 + 1;
+    if (p.causal)
+        for (int mt = 0; mt < mtiles; ++mt) per += mt / 2 + 1;
+    else
+        per = static_cast<long long>(mtiles) * ((rows + 255) / 256);
     p.units_per_bh = per;
     p.num_units = per * B * H;
     p.c2 = static_cast<float>(1.4426950408889634 / (std::sqrt(static_cast<double>(d)) * S));
@@ -421,6 +425,7 @@ pa_status launch_xattn(const pa_shape *s, int S, float tau, const void *q, pa_st
     if (r) return r;
     pa::XselParams sp{};
     sp.B = B; sp.H = H; sp.nb = nb; sp.rows = rows; sp.nchunk = p.nchunk; sp.S = S;
+    sp.causal = p.causal;
     sp.tau = tau;
     sp.part_s = p.part_s;
     sp.part_m = p.part_m;
@@ -796,7 +801,6 @@ pa_status pa_xattn_mask(const pa_shape *shape, int32_t stride, float tau, const 
                         size_t ws_bytes, pa_stream_t stream) {
     pa_status r;
     if ((r = check_shape(shape)) || (r = check_xstride(stride))) return r;
-    if (!causal_of(shape)) return fail(PA_ERR_UNSUPPORTED, "the XAttention estimator is causal only");
     if (!(tau > 0.0f && tau <= 1.0f))
         return fail(PA_ERR_INVALID_ARG, "tau must be in (0, 1] (got %g)", static_cast<double>(tau));
     if ((r = check_tensor(q, qs, "q")) || (r = check_tensor(k, ks, "k"))) return r;

@@ -36,6 +36,7 @@ struct XattnParams {
     long long units_per_bh; // output tiles per (b, h)
     long long num_units;
     float c2;               // log2(e) / (sqrt(d) * S)
+    int causal;             // 0: every strided column of every row (square rows of estimates)
     float *part_s;          // [B][H][nb][rows]   sum of 2^(x - m) over the block's valid columns
     float *part_m;          // [B][H][nchunk][rows]  row max of the 128-column chunk (log2 units)
     uint64_t timeout_ns;
@@ -55,6 +56,12 @@ __device__ __forceinline__ XUnit xattn_decode(const XattnParams &p, long long u)
     const long long w = u - bh * p.units_per_bh;
     x.b = static_cast<int>(bh / p.H);
     x.h = static_cast<int>(bh % p.H);
+    if (!p.causal) {  // every row tile needs every column tile
+        const long long ntn = (p.rows + 255) / 256;
+        x.mt = static_cast<int>(w / ntn);
+        x.nt = static_cast<int>(w % ntn);
+        return x;
+    }
     long long a = static_cast<long long>((sqrt(1.0 + 4.0 * static_cast<double>(w)) - 1.0) * 0.5);
     while (a > 0 && a * (a + 1) > w) --a;
     while ((a + 1) * (a + 2) <= w) ++a;
@@ -198,8 +205,11 @@ __global__ void __launch_bounds__(192, 1)
                     mbar_arrive(&acc_empty[acc]);  // the accumulator is in registers
                 }
                 const int C0 = x.nt * 256 + half * 128;  // first strided column of this chunk
-                if (R >= p.rows || C0 > R) continue;     // past the last row, or above the diagonal
-                const int lim = R - C0;                  // columns C0 + j with j <= lim are valid
+                // past the last row or column, or (causal) above the diagonal
+                if (R >= p.rows || C0 >= p.rows || (p.causal && C0 > R)) continue;
+                // columns C0 + j with j <= lim are valid: on or below the diagonal (causal) and
+                // inside the sequence (the columns past it are TMA zero fill)
+                const int lim = min(p.causal ? R - C0 : 127, p.rows - 1 - C0);
 #pragma unroll
                 for (int j = 0; j < 128; ++j)
                     if (j > lim) r[j] = 0xFF800000u;     // -inf
@@ -224,7 +234,8 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                     for (int j = 0; j < CPB; ++j)
                         acc4[j & 3] += ex2(fmaf(__uint_as_float(r[kbl * CPB + j]), p.c2, -m2));
-                    if (kb <= qb) p.part_s[(bh * p.nb + kb) * p.rows + R] = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
+                    if (p.causal ? kb <= qb : kb < p.nb)
+                        p.part_s[(bh * p.nb + kb) * p.rows + R] = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
                 }
             }
         }
@@ -247,6 +258,7 @@ __global__ void __launch_bounds__(192, 1)
 // ------------------------------------------------------------ selection
 struct XselParams {
     int B, H, nb, rows, nchunk, S;
+    int causal;
     float tau;
     const float *part_s;  // as XattnParams
     const float *part_m;
@@ -279,9 +291,10 @@ __global__ void __launch_bounds__(256) xattn_select_kernel(XselParams p) {
     const int tid = threadIdx.x;
     const int CPB = 128 / p.S;          // strided rows of the query block (<= 32)
     const int R0 = qb * CPB;
-    const int cq = R0 / 128;            // the rows' last 128-column chunk
-    const int n = qb + 1;
-    const long long T = static_cast<long long>(p.nb) * (p.nb + 1) / 2;
+    const int cq = p.causal ? R0 / 128 : p.nchunk - 1;  // the rows' last 128-column chunk
+    const int n = p.causal ? qb + 1 : p.nb;              // blocks of the row
+    const long long T = p.causal ? static_cast<long long>(p.nb) * (p.nb + 1) / 2 : static_cast<long long>(p.nb) * p.nb;
+    const long long row_at = p.causal ? static_cast<long long>(qb) * (qb + 1) / 2 : static_cast<long long>(qb) * p.nb;
     const float *ps = p.part_s + bh * p.nb * static_cast<long long>(p.rows) + R0;
     const float *pm = p.part_m + bh * p.nchunk * static_cast<long long>(p.rows) + R0;
     const long long rs = p.rows;
@@ -302,7 +315,7 @@ __global__ void __launch_bounds__(256) xattn_select_kernel(XselParams p) {
     // 2. each row's softmax denominator over the blocks 0..qb
     const float Mr = rowM[r];
     float L = 0.0f;
-    for (int kb = sl; kb <= qb; kb += slots) L += exp2f(pm[(kb / p.S) * rs + r] - Mr) * ps[kb * rs + r];
+    for (int kb = sl; kb < n; kb += slots) L += exp2f(pm[(kb / p.S) * rs + r] - Mr) * ps[kb * rs + r];
     red[tid] = L;
     __syncthreads();
     if (tid < CPB) {
@@ -326,7 +339,7 @@ __global__ void __launch_bounds__(256) xattn_select_kernel(XselParams p) {
                 flag_status(kStNonFinite);
                 e = 0.0f;
             }
-            if (p.mass) p.mass[bh * T + static_cast<long long>(qb) * (qb + 1) / 2 + kb] = e;
+            if (p.mass) p.mass[bh * T + row_at + kb] = e;
             key = (static_cast<unsigned long long>(xsel_desc_key(e)) << 32) | static_cast<uint32_t>(kb);
         }
         keys[kb] = key;
@@ -349,7 +362,7 @@ __global__ void __launch_bounds__(256) xattn_select_kernel(XselParams p) {
         }
     }
     // 4. ranked list and the shortest prefix reaching tau (2^-40 fixed point)
-    int32_t *out = p.rank + bh * T + static_cast<long long>(qb) * (qb + 1) / 2;
+    int32_t *out = p.rank + bh * T + row_at;
     for (int i = tid; i < n; i += blockDim.x) out[i] = static_cast<int32_t>(keys[i] & 0xFFFFFFFFu);
     const long long tfx = __double2ll_rn(static_cast<double>(p.tau) * 1099511627776.0);
     const int per = (n + 255) / 256;    // <= 16 entries per thread

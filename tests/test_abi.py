@@ -165,9 +165,6 @@ def test_noncausal_shape_sizes_and_errors(L):
     assert pa.workspace_size(s, pa.make_budget(pa.FIXED_FRACTION, 0, 100)) == 0
     st = pa.Strides(0, 512, 64)
     assert L.pa_pool_heads(ctypes.byref(s), 16, st, 16, st, 16, 16, None) == 1
-    s.non_causal = 1
-    assert L.pa_xattn_mask(ctypes.byref(s), 8, ctypes.c_float(0.9), 16, st, 16, st, 16, 16, None, 256, 1 << 30,
-                           None) == 2
 
 
 def test_varlen_validation_and_workspace(L):

@@ -67,7 +67,8 @@ MUTANTS = [
     ("noncausal_budget_row_scaled", ": clampi(kh, forced(qb), nb);",
      ": clampi(((int64_t)kh * (qb + 1) + nb - 1) / nb, forced(qb), nb);"),
     ("noncausal_dense_still_causal", "int nkeys = causal ? i + 1 : N;", "int nkeys = i + 1;"),
-    ("noncausal_rank_keeps_only_lower_blocks", "int len = row_len(causal, nb, qb);", "int len = qb + 1;"),
+    ("noncausal_rank_keeps_only_lower_blocks", "int len = row_len(causal, nb, qb);\n                out[0] = 0;",
+     "int len = qb + 1;\n                out[0] = 0;"),
     ("skip_threshold_log2", "double lnl = (lambda > 0.0) ? log(lambda) : -INFINITY;",
      "double lnl = (lambda > 0.0) ? log2(lambda) : -INFINITY;"),
 ]

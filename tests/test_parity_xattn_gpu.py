@@ -82,6 +82,35 @@ def test_xattn_parity(case):
     assert diff.max() <= 2e-2 and diff.mean() <= 2e-3, (diff.max(), diff.mean())
 
 
+@pytest.mark.parametrize("N,S,d", [(1024, 8, 64), (1152, 16, 128), (640, 4, 128)])
+def test_xattn_noncausal_parity(N, S, d):
+    """Non-causal estimates (every strided column; the last column tile is
+    ragged when N/S is not a multiple of 256), lists and counts over all nb
+    blocks, and the non-causal attention they drive."""
+    H, Hkv, tau = 4, 2, 0.9
+    w = synth.small_workload(seqlen=N, heads=H, kv_heads=Hkv, head_dim=d, groups=H, needles=8, seed=760 + S)
+    x = synth.make_inputs(w)
+    qc, kc, vc = x["q"], x["k"], x["v"]
+    q, k, v = qc.cuda(), kc.cuda(), vc.cuda()
+    nb = N // 128
+    rank, cnt, mass = pa.xattn_mask(q, k, S, tau, causal=False)
+    o = pa.block_sparse_attn(q, k, v, rank, cnt, H, causal=False)
+    torch.cuda.synchronize()
+    assert pa.device_status() == 0
+    mg = mass.double().cpu().numpy()
+    ref = oracle.xattn_mass(qc, kc, S, causal=False)
+    assert np.all(np.abs(mg - ref) <= 2e-5 + 2e-3 * ref), np.abs(mg - ref).max()
+    np.testing.assert_allclose(mg.reshape(1, H, nb, nb).sum(-1), 1.0, atol=1e-4)
+    rank_ref, cnt_ref = oracle.find_blocks(mass.cpu().numpy(), nb, float(np.float32(tau)), causal=False)
+    assert np.array_equal(rank.cpu().numpy(), rank_ref)
+    assert np.array_equal(cnt.cpu().numpy(), cnt_ref)
+    items = [(0, h, qb) for h in range(H) for qb in range(nb)]
+    oref, _ = oracle.sparse_attn(qc, kc, vc, rank.cpu().numpy(), cnt.cpu().numpy(), H, items, causal=False)
+    og = o.float().cpu().numpy()
+    diff = np.abs(np.stack([og[0, qb * 128:(qb + 1) * 128, h] for (_, h, qb) in items]) - oref)
+    assert diff.max() <= 2e-2 and diff.mean() <= 2e-3, (diff.max(), diff.mean())
+
+
 def test_xattn_full_size_sampled():
     """The 32K Llama shape at S = 8: estimates of sampled (head, query block)
     rows against the oracle on the matching token range, lists complete and
