@@ -244,10 +244,10 @@ class XPipeline(Pipeline):
     pa_xattn_mask (strided antidiagonal GEMM + selection) then the same
     attention call with one list per head."""
 
-    def __init__(self, q, k, v, S, tau, skip=0.0):
+    def __init__(self, q, k, v, S, tau, skip=0.0, causal=True):
         import block_sparse_attention_pa_b200 as pa
         B, N, H, d = q.shape
-        super().__init__(q, k, v, H, 1, 0.0, 1000, 1, skip, proxies=False)
+        super().__init__(q, k, v, H, 1, 0.0, 1000, 1, skip, proxies=False, causal=causal)
         self.S, self.tau = S, tau
         self.xws = torch.empty(max(int(self.L.pa_xattn_workspace_size(ctypes.byref(self.shape), S)), 256),
                                device=q.device, dtype=torch.uint8)
@@ -491,7 +491,7 @@ def main():
     skip = args.skip_threshold
     xattn = args.estimator == "xattn"
     if xattn:
-        pipe = XPipeline(q, k, v, args.xattn_stride, args.tau, skip)
+        pipe = XPipeline(q, k, v, args.xattn_stride, args.tau, skip, causal=not args.non_causal)
     else:
         pipe = Pipeline(q, k, v, G, mode, gamma, frac, stride, skip, causal=not args.non_causal)
     sampler = None if args.no_clocks else ClockSampler(local)
@@ -550,9 +550,14 @@ def main():
         # strided antidiagonal GEMM: executed 128 x 256 tiles; exact causal work beside it
         S = args.xattn_stride
         rows = w.seqlen // S
-        tiles = sum(mt // 2 + 1 for mt in range((rows + 127) // 128))
+        mtiles = (rows + 127) // 128
+        if args.non_causal:
+            tiles = mtiles * ((rows + 255) // 256)
+            x_exact = B * H * rows * rows * 2 * S * d
+        else:
+            tiles = sum(mt // 2 + 1 for mt in range(mtiles))
+            x_exact = B * H * (rows * (rows + 1) // 2) * 2 * S * d
         x_exec = B * H * tiles * 2 * 128 * 256 * S * d
-        x_exact = B * H * (rows * (rows + 1) // 2) * 2 * S * d
         stage_roofline = {
             "xattn_estimate": {"ms": float(stages[1]), "TFLOP/s": x_exec / (stages[1] * 1e-3) / 1e12,
                                "frac_tensor": x_exec / (stages[1] * 1e-3) / 1e12 / peak,
