@@ -561,7 +561,7 @@ def main():
         stage_roofline = {
             "xattn_estimate": {"ms": float(stages[1]), "TFLOP/s": x_exec / (stages[1] * 1e-3) / 1e12,
                                "frac_tensor": x_exec / (stages[1] * 1e-3) / 1e12 / peak,
-                               "flops_executed": x_exec, "flops_exact_causal": x_exact},
+                               "flops_executed": x_exec, "flops_exact": x_exact},
             "attn": {"ms": attn_ms, "TFLOP/s": achieved, "frac_tensor": achieved / peak},
         }
 
