@@ -284,8 +284,9 @@ PA_API pa_status pa_block_sparse_attn_skip(const pa_shape *shape,
  * No block is forced into the set.  bf16 tensor-core products with fp32
  * accumulation; mass (nullable) fp32.  ws: device workspace of
  * ws_bytes >= pa_xattn_workspace_size(shape, S); tau in (0, 1].  The shape's
- * num_groups is not used; the shape must be causal (PA_ERR_UNSUPPORTED
- * otherwise). */
+ * num_groups is not used.  Non-causal shapes (shape->non_causal = 1; the
+ * pages' video-generation use) take every strided column, c < N/S, and
+ * rows of all nb blocks. */
 PA_API size_t pa_xattn_workspace_size(const pa_shape *shape, int32_t stride);
 
 PA_API pa_status pa_xattn_mask(const pa_shape *shape, int32_t stride, float tau,
