@@ -286,7 +286,7 @@ pa_status launch_tile_gemm_t(const CUtensorMap &a, const CUtensorMap &b, const p
     PA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     const long long grid = std::min<long long>(p.num_units, num_sms());
     if (grid <= 0) return PA_OK;
-    kern<<<static_cast<unsigned>(grid), 192, smem, st>>>(a, b, p);
+    kern<<<static_cast<unsigned>(grid), pa::kTileThreads, smem, st>>>(a, b, p);
     PA_CUDA(cudaGetLastError());
     return PA_OK;
 }

@@ -15,15 +15,16 @@
 //                max m and sum l of exp2 of the log2-scaled logits over the
 //                tile (the inputs of an exact softmax combine).
 //
-// Persistent, warp-specialised CTA (one per SM, 192 threads):
+// Persistent, warp-specialised CTA (one per SM, 320 threads):
 //   warp 0     TMA producer: the unit's A tile (double-buffered) and a ring of
 //              B stages of two 128-row key tiles, 128-byte swizzle.
 //   warp 1     allocates 512 TMEM columns (two fp32 128x256 accumulators) and
 //              issues tcgen05.mma (M=128, N=256, K=16: two key tiles per
 //              instruction, so each wait of the issuing thread covers twice
 //              the tensor work) from one thread.
-//   warps 2-5  epilogue: each thread owns one accumulator row (TMEM lane),
-//              reads it with tcgen05.ld and reduces it.
+//   warps 2-9  epilogue: warps 2-5 take the first key tile of each pair, warps
+//              6-9 the second; each thread owns one accumulator row (TMEM
+//              lane) of its tile, reads it with tcgen05.ld and reduces it.
 // A unit is a run of up to `chunk` consecutive tiles sharing one A tile.
 #pragma once
 #include "sm100.cuh"
@@ -31,6 +32,8 @@
 namespace pa {
 
 enum { MODE_SCORES = 0, MODE_MASS = 1 };
+
+constexpr int kTileThreads = 320;  // producer, MMA issuer, eight epilogue warps
 
 struct TileParams {
     int B, nb, NH;         // NH: proxy groups (scores) or q heads (mass)
@@ -111,7 +114,7 @@ struct TileSmem {
 __device__ __forceinline__ int pairs_of(const Unit &un) { return (un.kb1 - un.kb0 + 1) >> 1; }
 
 template <int D, int MODE>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kTileThreads, 1)
     tile_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      TileParams p) {
     using S = TileSmem<D>;
@@ -145,7 +148,7 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(&a_full[i], 1);
             mbar_init(&a_empty[i], 1);
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], 128);
+            mbar_init(&acc_empty[i], 256);
         }
         for (int i = 0; i < NST; ++i) {
             mbar_init(&b_full[i], 1);
@@ -251,7 +254,10 @@ __global__ void __launch_bounds__(192, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------ epilogue
+        // Warps 2..9: warp w reduces TMEM lanes 32 (w & 3) .. +31 of tile (w - 2) / 4
+        // of each key-tile pair, so two warps per SMSP share a pair.
         const int q4 = static_cast<int>(warp & 3);
+        const int jt = static_cast<int>(warp - 2) >> 2;
         const int row = q4 * 32 + static_cast<int>(lane);
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
         // A row -> (query block within the A tile, token offset inside that block)
@@ -260,7 +266,7 @@ __global__ void __launch_bounds__(192, 1)
         const int toff = (row % rows_per_qb) * p.stride + p.stride - 1;
         const int span = min(rows_per_qb, 32);  // lanes of a warp that share a query block
         const int wpq = rows_per_qb / 32;       // warps that share a query block (0: part of one warp)
-        long long pair = 0, tile = 0;
+        long long pair = 0;
         bool ok = true;
         for (long long u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
             const Unit un = decode_unit(p, u, MODE);
@@ -270,79 +276,73 @@ __global__ void __launch_bounds__(192, 1)
                 const int nt = min(2, un.kb1 - kb0);
                 if (!warp_wait(&acc_full[acc], (pair >> 1) & 1, wc)) { ok = false; break; }
                 tc_fence_after();
-                float mx[2];
-                float lsum[2];
-                for (int j = 0; j < nt; ++j, ++tile) {
-                    const int kb = kb0 + j;
-                    const bool diag = p.causal && (kb == qbw);
-                    uint32_t r[128];
-                    tmem_ld128(lane_base + acc * 256 + j * 128, r);
-                    if (j == nt - 1) {
-                        // the accumulator pair is in registers: hand TMEM back to the MMA warp
-                        tc_fence_before();
-                        mbar_arrive(&acc_empty[acc]);
-                    }
-                    if (diag) {
-#pragma unroll
-                        for (int c = 0; c < 128; ++c)
-                            if (c > toff) r[c] = 0xFF800000u;  // -inf above the diagonal (j > i)
-                    }
-                    float m8[16];
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        const uint32_t *v = r + 8 * c;
-                        m8[c] = fmax3(fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2])),
-                                      fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5])),
-                                      fmaxf(__uint_as_float(v[6]), __uint_as_float(v[7])));
-                    }
-                    mx[j] = fmax3(fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmax3(m8[6], m8[7], m8[8])),
-                                  fmax3(m8[9], m8[10], m8[11]), fmax3(m8[12], m8[13], fmaxf(m8[14], m8[15])));
-                    if (MODE == MODE_MASS) {
-                        // log2-domain row max and sum of exp2 over the valid entries
-                        const float m = mx[j] * p.scale;
-                        float acc8[8];
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) acc8[c] = 0.0f;
-#pragma unroll
-                        for (int c = 0; c < 128; ++c) acc8[c & 7] += ex2(fmaf(__uint_as_float(r[c]), p.scale, -m));
-                        lsum[j] = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) + ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
-                    }
+                if (jt >= nt) {  // a unit's odd last tile: nothing for this warp
+                    tc_fence_before();
+                    mbar_arrive(&acc_empty[acc]);
+                    continue;
                 }
-                for (int j = 0; j < nt; ++j) {
-                    const int kb = kb0 + j;
-                    const long long tj = tile - nt + j;
-                    if (MODE == MODE_SCORES) {
-                        float w = mx[j] * p.scale;
+                const int kb = kb0 + jt;
+                const long long tj = pair * 2 + jt;  // a distinct index per tile (reduction ring slot)
+                const bool diag = p.causal && (kb == qbw);
+                uint32_t r[128];
+                tmem_ld128(lane_base + acc * 256 + jt * 128, r);
+                // this tile is in registers: hand its TMEM back to the MMA warp
+                tc_fence_before();
+                mbar_arrive(&acc_empty[acc]);
+                if (diag) {
 #pragma unroll
-                        for (int o = 16; o > 0; o >>= 1)
-                            if (o < span) w = fmaxf(w, __shfl_xor_sync(0xffffffffu, w, o));
-                        // tiles above this query block's diagonal, and A rows past the last
-                        // block (zero-filled), give no score
-                        const bool valid = (!p.causal || kb <= qbw) && qbw < p.nb;
-                        if (valid && (static_cast<int>(lane) & (span - 1)) == 0) {
-                            const long long T = p.causal ? static_cast<long long>(p.nb) * (p.nb + 1) / 2
-                                                         : static_cast<long long>(p.nb) * p.nb;
-                            const long long idx = (static_cast<long long>(un.b) * p.NH + un.bh_head) * T +
-                                                  (p.causal ? static_cast<long long>(qbw) * (qbw + 1) / 2
-                                                            : static_cast<long long>(qbw) * p.nb) + kb;
-                            if (wpq <= 1) {
-                                p.scores[idx] = w;
-                            } else {
-                                const int slot = static_cast<int>(tj & 7) * 2 + (qsub & 1);
-                                atomicMax(&red_max[slot], f2ord(w));
-                                __threadfence_block();
-                                if (atomicAdd(&red_cnt[slot], 1u) == static_cast<uint32_t>(wpq - 1)) {
-                                    const uint32_t best = atomicExch(&red_max[slot], 0u);
-                                    atomicExch(&red_cnt[slot], 0u);
-                                    p.scores[idx] = ord2f(best);
-                                }
+                    for (int c = 0; c < 128; ++c)
+                        if (c > toff) r[c] = 0xFF800000u;  // -inf above the diagonal (j > i)
+                }
+                float m8[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const uint32_t *v = r + 8 * c;
+                    m8[c] = fmax3(fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2])),
+                                  fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5])),
+                                  fmaxf(__uint_as_float(v[6]), __uint_as_float(v[7])));
+                }
+                const float mx = fmax3(fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                                             fmax3(m8[6], m8[7], m8[8])),
+                                       fmax3(m8[9], m8[10], m8[11]), fmax3(m8[12], m8[13], fmaxf(m8[14], m8[15])));
+                if (MODE == MODE_SCORES) {
+                    float w = mx * p.scale;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1)
+                        if (o < span) w = fmaxf(w, __shfl_xor_sync(0xffffffffu, w, o));
+                    // tiles above this query block's diagonal, and A rows past the last
+                    // block (zero-filled), give no score
+                    const bool valid = (!p.causal || kb <= qbw) && qbw < p.nb;
+                    if (valid && (static_cast<int>(lane) & (span - 1)) == 0) {
+                        const long long T = p.causal ? static_cast<long long>(p.nb) * (p.nb + 1) / 2
+                                                     : static_cast<long long>(p.nb) * p.nb;
+                        const long long idx = (static_cast<long long>(un.b) * p.NH + un.bh_head) * T +
+                                              (p.causal ? static_cast<long long>(qbw) * (qbw + 1) / 2
+                                                        : static_cast<long long>(qbw) * p.nb) + kb;
+                        if (wpq <= 1) {
+                            p.scores[idx] = w;
+                        } else {
+                            const int slot = static_cast<int>(tj & 7) * 2 + (qsub & 1);
+                            atomicMax(&red_max[slot], f2ord(w));
+                            __threadfence_block();
+                            if (atomicAdd(&red_cnt[slot], 1u) == static_cast<uint32_t>(wpq - 1)) {
+                                const uint32_t best = atomicExch(&red_max[slot], 0u);
+                                atomicExch(&red_cnt[slot], 0u);
+                                p.scores[idx] = ord2f(best);
                             }
                         }
-                    } else {
-                        const long long idx =
-                            ((static_cast<long long>(un.b) * p.H + un.bh_head) * p.nb + kb) * 128 + row;
-                        p.partial[idx] = make_float2(mx[j] * p.scale, lsum[j]);
                     }
+                } else {
+                    // log2-domain row max and sum of exp2 over the valid entries
+                    const float m = mx * p.scale;
+                    float acc8[8];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) acc8[c] = 0.0f;
+#pragma unroll
+                    for (int c = 0; c < 128; ++c) acc8[c & 7] += ex2(fmaf(__uint_as_float(r[c]), p.scale, -m));
+                    const float lsum = ((acc8[0] + acc8[1]) + (acc8[2] + acc8[3])) + ((acc8[4] + acc8[5]) + (acc8[6] + acc8[7]));
+                    const long long idx = ((static_cast<long long>(un.b) * p.H + un.bh_head) * p.nb + kb) * 128 + row;
+                    p.partial[idx] = make_float2(m, lsum);
                 }
             }
         }
