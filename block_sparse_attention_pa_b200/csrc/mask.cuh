@@ -12,59 +12,109 @@
 //                        masses along the last row's list -> k_h, then the
 //                        per-row counts
 #pragma once
+#include <cooperative_groups.h>
+
 #include "sm100.cuh"
 
 namespace pa {
 
 // ------------------------------------------------------------ mass combine
 // partial: [B*H][nb][128] (m, l) with m the log2-domain row max of a tile and
-// l the sum of exp2(x - m) over its valid entries.
-__global__ void __launch_bounds__(256) mass_combine_kernel(const float2 *__restrict__ partial,
-                                                           float *__restrict__ mass, int nb) {
-    __shared__ float sM[2][128], sL[2][128];
-    const long long bh = blockIdx.x;
+// l the sum of exp2(x - m) over its valid entries (m = -inf, l = 0 for a tile
+// with no valid entry in the row).
+//
+// One cluster of kMcCta CTAs per (b, h); CTA c owns the key blocks
+// [c*nb/kMcCta, (c+1)*nb/kMcCta).  Each CTA reduces its blocks to a per-row
+// (M, L); after a cluster barrier every CTA combines the kMcCta partial
+// statistics of each row in CTA order through distributed shared memory (the
+// same fixed order in every CTA, so all hold identical normalisers and the
+// result is deterministic), then writes mass[kb] for its own blocks.
+constexpr int kMcCta = 8;
+constexpr int kMcThreads = 512;
+
+// (M, L) <- (M, L) merged with the tile statistics v[0..n), in log2 domain
+template <int n>
+__device__ __forceinline__ void online_merge(float &M, float &L, const float2 (&v)[n]) {
+    float mx = M;
+#pragma unroll
+    for (int j = 0; j < n; ++j) mx = fmaxf(mx, v[j].x);
+    if (mx == -INFINITY) return;  // nothing valid so far
+    float l = (M == -INFINITY) ? 0.0f : L * exp2f(M - mx);
+#pragma unroll
+    for (int j = 0; j < n; ++j) l += (v[j].x == -INFINITY) ? 0.0f : v[j].y * exp2f(v[j].x - mx);
+    M = mx;
+    L = l;
+}
+
+__global__ void __cluster_dims__(kMcCta, 1, 1) __launch_bounds__(kMcThreads)
+    mass_combine_kernel(const float2 *__restrict__ partial, float *__restrict__ mass, int nb) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    __shared__ float sM[4][128], sL[4][128];  // per quarter, then [0] = this CTA's (M, L)
+    __shared__ float gM[128], gI[128];         // row max and 1/L over all blocks
+    const long long bh = blockIdx.x / kMcCta;
+    const int c = static_cast<int>(cluster.block_rank());
+    const int lo = static_cast<int>(static_cast<long long>(c) * nb / kMcCta);
+    const int hi = static_cast<int>(static_cast<long long>(c + 1) * nb / kMcCta);
     const float2 *part = partial + bh * nb * 128;
     const int tid = threadIdx.x;
-    const int r = tid & 127, half = tid >> 7;
+    const int r = tid & 127, qt = tid >> 7;  // row, quarter of the CTA's blocks
+
     float M = -INFINITY, L = 0.0f;
-    for (int kb = half; kb < nb; kb += 2) {
-        const float2 v = part[static_cast<long long>(kb) * 128 + r];
-        if (v.x > M) {
-            L = L * exp2f(M - v.x) + v.y;
-            M = v.x;
-        } else {
-            L += v.y * exp2f(v.x - M);
-        }
+    int kb = lo + qt;
+    for (; kb + 12 < hi; kb += 16) {  // four independent loads per merge
+        float2 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = part[static_cast<long long>(kb + 4 * j) * 128 + r];
+        online_merge<4>(M, L, v);
     }
-    sM[half][r] = M;
-    sL[half][r] = L;
+    for (; kb < hi; kb += 4) {
+        float2 v[1] = {part[static_cast<long long>(kb) * 128 + r]};
+        online_merge<1>(M, L, v);
+    }
+    sM[qt][r] = M;
+    sL[qt][r] = L;
     __syncthreads();
     if (tid < 128) {
-        const float M0 = sM[0][r], M1 = sM[1][r];
-        const float Mx = fmaxf(M0, M1);
-        const float Lx = (M0 == -INFINITY ? 0.0f : sL[0][r] * exp2f(M0 - Mx)) +
-                         (M1 == -INFINITY ? 0.0f : sL[1][r] * exp2f(M1 - Mx));
-        sM[0][r] = Mx;
-        sL[0][r] = 1.0f / Lx;
+        float2 v[3] = {make_float2(sM[1][r], sL[1][r]), make_float2(sM[2][r], sL[2][r]),
+                       make_float2(sM[3][r], sL[3][r])};
+        float m0 = sM[0][r], l0 = sL[0][r];
+        online_merge<3>(m0, l0, v);
+        sM[0][r] = m0;
+        sL[0][r] = l0;
     }
-    __syncthreads();
+    cluster.sync();  // every CTA's (M, L) visible cluster-wide
+    if (tid < 128) {
+        float Mx = -INFINITY, Lx = 0.0f;
+#pragma unroll 1
+        for (int cc = 0; cc < kMcCta; ++cc) {
+            const float *rM = cluster.map_shared_rank(&sM[0][0], cc);
+            const float *rL = cluster.map_shared_rank(&sL[0][0], cc);
+            float2 v[1] = {make_float2(rM[r], rL[r])};
+            online_merge<1>(Mx, Lx, v);
+        }
+        gM[r] = Mx;
+        gI[r] = 1.0f / Lx;
+    }
+    cluster.sync();  // remote reads done before any CTA exits; gM/gI visible
+
     const int warp = tid >> 5, lane = tid & 31;
     float Mr[4], Ir[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        Mr[j] = sM[0][lane + 32 * j];
-        Ir[j] = sL[0][lane + 32 * j];
+        Mr[j] = gM[lane + 32 * j];
+        Ir[j] = gI[lane + 32 * j];
     }
-    for (int kb = warp; kb < nb; kb += 8) {
+    for (int b = lo + warp; b < hi; b += kMcThreads / 32) {
         float s = 0.0f;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const float2 v = part[static_cast<long long>(kb) * 128 + lane + 32 * j];
-            s += v.y * exp2f(v.x - Mr[j]) * Ir[j];
+            const float2 v = part[static_cast<long long>(b) * 128 + lane + 32 * j];
+            s += (v.x == -INFINITY) ? 0.0f : v.y * exp2f(v.x - Mr[j]) * Ir[j];
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == 0) mass[bh * nb + kb] = s * (1.0f / 128.0f);
+        if (lane == 0) mass[bh * nb + b] = s * (1.0f / 128.0f);
     }
 }
 

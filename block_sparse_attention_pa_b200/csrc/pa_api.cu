@@ -344,7 +344,7 @@ pa_status launch_mass(const pa_shape *s, const void *q, pa_strides qs, const voi
     r = d == 128 ? launch_tile_gemm_t<128, pa::MODE_MASS>(ma, mb, p, st)
                  : launch_tile_gemm_t<64, pa::MODE_MASS>(ma, mb, p, st);
     if (r) return r;
-    pa::mass_combine_kernel<<<B * H, 256, 0, st>>>(partial, mass, nb);
+    pa::mass_combine_kernel<<<B * H * pa::kMcCta, pa::kMcThreads, 0, st>>>(partial, mass, nb);
     PA_CUDA(cudaGetLastError());
     return PA_OK;
 }
