@@ -320,27 +320,49 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                             IDESC_PV, kk > 0 ? 1u : acc0);
                 umma_commit(&o_done[t]);
             };
-            auto active = [&](int t, int kb) { return (bm[t * 128 + (kb >> 5)] >> (kb & 31)) & 1u; };
+            // Visit cursor: the bitmap word holding the current block, of both
+            // heads, stays in registers, so shared memory is read once per 32
+            // blocks instead of on every step (shared-memory reads of this
+            // thread queue behind the tensor core's operand reads).
+            int cw = kb_first >> 5;
+            uint32_t w0 = bm[cw], w1 = bm[128 + cw];
+            // next visited block after kb (a block of word cw) and its per-head flags; -1 past the row
+            auto next_visit = [&](int kb, uint32_t &f0, uint32_t &f1) -> int {
+                const int sh = (kb & 31) + 1;
+                uint32_t m = sh < 32 ? (w0 | w1) & (0xFFFFFFFFu << sh) : 0u;
+                while (m == 0u) {
+                    if (++cw >= words) return -1;
+                    w0 = bm[cw];
+                    w1 = bm[128 + cw];
+                    m = w0 | w1;
+                }
+                const int bit = __ffs(static_cast<int>(m)) - 1;
+                f0 = (w0 >> bit) & 1u;
+                f1 = (w1 >> bit) & 1u;
+                return (cw << 5) + bit;
+            };
+            uint32_t c0 = (w0 >> (kb_first & 31)) & 1u, c1 = (w1 >> (kb_first & 31)) & 1u;  // heads active at kb
             int seen0 = 0, seen1 = 0;  // tiles of each head whose P was handed over
             int pv0 = 0, pv1 = 0;      // SKIP: PV products issued for each head
             bool ok = mbar_wait(q_full, 0, wc) && mbar_wait(&k_full[0], 0, wc);
             if (ok) {
                 tc_fence_after();
-                for (int t = 0; t < 2; ++t)
-                    if (active(t, kb_first)) issue_qk(t, 0);
+                if (c0) issue_qk(0, 0);
+                if (c1) issue_qk(1, 0);
                 umma_commit(&k_empty[0]);
             }
             int i = 0;
             for (int kb = kb_first; kb >= 0 && ok; ++i) {
                 const int s = i % KS;
                 const int s1 = (i + 1) % KS;
-                const int kb_next = next_block(bm, bm + 128, kb + 1, words);
+                uint32_t n0 = 0u, n1 = 0u;  // heads active at kb_next
+                const int kb_next = next_visit(kb, n0, n1);
                 const bool has_next = kb_next >= 0;
                 if (!mbar_wait(&v_full[s], (i / KS) & 1, wc)) break;
                 if (has_next && !mbar_wait(&k_full[s1], ((i + 1) / KS) & 1, wc)) break;
                 tc_fence_after();
                 for (int t = 0; t < 2; ++t) {
-                    if (active(t, kb)) {
+                    if (t ? c1 : c0) {
                         int &seen = t ? seen1 : seen0;
                         int &pv = t ? pv1 : pv0;
                         if (!mbar_wait(&p_full[t], seen & 1, wc)) { ok = false; break; }
@@ -357,12 +379,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                             ++seen;
                         }
                     }
-                    if (has_next && active(t, kb_next)) issue_qk(t, s1);
+                    if (has_next && (t ? n1 : n0)) issue_qk(t, s1);
                 }
                 if (!ok) break;
                 umma_commit(&v_empty[s]);
                 if (has_next) umma_commit(&k_empty[s1]);
                 kb = kb_next;
+                c0 = n0;
+                c1 = n1;
             }
         }
         if (lane == 0) {
@@ -452,13 +476,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             } else {
                 m = m_new;
             }
-            // P = 2^(x - m) as bf16 pairs written over the first 64 columns of S;
-            // a share of the exponentials runs on the FMA pipe (ex2_poly).
+            // P = 2^(x - m) as bf16 pairs written over the first 64 columns of S.
+            // Each column pair takes one packed FMA for x = s * scale - m and
+            // one packed add into four partial row sums; a share of the pairs
+            // of a non-diagonal tile takes its exponentials from the FMA-pipe
+            // polynomial instead of the MUFU unit.
             const float negm = (m == -INFINITY) ? 0.0f : -m;
-            const float c2 = p.scale_log2;
-            float acc[8];
+            const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
+            const float2 nm = make_float2(negm, negm);
+            float2 acc[4];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+            for (int j = 0; j < 4; ++j) acc[j] = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t pk[32];
@@ -466,32 +494,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int j = half * 32 + jj;
-                        const float e0 = ex2(fmaf(__uint_as_float(s[2 * j]), c2, negm));
-                        const float e1 = ex2(fmaf(__uint_as_float(s[2 * j + 1]), c2, negm));
-                        acc[j & 7] += e0 + e1;
-                        pk[jj] = pack_bf16x2(e0, e1);
+                        const float2 x =
+                            __ffma2_rn(make_float2(__uint_as_float(s[2 * j]), __uint_as_float(s[2 * j + 1])), c2, nm);
+                        const float2 e = make_float2(ex2(x.x), ex2(x.y));
+                        acc[j & 3] = __fadd2_rn(acc[j & 3], e);
+                        pk[jj] = pack_bf16x2(e.x, e.y);
                     }
                 } else {
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) {
                         const int j = half * 32 + jj;
-                        const float x0 = fmaf(__uint_as_float(s[2 * j]), c2, negm);
-                        const float x1 = fmaf(__uint_as_float(s[2 * j + 1]), c2, negm);
-                        float e0, e1;
-                        if ((j & 7) < kPolyPairsPer8) {
-                            e0 = ex2_poly(x0);
-                            e1 = ex2_poly(x1);
-                        } else {
-                            e0 = ex2(x0);
-                            e1 = ex2(x1);
-                        }
-                        acc[j & 7] += e0 + e1;
-                        pk[jj] = pack_bf16x2(e0, e1);
+                        const float2 x =
+                            __ffma2_rn(make_float2(__uint_as_float(s[2 * j]), __uint_as_float(s[2 * j + 1])), c2, nm);
+                        const float2 e = ((j & 7) < kPolyPairsPer8) ? ex2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
+                        acc[j & 3] = __fadd2_rn(acc[j & 3], e);
+                        pk[jj] = pack_bf16x2(e.x, e.y);
                     }
                 }
                 tmem_st32(s_addr + half * 32, pk);
             }
-            l += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+            l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&p_full[t]);
