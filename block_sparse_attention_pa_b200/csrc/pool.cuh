@@ -28,13 +28,21 @@ struct PoolParams {
     int stride;  // query-row stride r (1: every row)
 };
 
-__device__ __forceinline__ void add_bf16x8(double (&acc)[8], const uint4 &v) {
+// The 8 bf16 values of v as fp64 (exact).
+__device__ __forceinline__ void to_f64x8(double (&x)[8], const uint4 &v) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        acc[2 * i] += static_cast<double>(__uint_as_float(w[i] << 16));
-        acc[2 * i + 1] += static_cast<double>(__uint_as_float(w[i] & 0xFFFF0000u));
+        x[2 * i] = static_cast<double>(__uint_as_float(w[i] << 16));
+        x[2 * i + 1] = static_cast<double>(__uint_as_float(w[i] & 0xFFFF0000u));
     }
+}
+
+__device__ __forceinline__ void add_bf16x8(double (&acc)[8], const uint4 &v) {
+    double x[8];
+    to_f64x8(x, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] += x[j];
 }
 
 // sum / n rounded to bf16.  When n is a power of two, sum * (1/n) is exact and
@@ -78,25 +86,50 @@ __global__ void __launch_bounds__(256, 2) pool_heads_kernel(PoolParams p) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) aq[j] = ak[j] = 0.0;
 
-    // all 16-byte loads of a block of 6 heads are in flight before the first
-    // add; the adds then run in ascending head order (the oracle's order)
-    for (int t0 = 0; t0 < hpg; t0 += 6) {
-        const int n = min(6, hpg - t0);
-        uint4 qv[6], kvv[6];
+    // The k proxy adds, for every q head h of the group in ascending order, the
+    // row of its KV head v(h) = h * Hkv / H; v(h) does not decrease with h, so
+    // each KV row is converted to fp64 once and added once per q head reading
+    // it, which is the same sequence of additions.  The distinct KV rows of
+    // the group are loaded first (up to 8 per pass) and the q heads are summed
+    // while those loads are in flight.
+    const int hend = h0 + hpg;
+    const int v_lo = static_cast<int>(static_cast<int64_t>(h0) * p.Hkv / p.H);
+    const int v_hi = static_cast<int>(static_cast<int64_t>(hend - 1) * p.Hkv / p.H);
+    bool q_done = !doq;
+    for (int v0 = v_lo; v0 <= v_hi; v0 += 8) {
+        const int nv = min(8, v_hi - v0 + 1);
+        uint4 kvv[8];
 #pragma unroll
-        for (int t = 0; t < 6; ++t) {
-            if (t < n) {
-                const int h = h0 + t0 + t;
-                const int kvh = static_cast<int>(static_cast<int64_t>(h) * p.Hkv / p.H);
-                if (doq) qv[t] = __ldg(reinterpret_cast<const uint4 *>(qrow + h * p.qsh));
-                kvv[t] = __ldg(reinterpret_cast<const uint4 *>(krow + kvh * p.ksh));
+        for (int t = 0; t < 8; ++t)
+            if (t < nv) kvv[t] = __ldg(reinterpret_cast<const uint4 *>(krow + (v0 + t) * p.ksh));
+        if (!q_done) {
+            // q heads in blocks of 6: all 16-byte loads of a block in flight
+            // before the first add, the adds in ascending head order
+            for (int t0 = 0; t0 < hpg; t0 += 6) {
+                const int n = min(6, hpg - t0);
+                uint4 qv[6];
+#pragma unroll
+                for (int t = 0; t < 6; ++t)
+                    if (t < n) qv[t] = __ldg(reinterpret_cast<const uint4 *>(qrow + (h0 + t0 + t) * p.qsh));
+#pragma unroll
+                for (int t = 0; t < 6; ++t)
+                    if (t < n) add_bf16x8(aq, qv[t]);
             }
+            q_done = true;
         }
 #pragma unroll
-        for (int t = 0; t < 6; ++t) {
-            if (t < n) {
-                if (doq) add_bf16x8(aq, qv[t]);
-                add_bf16x8(ak, kvv[t]);
+        for (int t = 0; t < 8; ++t) {
+            if (t < nv) {
+                const int v = v0 + t;
+                // q heads reading KV head v: [ceil(v H / Hkv), ceil((v+1) H / Hkv)) within the group
+                const int a = max(h0, static_cast<int>((static_cast<int64_t>(v) * p.H + p.Hkv - 1) / p.Hkv));
+                const int z = min(hend, static_cast<int>((static_cast<int64_t>(v + 1) * p.H + p.Hkv - 1) / p.Hkv));
+                double x[8];
+                to_f64x8(x, kvv[t]);
+                for (int r = a; r < z; ++r) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) ak[j] += x[j];
+                }
             }
         }
     }
