@@ -71,6 +71,9 @@ def parse_args():
     ap.add_argument("--tau", type=float, default=0.9, help="XAttention find_blocks threshold")
     ap.add_argument("--skip-threshold", type=float, default=0.0,
                     help="running-max block skip in the attention: lambda in [0, 1] (0: off)")
+    ap.add_argument("--gen", choices=["literal", "logit"], default="literal",
+                    help="input generator: the workload's recipe, or the labelled extra with the direction "
+                         "weight in logit units (2 d^(1/4); per-head budgets then differ)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
@@ -515,6 +518,8 @@ def config_of(w, G, mode, gamma, frac, stride=1, skip=0.0):
 def main():
     args = parse_args()
     w = {**synth.WORKLOADS, **synth.EXTRA_WORKLOADS}[args.workload]
+    if args.gen == "logit":  # a labelled extra, named apart from the workload it modifies
+        w = w.replace(name=w.name + "_logit", logit_units=True)
     G = args.groups or w.num_groups
     mode = MODES[args.mode]
     gamma = args.gamma if args.gamma is not None else w.gamma

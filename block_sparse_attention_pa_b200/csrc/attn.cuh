@@ -5,7 +5,9 @@
 // One CTA computes one query block (128 rows) of one or two heads that share
 // a KV head.  Head t visits the first cnt_t entries of its proxy group's
 // ranked list (two heads of one group share the list); a K/V tile is loaded
-// once for both heads whenever either needs it.
+// once for both heads whenever either needs it.  The heads of a KV head are
+// paired per query block by their row counts (ranked by (cnt, head)), so the
+// two heads of a CTA share most of their tiles even when budgets differ.
 //
 // Warp roles (384 threads = three warpgroups, one CTA per SM, all 512 TMEM
 // columns).  At the start the third warpgroup hands registers to the two
@@ -59,8 +61,7 @@ constexpr int kPolyPairsPer8 = PA_POLY_PAIRS_PER8;
 
 struct AttnParams {
     int B, N, H, Hkv, G, nb;
-    int num_units;             // head units per (b, qb)
-    int units_per_kv;          // max head units of one KV head (grid stride)
+    int units_per_kv;          // max head units (CTAs) of one KV head per (b, qb): the grid stride
     const int32_t *rank;       // [B][G][T]
     const int32_t *cnt;        // [B][H][nb]
     float scale_log2;          // softmax_scale * log2(e)
@@ -71,10 +72,7 @@ struct AttnParams {
     float skip_log2;           // SKIP: log2(lambda) (lambda in (0, 1])
     uint8_t *skipped;          // SKIP: [B][H][T], 1 written for every skipped block, or nullptr
     uint64_t timeout_ns;
-    int16_t unit_h0[kMaxHeads];
-    int16_t unit_h1[kMaxHeads];  // -1: the unit has one head
-    int16_t kv_unit0[kMaxHeads];  // first unit of KV head kv (units are ordered by KV head)
-    int16_t kv_units[kMaxHeads];  // number of units of KV head kv
+    int16_t kv_units[kMaxHeads];  // head units of KV head kv: ceil(its q heads / 2)
 };
 
 // Smallest block index >= from whose bit is set in (a | b), or -1; words
@@ -178,10 +176,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int kv_of_cta = static_cast<int>(rest % p.Hkv);
     const int b = static_cast<int>(rest / p.Hkv);
     if (j >= p.kv_units[kv_of_cta]) return;  // this KV head has fewer units (whole CTA, before any sync)
-    const int unit = p.kv_unit0[kv_of_cta] + j;
-    const int h0 = p.unit_h0[unit];
-    const int h1 = p.unit_h1[unit];
-    const int kvh = static_cast<int>(static_cast<long long>(h0) * p.Hkv / p.H);
+    // The q heads of this KV head, [hk, hk + nh), are paired by their row counts
+    // for this query block: ranked by (cnt, head) and unit j takes ranks 2j and
+    // 2j+1.  Heads of one proxy group visit prefixes of the same list, so a pair
+    // with close counts shares most of its K/V tiles and both heads are busy on
+    // them.  Every CTA of (b, kv, qb) ranks the same counts the same way, so the
+    // units cover each head once.
+    const int kvh = kv_of_cta;
+    const int hk = static_cast<int>((static_cast<long long>(kvh) * p.H + p.Hkv - 1) / p.Hkv);
+    const int nh = static_cast<int>((static_cast<long long>(kvh + 1) * p.H + p.Hkv - 1) / p.Hkv) - hk;
+    __shared__ int pair_heads[2];
+    if (static_cast<int>(threadIdx.x) < nh) {
+        const int32_t *cq = p.cnt + (static_cast<long long>(b) * p.H + hk) * p.nb + qb;
+        const int me = static_cast<int>(threadIdx.x);
+        const int32_t c_me = cq[static_cast<long long>(me) * p.nb];
+        int r = 0;
+        for (int y = 0; y < nh; ++y) {
+            const int32_t c_y = cq[static_cast<long long>(y) * p.nb];
+            r += (c_y < c_me || (c_y == c_me && y < me)) ? 1 : 0;
+        }
+        if ((r >> 1) == j) pair_heads[r & 1] = hk + me;
+    }
+    if (threadIdx.x == 0 && 2 * j + 1 >= nh) pair_heads[1] = -1;  // an odd head count leaves the last unit one head
+    // The selected blocks of each head as a bitmap over 0..qb: head t takes the
+    // first c[t] entries of its list.  Every role then visits them in
+    // ascending block order (the result does not depend on the order), so the
+    // CTAs resident at one time sweep K/V in step.
+    for (int w = threadIdx.x; w < 256; w += blockDim.x) bm[w] = 0u;
+    __syncthreads();
+    // the roles below re-read the pair from shared memory where they need it
+    // (cheaper than keeping two registers live through every role)
+    const volatile int *pair = pair_heads;
+    const int h0 = pair[0];
+    const int h1 = pair[1];
     const long long T = p.causal ? static_cast<long long>(p.nb) * (p.nb + 1) / 2 : static_cast<long long>(p.nb) * p.nb;
     const long long row_off = p.causal ? static_cast<long long>(qb) * (qb + 1) / 2 : static_cast<long long>(qb) * p.nb;
     const int row_len = p.causal ? qb + 1 : p.nb;  // blocks in this query block's list
@@ -198,12 +225,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int ntiles = (h1 >= 0) ? 2 : 1;
     const int words = (row_len + 31) >> 5;  // bitmap words covering the row's blocks
 
-    // The selected blocks of each head as a bitmap over 0..qb: head t takes the
-    // first c[t] entries of its list.  Every role then visits them in
-    // ascending block order (the result does not depend on the order), so the
-    // CTAs resident at one time sweep K/V in step.
-    for (int w = threadIdx.x; w < 256; w += blockDim.x) bm[w] = 0u;
-    __syncthreads();
     for (int x = threadIdx.x; x < c[0] + c[1]; x += blockDim.x) {
         const int t = (x < c[0]) ? 0 : 1;
         const int kb = t ? list1[x - c[0]] : list0[x];
@@ -260,8 +281,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_arrive_expect_tx(q_full, ntiles * TB);
 #pragma unroll
             for (int cc = 0; cc < D / 64; ++cc) {
-                tma_load_4d(sQ + cc * 16384, &tmQ, q_full, cc * 64, h0, qb * 128, b);
-                if (h1 >= 0) tma_load_4d(sQ + TB + cc * 16384, &tmQ, q_full, cc * 64, h1, qb * 128, b);
+                tma_load_4d(sQ + cc * 16384, &tmQ, q_full, cc * 64, pair[0], qb * 128, b);
+                if (pair[1] >= 0) tma_load_4d(sQ + TB + cc * 16384, &tmQ, q_full, cc * 64, pair[1], qb * 128, b);
             }
             int issued = 0;
             int i = 0;
@@ -399,7 +420,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         reg_acquire<kRegsSoftmax>();
         // ---------------------------------------------------------- softmax
         const int t = static_cast<int>(warp >> 2);
-        const int h = t ? h1 : h0;
+        const int h = (t && pair[1] >= 0) ? pair[1] : pair[0];  // an unpaired unit's second warpgroup has no blocks
+        const long long skip_base = (static_cast<long long>(b) * p.H + h) * T + row_off;
         const uint32_t *bmt = bm + t * 128;
         const int q4 = static_cast<int>(warp & 3);
         const int row = q4 * 32 + static_cast<int>(lane);
@@ -408,7 +430,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t o_addr = lane_base + 256 + t * 128;
         float m = -INFINITY, l = 0.0f;
         float mtrue = -INFINITY;  // SKIP: exact running max (log2 units) of the tiles visited
-        const long long skip_base = (static_cast<long long>(b) * p.H + h) * T + row_off;
         bool ok = true;
         uint32_t s[128];
         int i = 0;    // tiles of this head so far

@@ -443,19 +443,19 @@ pa_status launch_xattn(const pa_shape *s, int S, float tau, const void *q, pa_st
 // Head units of the attention kernel: pairs of consecutive q heads that share
 // their KV head (so they share one K/V stream; each follows its own group's
 // ranked list); a head left over forms a unit alone.
-int build_units(const pa_shape *s, int16_t *h0, int16_t *h1) {
+// Head units of every KV head: its q heads h with h * Hkv / H == kv, two per
+// unit (the kernel pairs them by row count); returns the largest count.
+int build_units(const pa_shape *s, int16_t *kv_units) {
     const int H = s->num_q_heads, Hkv = s->num_kv_heads;
-    int n = 0;
-    int h = 0;
-    while (h < H) {
-        const int kv = static_cast<int>(static_cast<long long>(h) * Hkv / H);
-        const bool pair = h + 1 < H && static_cast<int>(static_cast<long long>(h + 1) * Hkv / H) == kv;
-        h0[n] = static_cast<int16_t>(h);
-        h1[n] = static_cast<int16_t>(pair ? h + 1 : -1);
-        ++n;
-        h += pair ? 2 : 1;
+    int most = 0;
+    for (int kv = 0; kv < Hkv; ++kv) {
+        const long long first = (static_cast<long long>(kv) * H + Hkv - 1) / Hkv;
+        const long long next = (static_cast<long long>(kv + 1) * H + Hkv - 1) / Hkv;
+        const int units = static_cast<int>((next - first + 1) / 2);
+        kv_units[kv] = static_cast<int16_t>(units);
+        most = std::max(most, units);
     }
-    return n;
+    return most;
 }
 
 template <int D, bool SKIP>
@@ -489,16 +489,7 @@ pa_status launch_attn(const pa_shape *s, const void *q, pa_strides qs, const voi
     if ((r = map_bnhd(&mv, v, B, N, Hkv, d, vs, "v"))) return r;
     pa::AttnParams p{};
     p.B = B; p.N = N; p.H = H; p.Hkv = Hkv; p.G = s->num_groups; p.nb = N / kBlk;
-    p.num_units = build_units(s, p.unit_h0, p.unit_h1);
-    // units are produced in ascending head order, hence grouped by KV head
-    for (int kv = 0; kv < Hkv; ++kv) p.kv_units[kv] = 0;
-    for (int u = 0; u < p.num_units; ++u) {
-        const int kv = static_cast<int>(static_cast<long long>(p.unit_h0[u]) * Hkv / H);
-        if (p.kv_units[kv] == 0) p.kv_unit0[kv] = static_cast<int16_t>(u);
-        ++p.kv_units[kv];
-    }
-    p.units_per_kv = 0;
-    for (int kv = 0; kv < Hkv; ++kv) p.units_per_kv = std::max<int>(p.units_per_kv, p.kv_units[kv]);
+    p.units_per_kv = build_units(s, p.kv_units);
     p.rank = rank; p.cnt = cnt;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.o = static_cast<__nv_bfloat16 *>(o);

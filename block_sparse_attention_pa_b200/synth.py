@@ -17,6 +17,12 @@ workloads on the ProxyAttn pages, "5. Experiments"; there is no dataset here):
 * ``n_needles`` positions are drawn without replacement from ``[1, N)`` and
   ``K[:, pos, kvh] += 2.0 * u_{dir(kvh)}`` for every KV head.
 * ``K[:, 0] *= 4`` (an attention sink).
+* Optional, a labelled extra that never replaces a workload below
+  (``logit_units``): the direction weight 2.0 on Q and on the needles becomes
+  ``w = 2 d^(1/4)``, so a needle lifts the scaled logit of head h by
+  ``w^2 s_h / sqrt(d) = 4 s_h`` instead of ``4 s_h / sqrt(d)`` (about 0.35 s_h
+  at d = 128).  Attention is then concentrated enough that the per-head
+  dynamic budgets differ.
 * Optional, for the running-max block skip only (``sink_logit`` > 0, a
   labelled extra, never one of the five workloads below): ``K[:, 0, kvh] +=
   (sink_logit * sqrt(d) / 2) * u_{dir(kvh)}``, which lifts the sink's scaled
@@ -49,6 +55,7 @@ class Workload:
     per_group_direction: bool
     seed: int
     sink_logit: float = 0.0
+    logit_units: bool = False
 
     @property
     def nb(self) -> int:
@@ -97,11 +104,12 @@ def make_inputs(w: Workload, device="cpu", seed: int | None = None):
     # direction index of each q head / kv head (GQA group = q heads of one kv head)
     q_dir = (torch.arange(H, device=dev) * Hkv // H) if n_dirs > 1 else torch.zeros(H, dtype=torch.long, device=dev)
     kv_dir = torch.arange(Hkv, device=dev) if n_dirs > 1 else torch.zeros(Hkv, dtype=torch.long, device=dev)
-    q += (2.0 * s[:, None] * u[q_dir])[None, None]
+    wu = 2.0 * d ** 0.25 if w.logit_units else 2.0  # direction weight
+    q += (wu * s[:, None] * u[q_dir])[None, None]
     n_needles = min(w.n_needles, max(N - 1, 0))
     if n_needles > 0:
         needles = torch.randperm(N - 1, generator=g, device=dev)[:n_needles] + 1
-        k[:, needles] += (2.0 * u[kv_dir])[None, None]
+        k[:, needles] += (wu * u[kv_dir])[None, None]
     else:
         needles = torch.zeros(0, dtype=torch.long, device=dev)
     k[:, 0] *= 4.0
@@ -117,8 +125,9 @@ def make_inputs(w: Workload, device="cpu", seed: int | None = None):
 
 
 def small_workload(seqlen=512, heads=4, kv_heads=2, head_dim=64, groups=1, gamma=0.9,
-                   needles=8, batch=1, seed=7, sharp=True, per_group=False, sink_logit=0.0) -> Workload:
+                   needles=8, batch=1, seed=7, sharp=True, per_group=False, sink_logit=0.0,
+                   logit_units=False) -> Workload:
     """A small custom workload for parity tests (sizes the oracle finishes in seconds)."""
     return Workload(f"custom_n{seqlen}_h{heads}_kv{kv_heads}_d{head_dim}_g{groups}",
                     batch, seqlen, heads, kv_heads, head_dim, groups, gamma, needles,
-                    sharp, per_group, seed, sink_logit)
+                    sharp, per_group, seed, sink_logit, logit_units)

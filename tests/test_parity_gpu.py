@@ -79,11 +79,32 @@ CASES = [
 ]
 
 
+# The labelled extra generator with the direction weight in logit units: the
+# per-head dynamic budgets differ, so the two heads of a CTA keep different
+# prefixes of their list on most query blocks.
+LOGIT_CASES = [
+    # name,               N,    H, Hkv, d,  G, mode,        gamma, frac, B
+    ("logit_gqa_d128",    2048, 8, 2, 128, 1, pa.DYNAMIC,   0.95, 0,   1),
+    ("logit_g2_d64",      1536, 6, 2,  64, 2, pa.DYNAMIC,   0.9,  0,   1),
+]
+
+
 @pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
 def test_stage_parity(case):
+    check_case(case, seed=100 + CASES.index(case), needles=8)
+
+
+@pytest.mark.parametrize("case", LOGIT_CASES, ids=[c[0] for c in LOGIT_CASES])
+def test_stage_parity_logit_units(case):
+    cnt = check_case(case, seed=300 + LOGIT_CASES.index(case), needles=24, logit_units=True)
+    # the budgets really differ between the heads that share a CTA
+    assert (cnt[:, 0::2] != cnt[:, 1::2]).any()
+
+
+def check_case(case, seed, needles, logit_units=False):
     name, N, H, Hkv, d, G, mode, gamma, frac, B = case
     w = synth.small_workload(seqlen=N, heads=H, kv_heads=Hkv, head_dim=d, groups=G, gamma=gamma, batch=B,
-                             needles=8, seed=100 + CASES.index(case))
+                             needles=needles, seed=seed, logit_units=logit_units)
     x = synth.make_inputs(w)
     qc, kc, vc = x["q"], x["k"], x["v"]
     q, k, v = qc.cuda(), kc.cuda(), vc.cuda()
@@ -123,6 +144,7 @@ def test_stage_parity(case):
     lgi = np.stack([lg[b, h, qb * 128:(qb + 1) * 128] for (b, h, qb) in items])
     compare_o(ogi, oref)
     assert np.abs(lgi - lref).max() < 1e-3
+    return mask.cnt.cpu().numpy()
 
 
 def test_prefill_equals_stages_and_dense_all():
