@@ -11,8 +11,9 @@ Acceptance:
                    estimates (ties to the lower index)
   O                max-abs <= 2e-2, mean-abs <= 2e-3 against o5 with the
                    GPU's lists (one list per head: num_groups = num_q_heads)
-Cases span several 128-row x 256-column output tiles, ragged last tiles
-(N/S not a multiple of 128), S = 4, 8, 16, d = 64 and 128, GQA, batch 2.
+Cases span several output tiles, ragged last tiles (N/S not a multiple of
+128), S = 4, 8, 16, d = 64 and 128, GQA, batch 2, block counts that do and do
+not allow 16-byte stores of the partial sums, and both estimate GEMMs.
 """
 import numpy as np
 import pytest
@@ -43,8 +44,12 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("pair", [False, True], ids=["one_sm", "sm_pair"])
 @pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
-def test_xattn_parity(case):
+def test_xattn_parity(case, pair, monkeypatch):
+    """Both estimate GEMMs: one SM per 128 x 256 tile, and the SM-pair kernel
+    (PA_XATTN_PAIR=1, 256 x 256 tiles on two SMs)."""
+    monkeypatch.setenv("PA_XATTN_PAIR", "1" if pair else "0")
     name, N, H, Hkv, d, S, tau, B = case
     w = synth.small_workload(seqlen=N, heads=H, kv_heads=Hkv, head_dim=d, groups=H, batch=B, needles=8,
                              seed=700 + CASES.index(case))
