@@ -589,8 +589,76 @@ __device__ __forceinline__ float xsel_key_value(uint32_t key) {
     return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord);
 }
 
+// Ascending bitonic sort of the 256*E keys in shared memory by a CTA of 256
+// threads.  Thread t holds keys t*E .. t*E+E-1 in registers: a compare-exchange
+// stage whose partner index differs by j < E stays in the thread, one with
+// E <= j < 32E is a warp shuffle, and only the stages with j >= 32E go through
+// shared memory (6 of the 55 stages for 1024 keys).  The result is the unique
+// ascending order of the keys (they are distinct), back in shared memory.
+// the in-thread stage with partner distance J < E (J a compile-time constant,
+// so the key array stays in registers)
+template <int E, int J>
+__device__ __forceinline__ void bitonic_stage_in_thread(unsigned long long (&v)[E], int k, int tid) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        if ((e & J) == 0) {
+            const int i = tid * E + e;
+            const unsigned long long a = v[e], c = v[e ^ J];
+            if ((a > c) == ((i & k) == 0)) {
+                v[e] = c;
+                v[e ^ J] = a;
+            }
+        }
+    }
+}
+
+template <int E>
+__device__ __forceinline__ void bitonic_sort_256(unsigned long long *keys) {
+    constexpr int PP = 256 * E;
+    const int tid = static_cast<int>(threadIdx.x);
+    unsigned long long v[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) v[e] = keys[tid * E + e];
+    for (int k = 2; k <= PP; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            if (j >= 32 * E) {
+                __syncthreads();  // every thread has read the previous stage's keys
+#pragma unroll
+                for (int e = 0; e < E; ++e) keys[tid * E + e] = v[e];
+                __syncthreads();
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const int i = tid * E + e, l = i ^ j;
+                    const unsigned long long w = keys[l];
+                    const bool keep_min = (i < l) == ((i & k) == 0);
+                    v[e] = keep_min ? (v[e] < w ? v[e] : w) : (v[e] < w ? w : v[e]);
+                }
+            } else if (j >= E) {
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const int i = tid * E + e, l = i ^ j;
+                    const unsigned long long w = __shfl_xor_sync(0xffffffffu, v[e], j / E);
+                    const bool keep_min = (i < l) == ((i & k) == 0);
+                    v[e] = keep_min ? (v[e] < w ? v[e] : w) : (v[e] < w ? w : v[e]);
+                }
+            } else if (j == 4) {
+                if constexpr (E > 4) bitonic_stage_in_thread<E, 4>(v, k, tid);
+            } else if (j == 2) {
+                if constexpr (E > 2) bitonic_stage_in_thread<E, 2>(v, k, tid);
+            } else {
+                if constexpr (E > 1) bitonic_stage_in_thread<E, 1>(v, k, tid);
+            }
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < E; ++e) keys[tid * E + e] = v[e];
+    __syncthreads();
+}
+
 // One CTA of 256 threads per (b, h, qb), long rows first; dynamic shared
-// memory holds P >= qb+1 (a power of two) 64-bit sort keys.
+// memory holds max(P, 256) 64-bit sort keys, P >= qb+1 a power of two.
+template <int S>
 __global__ void __launch_bounds__(256) xattn_select_kernel(XselParams p) {
     extern __shared__ unsigned long long keys[];
     __shared__ float red[256];
@@ -600,7 +668,8 @@ __global__ void __launch_bounds__(256) xattn_select_kernel(XselParams p) {
     const long long bh = blockIdx.x / p.nb;
     const int qb = p.nb - 1 - static_cast<int>(blockIdx.x % p.nb);
     const int tid = threadIdx.x;
-    const int CPB = 128 / p.S;          // strided rows of the query block (<= 32)
+    constexpr int CPB = 128 / S;        // strided rows of the query block (<= 32); compile-time, so
+                                        // the loops over them unroll and their loads overlap
     const int R0 = qb * CPB;
     const int cq = p.causal ? R0 / 128 : p.nchunk - 1;  // the rows' last 128-column chunk
     const int n = p.causal ? qb + 1 : p.nb;              // blocks of the row
@@ -612,9 +681,10 @@ __global__ void __launch_bounds__(256) xattn_select_kernel(XselParams p) {
     const long long rs = p.rows;
 
     // 1. each strided row's max over its chunks (slots threads per row)
-    const int slots = 256 / CPB;
+    constexpr int slots = 256 / CPB;
     const int r = tid / slots, sl = tid % slots;
     float M = -INFINITY;
+#pragma unroll 4
     for (int ch = sl; ch <= cq; ch += slots) M = fmaxf(M, pm[ch * rs + r]);
     red[tid] = M;
     __syncthreads();
@@ -629,7 +699,8 @@ __global__ void __launch_bounds__(256) xattn_select_kernel(XselParams p) {
     const float Mr = rowM[r];
     const float *psr = ps + static_cast<long long>(r) * p.nb;
     float L = 0.0f;
-    for (int kb = sl; kb < n; kb += slots) L += exp2f(pm[(kb / p.S) * rs + r] - Mr) * psr[kb];
+#pragma unroll 4
+    for (int kb = sl; kb < n; kb += slots) L += exp2f(pm[(kb / S) * rs + r] - Mr) * psr[kb];
     red[tid] = L;
     __syncthreads();
     if (tid < CPB) {
@@ -638,14 +709,15 @@ __global__ void __launch_bounds__(256) xattn_select_kernel(XselParams p) {
         rowI[tid] = 1.0f / l;
     }
     __syncthreads();
-    // 3. block estimates -> sort keys
-    int P = 1;
+    // 3. block estimates -> sort keys (padded with the largest key to at least 256)
+    int P = 256;
     while (P < n) P <<= 1;
     for (int kb = tid; kb < P; kb += blockDim.x) {
         unsigned long long key = ~0ull;
         if (kb < n) {
             float e = 0.0f;
-            const float *mcol = pm + (kb / p.S) * rs;
+            const float *mcol = pm + (kb / S) * rs;
+#pragma unroll
             for (int x = 0; x < CPB; ++x)
                 e += exp2f(mcol[x] - rowM[x]) * ps[static_cast<long long>(x) * p.nb + kb] * rowI[x];
             e *= 1.0f / static_cast<float>(CPB);
@@ -660,19 +732,29 @@ __global__ void __launch_bounds__(256) xattn_select_kernel(XselParams p) {
     }
     if (tid == 0) kmin = n;
     __syncthreads();
-    for (int k = 2; k <= P; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int i = tid; i < P; i += blockDim.x) {
-                const int ixj = i ^ j;
-                if (ixj > i) {
-                    const unsigned long long a = keys[i], c = keys[ixj];
-                    if ((a > c) == ((i & k) == 0)) {
-                        keys[i] = c;
-                        keys[ixj] = a;
+    if (P == 256) {
+        bitonic_sort_256<1>(keys);
+    } else if (P == 512) {
+        bitonic_sort_256<2>(keys);
+    } else if (P == 1024) {
+        bitonic_sort_256<4>(keys);
+    } else if (P == 2048) {
+        bitonic_sort_256<8>(keys);
+    } else {
+        for (int k = 2; k <= P; k <<= 1) {
+            for (int j = k >> 1; j > 0; j >>= 1) {
+                for (int i = tid; i < P; i += blockDim.x) {
+                    const int ixj = i ^ j;
+                    if (ixj > i) {
+                        const unsigned long long a = keys[i], c = keys[ixj];
+                        if ((a > c) == ((i & k) == 0)) {
+                            keys[i] = c;
+                            keys[ixj] = a;
+                        }
                     }
                 }
+                __syncthreads();
             }
-            __syncthreads();
         }
     }
     // 4. ranked list and the shortest prefix reaching tau (2^-40 fixed point)
