@@ -463,7 +463,7 @@ pa_status launch_xattn(const pa_shape *s, int S, float tau, const void *q, pa_st
         r = d == 128 ? launch_xattn_gemm_d<128>(S, mq, mk, p, st) : launch_xattn_gemm_d<64>(S, mq, mk, p, st);
     if (r) return r;
     pa::XselParams sp{};
-    sp.B = B; sp.H = H; sp.nb = nb; sp.rows = rows; sp.nchunk = p.nchunk; sp.S = S;
+    sp.B = B; sp.H = H; sp.nb = nb; sp.rows = rows; sp.nchunk = p.nchunk;
     sp.causal = p.causal;
     sp.tau = tau;
     sp.part_s = p.part_s;

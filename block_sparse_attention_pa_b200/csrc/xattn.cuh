@@ -568,7 +568,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
 
 // ------------------------------------------------------------ selection
 struct XselParams {
-    int B, H, nb, rows, nchunk, S;
+    int B, H, nb, rows, nchunk;  // the stride S is the kernel's template argument
     int causal;
     float tau;
     const float *part_s;  // as XattnParams

@@ -37,6 +37,15 @@
  *   independent except for the shared device status word.
  * Supported.  block = 128, d in {64, 128}, N % 128 == 0, 1 <= N/128 <= 4096,
  *   H % Hkv == 0, H % G == 0, H <= 128, B >= 1.  Others: PA_ERR_UNSUPPORTED.
+ * Environment.
+ *   PA_WAIT_TIMEOUT_MS  bound, in ms, of every wait inside the kernels
+ *                       (default 2000; read once, at the first launch); a
+ *                       wait that runs out records PA_ERR_TIMEOUT and the
+ *                       kernel abandons its work.
+ *   PA_XATTN_PAIR=1     (read at every call) pa_xattn_mask runs its estimate
+ *                       GEMM on SM pairs (two-CTA clusters, 256x256 tiles);
+ *                       the results are the same as with the default one-SM
+ *                       kernel.
  */
 #ifndef PA_H
 #define PA_H
