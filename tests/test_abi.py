@@ -73,6 +73,10 @@ def test_workspace_size_formula(L):
     (dict(N=128 * 4097), 2),    # too long
     (dict(H=0), 1),             # non-positive
     (dict(B=0), 1),
+    (dict(N=0), 1),             # empty sequence
+    (dict(N=-128), 1),
+    (dict(Hkv=0), 1),
+    (dict(G=0), 1),
 ])
 def test_bad_shapes_rejected_before_launch(L, bad, code):
     s = shape(**bad)
