@@ -283,7 +283,7 @@ PA_API pa_status pa_block_sparse_attn_skip(const pa_shape *shape,
  *   z[R][c] = sum_{t<S} q[R*S + S-1-t] . k[c*S + t] / (sqrt(d) * S)
  * for strided rows R and columns c (the antidiagonal sum of each S x S
  * sub-block of the score map); each row R is softmax-normalised over c <= R
- * (the causal mask at the sub-block level, a reading: the box shows none);
+ * (the causal mask at the sub-block level, a reading: the algorithm shows none);
  *   mass[b][h][tri(qb)+kb] = (S/128) * sum over the 128/S rows R of block qb
  *                            of the probability in block kb's 128/S columns;
  *   rank[b][h][tri(qb) ..]  = blocks 0..qb by (mass desc, lower index first);

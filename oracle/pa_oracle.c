@@ -521,14 +521,15 @@ void pa_oracle_sparse_attn_skip(int N, int H, int Hkv, int d, int G,
 
 /* --------------------------------------- o8 XAttention antidiagonal estimate */
 /* XAttention blog, 2.1 "importance prediction" and 2.2 "threshold block
- * selection" (its block-selection algorithm box).  For head h, query block qb
+ * selection" (its block-selection algorithm).  For head h, query block qb
  * and stride S (S divides 128): every S x S sub-block of the token-level score
  * map is scored by the sum along its antidiagonal, i.e. strided row
  * R = qb*128/S + r (tokens R*S .. R*S+S-1) against strided column c (tokens
  * c*S .. c*S+S-1) scores
  *     z[R][c] = sum_{t<S} q[R*S + S-1-t] . k[c*S + t] / (sqrt(d) * S),
- * the box's reshaped product (query rows taken from S-1 down to 0, key rows
- * from 0 up).  Readings where the box is silent: the causal mask applies at the
+ * the reshaped product of that algorithm (query rows taken from S-1 down to
+ * 0, key rows from 0 up).  Readings where the algorithm is silent: the causal
+ * mask applies at the
  * strided level (c <= R: sub-blocks on or below the diagonal; non-causal: every
  * column, the pages' video-generation use); each strided row
  * is softmax-normalised over its valid columns; the estimate of block kb is the
