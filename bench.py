@@ -515,11 +515,18 @@ def config_of(w, G, mode, gamma, frac, stride=1, skip=0.0):
 
 
 # ------------------------------------------------------------------- main
+def resolve_workload(args) -> synth.Workload:
+    """The workload the flags name; --gen logit is a labelled extra, named
+    apart from the workload it modifies."""
+    w = {**synth.WORKLOADS, **synth.EXTRA_WORKLOADS}[args.workload]
+    if args.gen == "logit":
+        w = w.replace(name=w.name + "_logit", logit_units=True)
+    return w
+
+
 def main():
     args = parse_args()
-    w = {**synth.WORKLOADS, **synth.EXTRA_WORKLOADS}[args.workload]
-    if args.gen == "logit":  # a labelled extra, named apart from the workload it modifies
-        w = w.replace(name=w.name + "_logit", logit_units=True)
+    w = resolve_workload(args)
     G = args.groups or w.num_groups
     mode = MODES[args.mode]
     gamma = args.gamma if args.gamma is not None else w.gamma

@@ -84,3 +84,17 @@ def test_selected_blocks_matches_loops():
                 for kb in rank[b, g, s:s + cnt[b, h, qb]]:
                     ref[b, h, s + kb] = True
     assert np.array_equal(got, ref)
+
+
+def test_gen_logit_is_a_labelled_extra(monkeypatch):
+    """--gen logit keeps the workload's shape but switches the generator to the
+    logit-unit recipe and renames the workload, so a bench line can never be
+    mistaken for the literal configuration."""
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--workload", "llama8b_n32k", "--gen", "logit"])
+    w = bench.resolve_workload(bench.parse_args())
+    base = bench.synth.WORKLOADS["llama8b_n32k"]
+    assert w.logit_units and w.name == "llama8b_n32k_logit"
+    assert (w.seqlen, w.num_q_heads, w.num_kv_heads, w.head_dim, w.gamma) == \
+        (base.seqlen, base.num_q_heads, base.num_kv_heads, base.head_dim, base.gamma)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--workload", "llama8b_n32k"])
+    assert bench.resolve_workload(bench.parse_args()) == base
