@@ -824,3 +824,44 @@ def test_noncausal_scores_mass_rank_budget():
         assert list(cnt[0, h]) == [max(kh, 1)] + [max(kh, 2)] * (nb - 1)
     _, cf = oracle.budget(r, None, 3, 3, nb, oracle.FIXED_FRACTION, 0, 300, causal=False)
     assert (cf == 2).all()  # ceil(0.3 * 4) = 2
+
+
+def _post_softmax_block_max(qp, kp, scale):
+    """The reading the oracle does not take: a per-row causal softmax of the
+    proxy logits before the 128 x 128 max-pool (numpy, fp64)."""
+    N = qp.shape[0]
+    z = scale * (qp @ kp.T)
+    z[np.triu_indices(N, 1)] = -np.inf
+    p = np.exp(z - z.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    nb = N // 128
+    return np.array([p[qb * 128:(qb + 1) * 128, kb * 128:(kb + 1) * 128].max()
+                     for qb in range(nb) for kb in range(qb + 1)])
+
+
+def test_rank_invariant_under_positive_scale():
+    """Proxy scores are pre-softmax scaled logits, so any positive factor on
+    them (a different softmax scale, or pooling by sum instead of mean) scales
+    every block maximum by that factor and leaves the ranked lists unchanged.
+    Powers of two keep the scaling exact, so lists must match entry for entry.
+    The same change of scale reorders the lists of the post-softmax reading,
+    which is what makes the test able to tell the two readings apart."""
+    w = synth.small_workload(seqlen=1024, heads=4, kv_heads=2, head_dim=64, needles=8, seed=17)
+    x = synth.make_inputs(w)
+    _, _, qpb, kpb = oracle.pool(x["q"], x["k"], 1)
+    nb = 8
+    base = oracle.block_scores(qpb, kpb)
+    ranked = oracle.rank(base, nb)
+    for c in (2.0 ** -7, 2.0 ** -3, 2.0 ** 4):
+        sc = oracle.block_scores(qpb, kpb, scale=c)
+        np.testing.assert_array_equal(sc, base * (c * 8.0))
+        np.testing.assert_array_equal(oracle.rank(sc, nb), ranked)
+    # group sum instead of group mean (4 heads: a factor of 4 on both proxies)
+    sc = oracle.block_scores((qpb.float() * 4).bfloat16(), (kpb.float() * 4).bfloat16())
+    np.testing.assert_array_equal(oracle.rank(sc, nb), ranked)
+    # the post-softmax reading is not invariant on the same input
+    q0 = qpb[0, 0].double().numpy()
+    k0 = kpb[0, 0].double().numpy()
+    lists = [oracle.rank(_post_softmax_block_max(q0, k0, c)[None, None], nb)
+             for c in (2.0 ** -7, 1 / 8.0, 2.0 ** 4)]
+    assert any(not np.array_equal(lists[0], l) for l in lists[1:])
