@@ -474,9 +474,10 @@ pa_status launch_xattn(const pa_shape *s, int S, float tau, const void *q, pa_st
     int P = 256;  // the selection sorts at least 256 keys
     while (P < nb) P <<= 1;
     auto sel = S == 4 ? pa::xattn_select_kernel<4> : S == 8 ? pa::xattn_select_kernel<8> : pa::xattn_select_kernel<16>;
-    PA_CUDA(cudaFuncSetAttribute(sel, cudaFuncAttributeMaxDynamicSharedMemorySize, P * 8));
+    const int smem = P * 8 + static_cast<int>((pa::xsel_sort_temp_bytes(P) + 15) / 16 * 16);
+    PA_CUDA(cudaFuncSetAttribute(sel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     const long long grid = static_cast<long long>(B) * H * nb;
-    sel<<<static_cast<unsigned>(grid), 256, P * 8, st>>>(sp);
+    sel<<<static_cast<unsigned>(grid), 256, smem, st>>>(sp);
     PA_CUDA(cudaGetLastError());
     return PA_OK;
 }

@@ -25,6 +25,8 @@
 //                       shortest prefix whose estimates reach tau in 2^-40
 //                       fixed point (find_blocks).
 #pragma once
+#include <cub/block/block_radix_sort.cuh>
+
 #include "sm100.cuh"
 
 namespace pa {
@@ -656,8 +658,45 @@ __device__ __forceinline__ void bitonic_sort_256(unsigned long long *keys) {
     __syncthreads();
 }
 
+// The sort of 1024 or 2048 keys: a stable LSD radix sort (CUB's
+// BlockRadixSort, 4-bit digits) of the upper 32 bits, the descending-estimate
+// code, with the lower 32 bits, the block index, carried along as values.
+// Thread t hands in entries t*E .. t*E+E-1, i.e. the keys in block-index
+// order, and gets back the same positions of the sorted sequence.  A stable
+// sort leaves equal estimates in index order, so the result is the ascending
+// order of the whole 64-bit keys, as the bitonic network produces.  Shorter
+// rows keep the bitonic network, which is faster there (eight radix passes
+// with block-wide scans cost more than the shuffle stages for 256 keys).
+template <int E>
+using XselRadixSort = cub::BlockRadixSort<uint32_t, 256, E, uint32_t>;
+
+// Shared memory the selection kernel needs beyond its P keys for the sort.
+__host__ __device__ constexpr size_t xsel_sort_temp_bytes(int P) {
+    return P == 1024   ? sizeof(typename XselRadixSort<4>::TempStorage)
+           : P == 2048 ? sizeof(typename XselRadixSort<8>::TempStorage)
+                       : 0;
+}
+
+template <int E>
+__device__ __forceinline__ void radix_sort_keys(unsigned long long *keys, void *temp) {
+    const int tid = static_cast<int>(threadIdx.x);
+    uint32_t k[E], v[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const unsigned long long x = keys[tid * E + e];
+        k[e] = static_cast<uint32_t>(x >> 32);
+        v[e] = static_cast<uint32_t>(x);
+    }
+    XselRadixSort<E>(*reinterpret_cast<typename XselRadixSort<E>::TempStorage *>(temp)).Sort(k, v);
+    __syncthreads();  // every thread's reads of the keys are done
+#pragma unroll
+    for (int e = 0; e < E; ++e) keys[tid * E + e] = (static_cast<unsigned long long>(k[e]) << 32) | v[e];
+    __syncthreads();
+}
+
 // One CTA of 256 threads per (b, h, qb), long rows first; dynamic shared
-// memory holds max(P, 256) 64-bit sort keys, P >= qb+1 a power of two.
+// memory holds max(P, 256) 64-bit sort keys, P >= qb+1 a power of two,
+// followed (P = 1024, 2048) by the radix sort's temporary storage.
 template <int S>
 __global__ void __launch_bounds__(256) xattn_select_kernel(XselParams p) {
     extern __shared__ unsigned long long keys[];
@@ -737,9 +776,9 @@ __global__ void __launch_bounds__(256) xattn_select_kernel(XselParams p) {
     } else if (P == 512) {
         bitonic_sort_256<2>(keys);
     } else if (P == 1024) {
-        bitonic_sort_256<4>(keys);
+        radix_sort_keys<4>(keys, keys + P);
     } else if (P == 2048) {
-        bitonic_sort_256<8>(keys);
+        radix_sort_keys<8>(keys, keys + P);
     } else {
         for (int k = 2; k <= P; k <<= 1) {
             for (int j = k >> 1; j > 0; j >>= 1) {

@@ -143,3 +143,26 @@ def test_xattn_full_size_sampled():
         sl = slice(qb * (qb + 1) // 2, qb * (qb + 1) // 2 + qb + 1)
         got = mg[:, heads, sl].astype(np.float64)
         assert np.all(np.abs(got - ref[:, :, sl]) <= 2e-5 + 2e-3 * ref[:, :, sl])
+
+
+@pytest.mark.parametrize("causal", [True, False], ids=["causal", "noncausal"])
+def test_xattn_long_rows_lists_exact(causal):
+    """Rows of up to 1536 blocks (N = 196608): the selection sorts 256, 512,
+    1024 and 2048 keys in one launch (causal), or 2048 in every row
+    (non-causal).  Lists and counts are complete and bit-exact with the
+    oracle's find_blocks fed the GPU's estimates; every row's estimates sum
+    to one."""
+    w = synth.small_workload(seqlen=196608, heads=2, kv_heads=1, head_dim=64, needles=64, seed=41)
+    x = synth.make_inputs(w, device="cuda")
+    nb = w.seqlen // 128
+    rank, cnt, mass = pa.xattn_mask(x["q"], x["k"], 16, 0.9, causal=causal)
+    torch.cuda.synchronize()
+    assert pa.device_status() == 0
+    mg = mass.cpu().numpy()
+    rank_ref, cnt_ref = oracle.find_blocks(mg, nb, float(np.float32(0.9)), causal=causal)
+    assert np.array_equal(cnt.cpu().numpy(), cnt_ref)
+    assert np.array_equal(rank.cpu().numpy(), rank_ref)
+    for qb in (0, 300, 700, nb - 1):
+        lo = qb * (qb + 1) // 2 if causal else qb * nb
+        row = mg[:, :, lo:lo + (qb + 1 if causal else nb)].astype(np.float64)
+        assert np.all(np.abs(row.sum(axis=-1) - 1.0) < 1e-4)
