@@ -98,3 +98,23 @@ def test_gen_logit_is_a_labelled_extra(monkeypatch):
         (base.seqlen, base.num_q_heads, base.num_kv_heads, base.head_dim, base.gamma)
     monkeypatch.setattr(sys, "argv", ["bench.py", "--workload", "llama8b_n32k"])
     assert bench.resolve_workload(bench.parse_args()) == base
+
+
+def test_traffic_only_for_the_profiled_kernel_and_workload():
+    """roofline.traffic comes from the committed ncu counters only while the
+    attention sources hash to what was profiled, and only for the exact
+    workload and budget of the capture; anything else reports null."""
+    ctr = bench.counters_for("attn_kernel", bench.ATTN_SOURCES)
+    assert ctr is not None, "profiles/counters.json no longer matches the attention sources"
+    w = bench.synth.WORKLOADS[ctr["workload"]]
+    mode = {"dynamic": 0, "fixed": 1, "all": 2}[ctr["mode"]]
+    got = bench.traffic_for(ctr, w, ctr["groups"], mode, ctr.get("gamma", 0.95))
+    assert got == float(ctr["dram_bytes"]) == float(ctr["dram_bytes_read"] + ctr["dram_bytes_write"])
+    assert bench.traffic_for(ctr, w, ctr["groups"] + 3, mode, ctr.get("gamma", 0.95)) is None
+    assert bench.traffic_for(ctr, w, ctr["groups"], mode, 0.5) is None
+    other = bench.synth.WORKLOADS["llama8b_n32k"]
+    assert bench.traffic_for(ctr, other, ctr["groups"], mode, ctr.get("gamma", 0.95)) is None
+    assert bench.traffic_for(ctr, w, ctr["groups"], mode, ctr.get("gamma", 0.95), stride=4) is None
+    # a changed kernel source invalidates the counters
+    assert bench.counters_for("attn_kernel", bench.ATTN_SOURCES[:1]) is None
+    assert bench.traffic_for(None, w, ctr["groups"], mode, 0.95) is None
