@@ -21,8 +21,10 @@ def _worker(rank, world, port, out):
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         t = bench.max_over_ranks(10.0 + 5.0 * rank, torch.device("cpu"))
+        # one rank's rejected clock record makes every rank measure again
+        again = bench.agree_any(rank == 1, torch.device("cpu"), True)
         dist.barrier()
-        out[rank] = t
+        out[rank] = (t, again)
     finally:
         dist.destroy_process_group()
 
@@ -32,7 +34,7 @@ def test_max_over_ranks_gloo_world2():
     with mp.Manager() as m:
         out = m.dict()
         mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
-        assert out[0] == out[1] == 15.0
+        assert out[0] == out[1] == (15.0, True)
 
 
 def test_single_process_and_per_layer():
@@ -118,3 +120,16 @@ def test_traffic_only_for_the_profiled_kernel_and_workload():
     # a changed kernel source invalidates the counters
     assert bench.counters_for("attn_kernel", bench.ATTN_SOURCES[:1]) is None
     assert bench.traffic_for(None, w, ctr["groups"], mode, 0.95) is None
+
+
+def test_clock_records_that_force_a_second_measurement():
+    ok = {"sm_mhz": 1695.0, "sm_max_mhz": 1965.0, "samples": 20, "reasons": ["sw_power_cap"]}
+    assert not bench.clocks_rejected(ok)
+    assert not bench.clocks_rejected(None)
+    for r in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"):
+        assert bench.clocks_rejected(dict(ok, reasons=["sw_power_cap", r]))
+    # a clock held low with no power-cap reason reads as a leftover lock
+    assert bench.clocks_rejected(dict(ok, sm_mhz=1200.0, reasons=[]))
+    assert not bench.clocks_rejected(dict(ok, sm_mhz=1200.0))
+    assert not bench.clocks_rejected(dict(ok, sm_mhz=1900.0, reasons=[]))
+    assert bench.agree_any(True, "cpu", False) and not bench.agree_any(False, "cpu", False)
