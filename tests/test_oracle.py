@@ -865,3 +865,30 @@ def test_rank_invariant_under_positive_scale():
     lists = [oracle.rank(_post_softmax_block_max(q0, k0, c)[None, None], nb)
              for c in (2.0 ** -7, 1 / 8.0, 2.0 ** 4)]
     assert any(not np.array_equal(lists[0], l) for l in lists[1:])
+
+
+@pytest.mark.parametrize("S", [2, 4])
+@pytest.mark.parametrize("causal", [True, False])
+def test_xattn_mass_uniform_closed_form(S, causal):
+    """With every query zero all antidiagonal sums are 0, so each strided row's
+    softmax is uniform over its valid strided columns (c <= R when causal, all
+    N/S otherwise).  Block kb's estimate for query block qb is then the mean
+    over qb's 128/S strided rows R of (valid columns of kb) / (valid columns),
+    an exact rational worked out here without the oracle's loops."""
+    from fractions import Fraction
+    N, d = 512, 16
+    nb, per = N // 128, 128 // S
+    q = torch.zeros(1, N, 1, d).bfloat16()
+    k = (torch.randn(1, N, 1, d, generator=torch.Generator().manual_seed(3))).bfloat16()
+    got = oracle.xattn_mass(q, k, S, causal=causal)[0, 0]
+    for qb in range(nb):
+        for kb in range(qb + 1 if causal else nb):
+            est = Fraction(0)
+            for i in range(per):
+                R = qb * per + i
+                valid = R + 1 if causal else N // S
+                inside = (min(R, (kb + 1) * per - 1) - kb * per + 1) if causal else per
+                est += Fraction(max(inside, 0), valid)
+            est /= per
+            at = (qb * (qb + 1) // 2 if causal else qb * nb) + kb
+            assert got[at] == pytest.approx(float(est), rel=1e-12, abs=1e-15), (qb, kb)
