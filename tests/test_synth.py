@@ -65,3 +65,22 @@ def test_logit_units_make_per_head_budgets_differ():
     assert (budgets[False] >= nb - 2).all() and len(set(budgets[False].tolist())) == 1
     assert budgets[True].max() - budgets[True].min() >= 5
     assert int(np.argmin(budgets[True])) == int(np.argmax(s))
+
+
+def test_per_group_directions_are_shared_within_a_group_only():
+    """The Qwen-shaped recipe draws one direction per GQA group: the mean q row
+    of a head points along its group's u_g (shared by the group's heads, scaled
+    by s_h), and the groups' directions differ."""
+    w = synth.small_workload(seqlen=2048, heads=8, kv_heads=4, head_dim=64, needles=0, seed=9, per_group=True)
+    x = synth.make_inputs(w)
+    mean = x["q"].float()[0].mean(dim=0)                 # [H, d]: 2 s_h u_{g(h)} + noise of size ~0.5/sqrt(N)
+    dirs = mean / mean.norm(dim=-1, keepdim=True)
+    cos = dirs @ dirs.T
+    for a in range(8):
+        for b in range(8):
+            same = a * 4 // 8 == b * 4 // 8
+            assert (cos[a, b] > 0.99) if same else (abs(cos[a, b]) < 0.6), (a, b, float(cos[a, b]))
+    # the norm of each head's mean is 2 s_h
+    assert torch.allclose(mean.norm(dim=-1), 2.0 * x["s"], rtol=0.03)
+    # no needles were asked for: K carries no direction apart from the sink scaling
+    assert x["needles"].numel() == 0
