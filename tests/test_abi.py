@@ -208,3 +208,21 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 128, 2, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         pa.pool_heads(q, q, 1)
+
+
+def test_header_compiles_and_links_as_plain_c(tmp_path):
+    """A C99 program (tests/c/abi_from_c.c) includes pa.h, links libpa.so and
+    gets argument errors back without a GPU."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(pa.LIB_PATH)
+    exe = tmp_path / "abi_from_c"
+    cc = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(root, "include"),
+                         os.path.join(root, "tests", "c", "abi_from_c.c"), "-o", str(exe),
+                         "-L", libdir, "-l:libpa.so", f"-Wl,-rpath,{libdir}"], capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0 and run.stdout.strip() == "ok", run.stdout + run.stderr
