@@ -22,8 +22,8 @@
 //              in ping-pong order  PV_0(i), QK_0(i+1), PV_1(i), QK_1(i+1), so
 //              the tensor core computes one head's products while the other
 //              head's softmax runs.
-//   softmax    one thread per query row (TMEM lane).  Two passes over S in TMEM (row max,
-//              then exp2/row sum/bf16 pack of P written back over S), online
+//   softmax    one thread per query row (TMEM lane).  S is read from TMEM once; row max,
+//              then exp2/row sum/bf16 pack of P, written back over S; online
 //              softmax with the running max raised only when it grows by more
 //              than 2^8 (then O is rescaled in TMEM), final O/l and LSE.
 // TMEM columns: S_0 [0,128)  S_1 [128,256)  O_0 [256,384)  O_1 [384,512);
