@@ -39,7 +39,8 @@
  *                             (BLASST introduction, 3.1): a visited block far
  *                             below the running max is left out.
  *
- * Readings where the pages are silent (all listed in the design notes):
+ * Readings where the pages are silent, each the plainest one that the
+ * surviving text supports:
  *   mean pooling; K pooled over the expanded KV heads of the group's q heads;
  *   pre-softmax scaled logits as token scores; proxies rounded to bf16 (RNE)
  *   before scoring; budget from exactly the last 128-row Q block; budget
@@ -352,14 +353,15 @@ void pa_oracle_sparse_attn(int N, int H, int Hkv, int d, int G,
 {
     int nb = N / BLK;
     int64_t T = rows_total(causal, nb);
-    #pragma omp parallel for schedule(dynamic, 1)
-    for (int it = 0; it < n_items; it++) {
-        int b = items[3 * it], h = items[3 * it + 1], qb = items[3 * it + 2];
-        int g = grp_of(h, H, G), kvh = kv_of(h, H, Hkv);
-        const int32_t *list = rank + ((int64_t)b * G + g) * T + row_at(causal, nb, qb);
-        int n = cnt[((int64_t)b * H + h) * nb + qb];
-        double *z = (double *)malloc(sizeof(double) * n * BLK);
+    /* every (item, row) pair is independent: one item keeps every thread busy */
+    #pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int it = 0; it < n_items; it++)
         for (int ii = 0; ii < BLK; ii++) {
+            int b = items[3 * it], h = items[3 * it + 1], qb = items[3 * it + 2];
+            int g = grp_of(h, H, G), kvh = kv_of(h, H, Hkv);
+            const int32_t *list = rank + ((int64_t)b * G + g) * T + row_at(causal, nb, qb);
+            int n = cnt[((int64_t)b * H + h) * nb + qb];
+            double *z = (double *)malloc(sizeof(double) * (n > 0 ? n : 1) * BLK);
             int i = qb * BLK + ii;
             double zmax = -INFINITY;
             for (int t = 0; t < n; t++)
@@ -390,9 +392,8 @@ void pa_oracle_sparse_attn(int N, int H, int Hkv, int d, int G,
                         o[c] += p * bf16_to_f64(v[b * vsb + (int64_t)j * vss + kvh * vsh + c]);
                 }
             if (lse) lse[(int64_t)it * BLK + ii] = zmax + log(den);
+            free(z);
         }
-        free(z);
-    }
 }
 
 /* ------------------------------------------------ o7 running-max block skip */
