@@ -78,6 +78,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the extra configurations of the 128K layer (G = 4, fixed 10 %%, logit units)")
     return ap.parse_args()
 
 
@@ -362,13 +364,6 @@ def input_bytes(pipe) -> int:
     return sum(t.numel() * t.element_size() for t in (pipe.q, pipe.k, pipe.v))
 
 
-def l2_policy(pipe) -> str:
-    """How the timed steps avoid reusing L2 contents (stated in the config)."""
-    if input_bytes(pipe) > 2 * L2_BYTES:
-        return "inputs larger than L2 (q+k+v per layer > 2 x 126 MB), no flush"
-    return "L2 flushed between timed steps (a 512 MiB buffer written outside the timed events)"
-
-
 def time_pipeline(pipe, steps, warmup, dist_on, sampler=None):
     """Mean per-stage times and the total of `steps` steps, each step timed
     between its own first and last event (so an L2 flush between steps is
@@ -397,6 +392,21 @@ def time_pipeline(pipe, steps, warmup, dist_on, sampler=None):
     total = sum(e[0].elapsed_time(e[4]) for e in evs)
     stages = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])
     return total, stages.mean(0), clocks
+
+
+# Dense bf16 tcgen05 rate of one SM: 4096 multiply-adds per clock (a
+# 128x128x16 MMA in 64 cycles, measured by an in-bounds microbenchmark).
+TENSOR_FLOP_PER_CLK_SM = 8192
+
+
+def tensor_busy(flops: float, ms: float, clocks, device):
+    """FLOPs of a launch over what the tensor pipes of every SM can do in its
+    duration at the median SM clock sampled in the timed region (None without
+    a clock record)."""
+    if not clocks or not clocks.get("sm_mhz"):
+        return None
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    return flops / (TENSOR_FLOP_PER_CLK_SM * sms * ms * 1e-3 * clocks["sm_mhz"] * 1e6)
 
 
 def counters_for(kernel_key: str, source_files):
@@ -433,65 +443,96 @@ ATTN_SOURCES = ["block_sparse_attention_pa_b200/csrc/attn.cuh", "block_sparse_at
 
 
 # ------------------------------------------------------------ CPU oracle
-def oracle_estimate(x, w: synth.Workload, G, mode, gamma, frac, size="baseline", seed=0, stride=1, skip=0.0):
+ORACLE_POOL_TOKENS = 8192      # o1 and o3 run on this token prefix
+ORACLE_SCORE_TILES = 64        # o2 tiles of the prefix's last query block (per group)
+ORACLE_ATTN_BLOCKS = 1536      # o5 items are drawn until they visit this many blocks
+
+
+def oracle_estimate(x, w: synth.Workload, G, mode, gamma, frac, seed=0, stride=1, skip=0.0):
     """Time the CPU oracle on a bounded sample of one layer and extrapolate to
-    ms per layer.  x: CPU bf16 tensors.  Returns (ms_per_layer, per-stage
-    seconds, description of the sample)."""
+    ms per layer.  The CPU-baseline leg and every step of the reference arm
+    take the same sample (only the seed of the attention items changes), and
+    every stage's sample keeps all the oracle's threads busy.  x: CPU bf16
+    tensors.  Returns (ms_per_layer, per-stage seconds, threads used per stage,
+    description of the sample)."""
     import oracle
+    threads = oracle.num_threads()
     rng = np.random.default_rng(seed)
     q, k, v = x["q"], x["k"], x["v"]
     B, N, H, d = q.shape
     Hkv = k.shape[2]
     nb = N // 128
     T = nb * (nb + 1) // 2
-    if size == "baseline":   # about 10-30 s of CPU work at 128K
-        pool_tokens, n_tiles, mass_heads, n_items = N, nb, H // Hkv * 2, 8
-    else:                    # one reference-arm step: a few seconds
-        pool_tokens, n_tiles, mass_heads, n_items = min(N, 8192), 64, 1, 1
-    det = {}
-    # o1 pool on the first pool_tokens tokens
+    npre = min(N, ORACLE_POOL_TOKENS)
+    det, used = {}, {}
+    # o1 pool on the first npre tokens (parallel over tokens)
     t0 = time.perf_counter()
-    _, _, qpb, kpb = oracle.pool(q[:, :pool_tokens], k[:, :pool_tokens], G)
-    det["pool_s"] = (time.perf_counter() - t0) * N / pool_tokens
-    # o2 block scores of n_tiles tiles of the last query block inside the pooled tokens
-    nbp = pool_tokens // 128
-    kbs = np.linspace(0, nbp - 1, min(n_tiles, nbp)).astype(int)
+    _, _, qpb, kpb = oracle.pool(q[:, :npre], k[:, :npre], G)
+    det["pool_s"] = (time.perf_counter() - t0) * N / npre
+    used["pool"] = min(threads, B * npre)
+    # o2 block scores of tiles of the prefix's last query block (parallel over tiles)
+    nbp = npre // 128
+    kbs = np.linspace(0, nbp - 1, min(ORACLE_SCORE_TILES, nbp)).astype(int)
     tiles = [(0, g, nbp - 1, int(kb)) for g in range(G) for kb in kbs]
     t0 = time.perf_counter()
     last = oracle.block_score_tiles(qpb, kpb, tiles, stride=stride)
     det["scores_s"] = (time.perf_counter() - t0) * (B * G * T) / len(tiles)
-    # o3 head mass of mass_heads heads (with their KV heads)
-    hk = max(1, mass_heads * Hkv // H)
+    used["scores"] = min(threads, len(tiles))
+    # o3 head mass (parallel over heads): whole GQA groups of heads, at least
+    # one head per thread, on the last query block of the npre-token prefix;
+    # its cost grows with the keys each row reads, i.e. linearly in N
+    per = H // Hkv
+    mass_heads = min(H, per * max(1, -(-threads // per)))
+    hk = mass_heads // per
     t0 = time.perf_counter()
-    mass_s = oracle.head_mass(q[:, :, :mass_heads].contiguous(), k[:, :, :hk].contiguous())
-    det["mass_s"] = (time.perf_counter() - t0) * H / mass_heads if mode == 0 else 0.0
-    # o4 ranking over the full [B, G, T] array (seeded fill; the sampled last-row tiles real)
+    mass_s = oracle.head_mass(q[:, :npre, :mass_heads].contiguous(), k[:, :npre, :hk].contiguous())
+    det["mass_s"] = (time.perf_counter() - t0) * (H / mass_heads) * (N / npre) if mode == 0 else 0.0
+    used["mass"] = min(threads, B * mass_heads)
+    # o4 ranking over the full [B, G, T] array (seeded fill; the sampled tiles real)
     scores = rng.standard_normal((B, G, T))
     if nbp == nb:
-        for (b, g, qb, kb), s in zip(tiles, last):
-            scores[b, g, T - nb + kb] = s
+        for (b, g, qb, kb), sc in zip(tiles, last):
+            scores[b, g, T - nb + kb] = sc
     t0 = time.perf_counter()
     rank = oracle.rank(scores, nb)
     det["rank_s"] = time.perf_counter() - t0
-    # budget with the sampled heads' masses repeated over all heads
-    mass = np.tile(mass_s, (1, -(-H // mass_heads), 1))[:, :H]
+    used["rank"] = min(threads, B * G * nb)
+    # budget (a plain loop) with the sampled heads' masses repeated over every
+    # head and spread from the prefix's nbp blocks over all nb (block kb takes
+    # an equal share of prefix block kb * nbp // nb), so that the visited-block
+    # count the attention is extrapolated to follows the sampled heads' budgets
+    ms_all = np.tile(mass_s, (1, -(-H // mass_heads), 1))[:, :H]
+    src = np.arange(nb) * nbp // nb
+    mass = ms_all[:, :, src] / np.bincount(src, minlength=nbp)[src]
     t0 = time.perf_counter()
     _, cnt = oracle.budget(rank, mass if mode == 0 else None, H, G, nb, mode, float(np.float32(gamma)), frac)
     det["budget_s"] = time.perf_counter() - t0
-    # o5 sparse attention on random (b, h, qb) items, extrapolated per visited block
-    items = [(int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(nb))) for _ in range(n_items)]
+    used["budget"] = 1
+    # o5 sparse attention on random (b, h, qb) items (parallel over items x
+    # rows), extrapolated per visited block
+    items, blocks = [], 0
+    if int(cnt.sum()) <= ORACLE_ATTN_BLOCKS:  # a small layer: every item once
+        items = [(b, h, qb) for b in range(B) for h in range(H) for qb in range(nb)]
+        blocks = int(cnt.sum())
+    else:
+        while blocks < ORACLE_ATTN_BLOCKS:
+            it = (int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(nb)))
+            if it not in items:
+                items.append(it)
+                blocks += int(cnt[it])
     t0 = time.perf_counter()
     if skip > 0.0:
         oracle.sparse_attn_skip(q, k, v, rank, cnt, G, items, skip)
     else:
         oracle.sparse_attn(q, k, v, rank, cnt, G, items)
     dt = time.perf_counter() - t0
-    blocks = sum(int(cnt[b, h, qb]) for b, h, qb in items)
     det["attn_s"] = dt * float(cnt.sum()) / max(blocks, 1)
-    sample = (f"pool of {pool_tokens}/{N} tokens; scores of {len(tiles)}/{B * G * T} tiles; head mass of "
-              f"{mass_heads}/{H} heads; full rank+budget; attention of {n_items} random (b,h,qb) items "
-              f"({blocks} of {int(cnt.sum())} visited blocks); each stage extrapolated linearly")
-    return sum(det.values()) * 1e3, det, sample
+    used["attn"] = min(threads, len(items) * 128)
+    sample = (f"pool of {npre}/{N} tokens; scores of {len(tiles)}/{B * G * T} tiles; head mass of "
+              f"{mass_heads}/{H} heads over the last query block of a {npre}-token prefix; full rank+budget; "
+              f"attention of {len(items)} random (b,h,qb) items ({blocks} of {int(cnt.sum())} visited blocks); "
+              f"each stage extrapolated linearly (tokens, tiles, heads x keys, visited blocks)")
+    return sum(det.values()) * 1e3, det, used, sample
 
 
 def cpu_model() -> str:
@@ -507,25 +548,31 @@ def cpu_model() -> str:
 
 
 def run_reference(args, w, G, mode, gamma, frac):
-    """The reference arm: the CPU oracle, timed on the host cores."""
+    """The reference arm: the CPU oracle, timed on the host cores, one bounded
+    sample of the layer per step (the same sample as the CPU-baseline leg)."""
     if int(os.environ.get("RANK", "0")) != 0:
         return
     import oracle
     x = synth.make_inputs(w, device="cpu")
     vals = []
     for i in range(args.warmup + args.steps):
-        ms, det, sample = oracle_estimate(x, w, G, mode, gamma, frac, size="step", seed=i,
-                                          stride=args.score_stride, skip=args.skip_threshold)
+        ms, det, used, sample = oracle_estimate(x, w, G, mode, gamma, frac, seed=i,
+                                                stride=args.score_stride, skip=args.skip_threshold)
         if i >= args.warmup:
             vals.append(ms)
     v = statistics.mean(vals)
     cores = oracle.num_threads()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "ms/layer", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": v, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_of(w, G, mode, gamma, frac, args.score_stride, args.skip_threshold),
-            "cpu_baseline": {"value": v, "unit": "ms/layer", "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
-                             "sample": sample},
+            "extrapolated": True,
+            "config": line_config(args, w, G, mode, gamma, frac, world),
+            "cpu_baseline": {"value": v, "unit": "ms/layer", "cores": cores, "kind": "oracle",
+                             "cpu_model": cpu_model(), "sample": sample, "threads_used": used,
+                             "extrapolated": True,
+                             "note": "value extrapolated from a bounded sample of the layer, so a step's "
+                                     "wall time is not the value"},
             "e2e": {"value": v, "unit": "ms/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -536,6 +583,22 @@ def config_of(w, G, mode, gamma, frac, stride=1, skip=0.0):
             "kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "groups": G, "budget": budget, "block": 128,
             "score_stride": stride, "skip_threshold": skip,
             "l2": "inputs larger than L2 (q+k+v per layer > 2 x 126 MB), no flush"}
+
+
+def line_config(args, w, G, mode, gamma, frac, world):
+    """The bench line's `config`, the same for both arms (the reference arm
+    names the workload its samples come from)."""
+    causal = not args.non_causal
+    l2 = ("inputs larger than L2 (q+k+v per layer > 2 x 126 MB), no flush"
+          if w.batch * w.seqlen * (w.num_q_heads + 2 * w.num_kv_heads) * w.head_dim * 2 > 2 * L2_BYTES else
+          "L2 flushed between timed steps (a 512 MiB buffer written outside the timed events)")
+    if args.estimator == "xattn":
+        cfg = config_of(w, w.num_q_heads, 1, 0.0, 1000, 1, args.skip_threshold) | {
+            "groups": w.num_q_heads, "budget": f"XAttention find_blocks tau={args.tau}",
+            "estimator": f"xattn antidiagonal stride {args.xattn_stride}"}
+    else:
+        cfg = config_of(w, G, mode, gamma, frac, args.score_stride, args.skip_threshold)
+    return cfg | {"parallelism": f"replicas x{world}", "causal": causal, "l2": l2}
 
 
 # ------------------------------------------------------------------- main
@@ -614,6 +677,12 @@ def main():
                 "peak_kind": f"{peaks_kind} bf16 sustained (kernel timed inside back-to-back steps)",
                 "flops_per_launch": flops_exec, "visited_tile_flops_per_launch": flops,
                 "exact_causal_flops_per_launch": flops_exact}
+    busy = tensor_busy(flops_exec, attn_ms, clocks, q.device)
+    if busy is not None:
+        roofline["tensor_busy"] = busy
+        roofline["tensor_busy_def"] = (f"flops_per_launch / ({TENSOR_FLOP_PER_CLK_SM} FLOP/clk x SMs x attention "
+                                       f"time x median SM clock of the timed region): the share of SM cycles the "
+                                       f"tensor pipe needs at the clock the kernel actually ran")
 
     # per-stage rooflines
     d = w.head_dim
@@ -661,11 +730,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded needle/sink generator; random inputs, no weights)",
-            "config": (config_of(w, G, mode, gamma, frac, stride, skip) if not xattn else
-                       config_of(w, H, 1, 0.0, 1000, 1, skip) | {
-                           "groups": H, "budget": f"XAttention find_blocks tau={args.tau}",
-                           "estimator": f"xattn antidiagonal stride {args.xattn_stride}"})
-                      | {"parallelism": f"replicas x{world}", "causal": not args.non_causal, "l2": l2_policy(pipe)},
+            "config": line_config(args, w, G, mode, gamma, frac, world),
             "est_ms": est_ms, "sparse_ms": attn_ms,
             "tflops_effective": flops / (attn_ms * 1e-3) / 1e12, "tflops_exact_causal": flops_exact / (attn_ms * 1e-3) / 1e12,
             "visited_blocks": visited, "density": density, "sparsity": 1.0 - density,
@@ -692,6 +757,11 @@ def main():
         line["layer_speedup_vs_dense"] = dense_attn / (est_ms + attn_ms)
         line["estimate_frac_of_dense"] = est_ms / dense_attn
         del dense
+
+    # extra configurations of the headline layer, timed in the same run
+    if (not args.no_extras and not args.no_dense and not xattn and not args.non_causal and mode == 0
+            and stride == 1 and skip == 0.0 and args.gen == "literal" and w.name == "llama8b_n128k"):
+        line["extras"] = run_extras(w, x, gamma, line["dense_attn_ms"], peak, dist_on, local, rank)
 
     # the same step captured once into a CUDA graph and replayed (launch costs
     # amortised; the stage split above comes from the eager run)
@@ -729,15 +799,66 @@ def main():
     if not args.no_cpu_baseline and world == 1 and rank == 0 and not xattn and not args.non_causal:
         import oracle
         xc = {n: x[n].cpu() for n in ("q", "k", "v")}
-        ms, det, sample = oracle_estimate(xc, w, G, mode, gamma, frac, size="baseline", stride=stride, skip=skip)
+        runs = [oracle_estimate(xc, w, G, mode, gamma, frac, seed=i, stride=stride, skip=skip) for i in range(2)]
+        ms = statistics.mean(r[0] for r in runs)
+        det = {key: statistics.mean(r[1][key] for r in runs) for key in runs[0][1]}
         line["cpu_baseline"] = {"value": ms, "unit": "ms/layer", "cores": oracle.num_threads(), "kind": "oracle",
-                                "cpu_model": cpu_model(), "sample": sample, "stage_s": det}
+                                "cpu_model": cpu_model(), "sample": runs[0][3] + "; mean of 2 samples (seeds 0, 1)",
+                                "stage_s": det, "threads_used": runs[0][2], "extrapolated": True}
 
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist_on:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
+
+
+def run_extras(w, x, gamma, dense_ms, peak, dist_on, local, rank):
+    """Other configurations of the same 128K Llama layer, a few timed steps each
+    (the dense time is the headline run's: the all-blocks kernel does the same
+    work on any input):
+      g4_r1, g4_r4  G = 4 proxy groups, every query row / every 4th row scored:
+                    the estimate's cost against the dense attention;
+      fixed_10pct   a fixed budget of 10 % of the causal blocks: sparse
+                    attention speed-up over dense;
+      logit_units   the labelled logit-unit input, where per-head dynamic
+                    budgets differ (two heads of a CTA keep different prefixes
+                    of their list)."""
+    out = {}
+    q, k, v = x["q"], x["k"], x["v"]
+    H = w.num_q_heads
+
+    def one(name, qq, kk, vv, G, mode, frac, stride):
+        pipe = Pipeline(qq, kk, vv, G, mode, gamma, frac, stride)
+        sampler = ClockSampler(local) if rank == 0 else None
+        total, stages, clocks = time_pipeline(pipe, 3, 2, dist_on, sampler)
+        vis, flops, _ = pipe.visited()
+        est, attn = float(stages[:3].sum()), float(stages[3])
+        tf = flops / (attn * 1e-3) / 1e12
+        r = {"groups": G, "score_stride": stride,
+             "budget": f"dynamic gamma={gamma}" if mode == 0 else f"fixed {frac / 10:.1f}% of causal blocks",
+             "est_ms": est, "est_stages_ms": [float(t) for t in stages[:3]], "attn_ms": attn,
+             "density": vis / (pipe.B * H * pipe.T), "attn_tflops": tf, "attn_frac_of_sustained": tf / peak,
+             "speedup_vs_dense": dense_ms / attn, "estimate_frac_of_dense": est / dense_ms,
+             "layer_ms": est + attn, "steps": 3}
+        busy = tensor_busy(flops, attn, clocks, qq.device)
+        if busy is not None:
+            r["tensor_busy"] = busy
+            r["sm_mhz"] = clocks["sm_mhz"]
+            r["clock_reasons"] = clocks["reasons"]
+        out[name] = r
+        del pipe
+
+    one("g4_r1", q, k, v, 4, 0, 0, 1)
+    one("g4_r4", q, k, v, 4, 0, 0, 4)
+    one("fixed_10pct", q, k, v, 1, 1, 100, 1)
+    wl = w.replace(name=w.name + "_logit", logit_units=True)
+    xl = synth.make_inputs(wl, device=q.device, seed=w.seed + rank)
+    one("logit_units", xl["q"], xl["k"], xl["v"], 1, 0, 0, 1)
+    out["logit_units"]["workload"] = wl.name
+    del xl
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_e2e(pa, w, G, mode, gamma, frac, x, args, dist_on, world, stride=1, skip=0.0, causal=True):

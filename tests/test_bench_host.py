@@ -133,3 +133,21 @@ def test_clock_records_that_force_a_second_measurement():
     assert not bench.clocks_rejected(dict(ok, sm_mhz=1200.0))
     assert not bench.clocks_rejected(dict(ok, sm_mhz=1900.0, reasons=[]))
     assert bench.agree_any(True, "cpu", False) and not bench.agree_any(False, "cpu", False)
+
+
+def test_cpu_sample_uses_every_thread_and_both_arms_share_config():
+    """The CPU-baseline leg and the reference arm take the same oracle sample,
+    whose stages keep every oracle thread busy, and print the same config."""
+    import argparse
+    import oracle
+    from block_sparse_attention_pa_b200 import synth
+    w = synth.small_workload(seqlen=1024, heads=8, kv_heads=2, head_dim=64)
+    x = synth.make_inputs(w)
+    ms, det, used, sample = bench.oracle_estimate(x, w, 1, 0, 0.95, 0, seed=0)
+    threads = oracle.num_threads()
+    assert ms > 0 and set(det) == {"pool_s", "scores_s", "mass_s", "rank_s", "budget_s", "attn_s"}
+    assert used["attn"] == min(threads, 8 * 8 * 128) and used["pool"] == min(threads, 1024)
+    args = argparse.Namespace(non_causal=False, estimator="proxy", score_stride=1, skip_threshold=0.0, tau=0.9,
+                              xattn_stride=8)
+    cfg = bench.line_config(args, w, 1, 0, 0.95, 0, 1)
+    assert cfg["parallelism"] == "replicas x1" and cfg["causal"] is True and cfg["workload"] == w.name
