@@ -6,8 +6,10 @@ Acceptance (stated with the method's configs):
   block scores  |gpu - ref| <= 1e-3 * max(|ref|, 1)
   rank, budget, cnt   bit-exact when the oracle is fed the GPU's fp32 scores
                 and masses (ties to the lower block index)
-  head mass     |gpu - ref| <= 2e-5 + 2e-3 * ref (fp32 logits of bf16
-                products, ex2.approx; derived in the design notes)
+  head mass     |gpu - ref| <= 2e-5 + 2e-3 * ref: the GPU's logits are fp32
+                sums of bf16 products (about 1e-6 relative error), its
+                exponentials ex2.approx (about 2^-22), and a mass adds up to
+                16K keys' probabilities in fp32
   O             max-abs <= 2e-2 and mean-abs <= 2e-3 against the fp64 oracle
                 run with the GPU's mask
 """
