@@ -99,6 +99,7 @@ def lib() -> ctypes.CDLL:
         L.pa_xattn_workspace_size.argtypes = [P(Shape), ctypes.c_int32]
         L.pa_xattn_mask.argtypes = [P(Shape), ctypes.c_int32, ctypes.c_float, vp, st, vp, st, vp, vp, vp, vp,
                                     ctypes.c_size_t, vp]
+        L.pa_build_mask_noalloc.argtypes = [P(Shape), P(Budget), vp, vp, st, vp, st, P(MaskBufs), vp]
         L.pa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp]
         L.pa_status_string.restype = ctypes.c_char_p
         L.pa_status_string.argtypes = [ctypes.c_int]
@@ -106,7 +107,8 @@ def lib() -> ctypes.CDLL:
         L.pa_abi_version.restype = ctypes.c_int32
         for name in ("pa_pool_heads", "pa_block_scores", "pa_build_mask", "pa_block_sparse_attn", "pa_prefill",
                      "pa_get_device_status", "pa_selftest_wait_timeout", "pa_pool_heads_strided",
-                     "pa_block_scores_strided", "pa_block_sparse_attn_skip", "pa_xattn_mask", "pa_prefill_varlen"):
+                     "pa_block_scores_strided", "pa_block_sparse_attn_skip", "pa_xattn_mask", "pa_prefill_varlen",
+                     "pa_build_mask_noalloc"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib

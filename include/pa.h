@@ -219,8 +219,10 @@ PA_API pa_status pa_build_mask(const pa_shape *shape, const pa_budget *budget,
  * 64K tokens); larger shapes return PA_ERR_UNSUPPORTED with that limit in
  * pa_last_error().  The other modes need no scratch.  The first call on each
  * device looks up the array's device address (cudaGetSymbolAddress, with that
- * device current); make that first call before any stream capture.  The call
- * allocates nothing.  All calls on a device share the one array, so two calls
+ * device current); make that first call before any stream capture.  The
+ * address is kept for the life of the process, so the device must not be
+ * reset (cudaDeviceReset, or a primary context released and created again)
+ * after that first call.  The call allocates nothing.  All calls on a device share the one array, so two calls
  * whose kernels overlap on the GPU (different streams, no ordering between
  * them) race on it; calls ordered on one stream are safe.  No contents carry
  * over between calls: each call writes every scratch byte it reads. */
