@@ -394,46 +394,14 @@ pa_status launch_xattn_gemm_d(int S, const CUtensorMap &mq, const CUtensorMap &m
     return launch_xattn_gemm_t<D, 16>(mq, mk, p, st);
 }
 
-// SM-pair variant: one cluster of two CTAs per 256 x 256 output tile, at most
-// one pair per two SMs.
-template <int D, int S>
-pa_status launch_xattn_gemm_pair_t(const CUtensorMap &mq, const CUtensorMap &mk, const pa::XattnParams &p,
-                                   cudaStream_t st) {
-    auto kern = pa::xattn_gemm_pair_kernel<D, S>;
-    const int smem = pa::XattnPairSmem<D, S>::BYTES;
-    PA_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-    const long long pairs = std::min<long long>(p.num_units, num_sms() / 2);
-    if (pairs <= 0) return PA_OK;
-    kern<<<static_cast<unsigned>(2 * pairs), 192, smem, st>>>(mq, mk, p);
-    PA_CUDA(cudaGetLastError());
-    return PA_OK;
-}
-
-template <int D>
-pa_status launch_xattn_gemm_pair_d(int S, const CUtensorMap &mq, const CUtensorMap &mk, const pa::XattnParams &p,
-                                   cudaStream_t st) {
-    if (S == 4) return launch_xattn_gemm_pair_t<D, 4>(mq, mk, p, st);
-    if (S == 8) return launch_xattn_gemm_pair_t<D, 8>(mq, mk, p, st);
-    return launch_xattn_gemm_pair_t<D, 16>(mq, mk, p, st);
-}
-
-// The XAttention estimate GEMM runs on SM pairs only with PA_XATTN_PAIR=1: the
-// pair kernel is correct but measured no faster than the one-SM kernel (the
-// one-SM GEMM is not bound by shared-memory or L2 bandwidth).
-bool xattn_pair_enabled() {
-    const char *e = std::getenv("PA_XATTN_PAIR");
-    return e && e[0] == '1';
-}
-
 pa_status launch_xattn(const pa_shape *s, int S, float tau, const void *q, pa_strides qs, const void *k,
                        pa_strides ks, int32_t *rank, int32_t *cnt, float *mass, void *ws, cudaStream_t st) {
     const int B = s->batch, H = s->num_q_heads, Hkv = s->num_kv_heads, N = s->seqlen, d = s->head_dim;
     const int nb = N / kBlk, rows = N / S;
-    const bool pair = xattn_pair_enabled();
     CUtensorMap mq, mk;
     pa_status r = map_bnhd_split(&mq, q, B, N, H, d, S, qs, 128, "q");
     if (r) return r;
-    if ((r = map_bnhd_split(&mk, k, B, N, Hkv, d, S, ks, pair ? 128 : 256, "k"))) return r;
+    if ((r = map_bnhd_split(&mk, k, B, N, Hkv, d, S, ks, 256, "k"))) return r;
     const XWsLayout w = xattn_ws_layout(s, S);
     uint8_t *base = static_cast<uint8_t *>(ws);
     pa::XattnParams p{};
@@ -443,10 +411,7 @@ pa_status launch_xattn(const pa_shape *s, int S, float tau, const void *q, pa_st
     const int mtiles = (rows + 127) / 128;
     p.causal = causal_of(s) ? 1 : 0;
     long long per = 0;
-    if (pair) {  // 256-row tiles: row tile m needs column tiles 0..m (causal)
-        const long long m2 = (rows + 255) / 256;
-        per = p.causal ? m2 * (m2 + 1) / 2 : m2 * m2;
-    } else if (p.causal) {
+    if (p.causal) {
         for (int mt = 0; mt < mtiles; ++mt) per += mt / 2 + 1;
     } else {
         per = static_cast<long long>(mtiles) * ((rows + 255) / 256);
@@ -457,10 +422,7 @@ pa_status launch_xattn(const pa_shape *s, int S, float tau, const void *q, pa_st
     p.part_s = reinterpret_cast<float *>(base + w.part_s);
     p.part_m = reinterpret_cast<float *>(base + w.part_m);
     p.timeout_ns = wait_timeout_ns();
-    if (pair)
-        r = d == 128 ? launch_xattn_gemm_pair_d<128>(S, mq, mk, p, st) : launch_xattn_gemm_pair_d<64>(S, mq, mk, p, st);
-    else
-        r = d == 128 ? launch_xattn_gemm_d<128>(S, mq, mk, p, st) : launch_xattn_gemm_d<64>(S, mq, mk, p, st);
+    r = d == 128 ? launch_xattn_gemm_d<128>(S, mq, mk, p, st) : launch_xattn_gemm_d<64>(S, mq, mk, p, st);
     if (r) return r;
     pa::XselParams sp{};
     sp.B = B; sp.H = H; sp.nb = nb; sp.rows = rows; sp.nchunk = p.nchunk;

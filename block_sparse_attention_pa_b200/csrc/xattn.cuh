@@ -269,305 +269,6 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-// ------------------------------------------------- SM-pair (2-CTA) GEMM
-// The same antidiagonal GEMM on an SM pair: a cluster of two CTAs computes a
-// 256-row x 256-column output tile with tcgen05.mma.cta_group::2 (M = 256,
-// N = 256).  Each CTA stages its own 128 strided rows of A and one 128-column
-// half of B per 64-feature chunk, so an SM moves 32 KB per chunk through shared
-// memory instead of 48 KB for the same tensor work.  The even CTA (the leader)
-// issues the MMAs; its full barriers count the bytes of both CTAs' copies; the
-// commits of the stage releases and of the accumulators reach both CTAs; both
-// CTAs' epilogues release an accumulator on the leader's barrier.  Every wait
-// is bounded, and both CTAs meet at the two cluster barriers (after set-up and
-// before teardown) on every path.
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// shared::cluster address of the variable at `local` in CTA `rank` of the cluster
-__device__ __forceinline__ uint32_t cluster_addr(const void *local, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
-}
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
-                 "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish_pair() {
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-// D[tmem of both CTAs] (+)= A[both CTAs' smem] * B[both CTAs' smem]^T, issued by the leader
-__device__ __forceinline__ void umma_ss_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                             uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-// arrive on the barrier at `bar`'s offset in every CTA of `mask` once the
-// leader's MMAs issued so far have completed
-__device__ __forceinline__ void umma_commit_pair(uint64_t *bar, uint16_t mask) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-            smem_u32(bar)),
-        "h"(mask)
-        : "memory");
-}
-// 5-D tile copy into this CTA's shared memory whose completion is counted on a
-// barrier of either CTA of the pair (`cluster_bar`, a shared::cluster address)
-__device__ __forceinline__ void tma_load_5d_pair(void *dst, const CUtensorMap *m, uint32_t cluster_bar, int c0,
-                                                 int c1, int c2, int c3, int c4) {
-    asm volatile(
-        "cp.async.bulk.tensor.5d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(cluster_bar)
-        : "memory");
-}
-
-// Output tiles of one (b, h) for the pair kernel: row tile mt covers strided
-// rows 256 mt .. 256 mt + 255 and (causal) needs column tiles 0 .. mt, so the
-// tiles before row tile mt number mt(mt+1)/2.
-__device__ __forceinline__ XUnit xattn_decode_pair(const XattnParams &p, long long u) {
-    XUnit x;
-    const long long bh = u / p.units_per_bh;
-    const long long w = u - bh * p.units_per_bh;
-    x.b = static_cast<int>(bh / p.H);
-    x.h = static_cast<int>(bh % p.H);
-    if (!p.causal) {
-        const long long ntn = (p.rows + 255) / 256;
-        x.mt = static_cast<int>(w / ntn);
-        x.nt = static_cast<int>(w % ntn);
-        return x;
-    }
-    long long a = static_cast<long long>((sqrt(1.0 + 8.0 * static_cast<double>(w)) - 1.0) * 0.5);
-    while (a > 0 && a * (a + 1) / 2 > w) --a;
-    while ((a + 1) * (a + 2) / 2 <= w) ++a;
-    x.mt = static_cast<int>(a);
-    x.nt = static_cast<int>(w - a * (a + 1) / 2);
-    return x;
-}
-
-template <int D, int S>
-struct XattnPairSmem {
-    static constexpr int A_BYTES = 128 * 64 * 2;   // one 64-wide K chunk of this CTA's 128 rows
-    static constexpr int B_BYTES = 128 * 64 * 2;   // one 64-wide K chunk of this CTA's 128-column half
-    static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int STAGES = 6;
-    static constexpr int KCHUNKS = S * D / 64;
-    static constexpr int BYTES = STAGES * STAGE + 1024 /*align*/ + 256 /*barriers*/;
-};
-
-template <int D, int S>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
-    xattn_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                           const XattnParams p) {
-    using SM = XattnPairSmem<D, S>;
-    constexpr int NST = SM::STAGES;
-    constexpr int KC = SM::KCHUNKS;
-    constexpr int CPT = D / 64;        // 64-wide chunks per token
-    constexpr int CPB = 128 / S;       // strided columns (and rows) per 128-token block
-    constexpr uint32_t IDESC = idesc_bf16_f32(256, 256, false, false);
-    constexpr uint16_t kBoth = 0x3;    // both CTAs of the pair
-
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + NST * SM::STAGE);
-    uint64_t *full = bars;                     // NST (the leader's count both CTAs' bytes)
-    uint64_t *empty = bars + NST;              // NST
-    uint64_t *acc_full = bars + 2 * NST;       // 2
-    uint64_t *acc_empty = bars + 2 * NST + 2;  // 2 (the leader's take both CTAs' epilogues)
-    uint64_t *drain = bars + 2 * NST + 4;      // 1
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * NST + 5);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-
-    const uint32_t rank = cluster_rank();
-    const bool leader = rank == 0;
-    const long long pair_id = blockIdx.x >> 1;
-    const long long num_pairs = gridDim.x >> 1;
-    const uint32_t warp = warp_id(), lane = lane_id();
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < NST; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1);
-        }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], 256);
-        }
-        mbar_init(drain, 1);
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmQ);
-        tma_prefetch_desc(&tmK);
-    }
-    if (warp == 1) {
-        tmem_alloc_pair(tmem_slot, 512);  // two 128x256 fp32 accumulators in each CTA
-        tmem_relinquish_pair();
-    }
-    tc_fence_before();
-    cluster_sync_all();  // both CTAs' barriers initialised and TMEM allocated
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const WaitCtl wc{abort_flag, p.timeout_ns};
-
-    if (warp == 0) {
-        // ---------------------------------------------------------- producer
-        // Both CTAs: this CTA's 128 strided rows of A and 128-column half of B;
-        // the bytes are counted on the leader's full barrier of the stage.
-        if (lane == 0) {
-            long long it = 0;
-            bool ok = true;
-            for (long long u = pair_id; u < p.num_units && ok && !*abort_flag; u += num_pairs) {
-                const XUnit x = xattn_decode_pair(p, u);
-                const int kvh = static_cast<int>(static_cast<long long>(x.h) * p.Hkv / p.H);
-                const int R0 = x.mt * 256 + static_cast<int>(rank) * 128;
-                const int C0 = x.nt * 256 + static_cast<int>(rank) * 128;
-                for (int kc = 0; kc < KC; ++kc, ++it) {
-                    const int s = static_cast<int>(it % NST);
-                    if (it >= NST && !mbar_wait(&empty[s], ((it / NST) - 1) & 1, wc)) { ok = false; break; }
-                    const int t = kc / CPT;             // token offset inside the S-token group
-                    const int c0 = (kc % CPT) * 64;     // feature offset inside the token
-                    uint8_t *st = smem + s * SM::STAGE;
-                    const uint32_t fb = cluster_addr(&full[s], 0);
-                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * SM::STAGE);
-                    // A: rows R, token R*S + S-1-t; B: columns c, token c*S + t
-                    tma_load_5d_pair(st, &tmQ, fb, c0, x.h, S - 1 - t, R0, x.b);
-                    tma_load_5d_pair(st + SM::A_BYTES, &tmK, fb, c0, kvh, t, C0, x.b);
-                }
-            }
-            if (leader)
-                for (long long t2 = (it > NST ? it - NST : 0); t2 < it; ++t2)
-                    mbar_wait_drain(&full[t2 % NST], (t2 / NST) & 1, p.timeout_ns);
-        }
-    } else if (warp == 1) {
-        // ---------------------------------------------------------- MMA issuer
-        if (leader && lane == 0) {
-            const uint64_t da0 = sdesc_sw128(smem_u32(smem), 16, 1024);
-            const uint64_t db0 = sdesc_sw128(smem_u32(smem + SM::A_BYTES), 16, 1024);
-            long long it = 0;
-            long long local = 0;
-            bool ok = true;
-            for (long long u = pair_id; u < p.num_units && ok; u += num_pairs, ++local) {
-                const int acc = static_cast<int>(local & 1);
-                if (local >= 2 && !mbar_wait(&acc_empty[acc], ((local >> 1) - 1) & 1, wc)) break;
-                tc_fence_after();
-                for (int kc = 0; kc < KC; ++kc, ++it) {
-                    const int s = static_cast<int>(it % NST);
-                    if (!mbar_wait(&full[s], (it / NST) & 1, wc)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint64_t off = static_cast<uint64_t>((s * SM::STAGE) >> 4);
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_ss_pair(tmem + acc * 256, da0 + off + static_cast<uint64_t>(kk * 2),
-                                     db0 + off + static_cast<uint64_t>(kk * 2), IDESC, (kc > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit_pair(&empty[s], kBoth);
-                }
-                if (ok) umma_commit_pair(&acc_full[acc], kBoth);
-            }
-        }
-        __syncwarp();
-    } else {
-        // ---------------------------------------------------------- epilogue
-        // Both CTAs: this CTA's 128 rows of the tile, from its own TMEM.
-        const int q4 = static_cast<int>(warp & 3);
-        const int row = q4 * 32 + static_cast<int>(lane);
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-        const uint32_t leader_acc_empty[2] = {cluster_addr(&acc_empty[0], 0), cluster_addr(&acc_empty[1], 0)};
-        long long local = 0;
-        for (long long u = pair_id; u < p.num_units; u += num_pairs, ++local) {
-            const XUnit x = xattn_decode_pair(p, u);
-            const int acc = static_cast<int>(local & 1);
-            if (!warp_wait(&acc_full[acc], (local >> 1) & 1, wc)) break;
-            tc_fence_after();
-            const int R = x.mt * 256 + static_cast<int>(rank) * 128 + row;  // this thread's strided row
-            const int qb = R / CPB;                                          // its query block
-            const long long bh = static_cast<long long>(x.b) * p.H + x.h;
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                uint32_t r[128];
-                __syncwarp();  // the TMEM load below is warp-collective
-                tmem_ld128(lane_base + acc * 256 + half * 128, r);
-                if (half == 1) {
-                    tc_fence_before();
-                    mbar_arrive_cluster(leader_acc_empty[acc]);  // the accumulator is in registers
-                }
-                const int C0 = x.nt * 256 + half * 128;  // first strided column of this chunk
-                if (R >= p.rows || C0 >= p.rows || (p.causal && C0 > R)) continue;
-                const int lim = min(p.causal ? R - C0 : 127, p.rows - 1 - C0);
-#pragma unroll
-                for (int j = 0; j < 128; ++j)
-                    if (j > lim) r[j] = 0xFF800000u;     // -inf
-                float m8[16];
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const uint32_t *v = r + 8 * c;
-                    m8[c] = fmax3(fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2])),
-                                  fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5])),
-                                  fmaxf(__uint_as_float(v[6]), __uint_as_float(v[7])));
-                }
-                const float mx = fmax3(fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
-                                             fmax3(m8[6], m8[7], m8[8])),
-                                       fmax3(m8[9], m8[10], m8[11]), fmax3(m8[12], m8[13], fmaxf(m8[14], m8[15])));
-                const float m2 = mx * p.c2;
-                const int ch = C0 / 128;
-                p.part_m[(bh * p.nchunk + ch) * p.rows + R] = m2;
-                // the chunk's S block sums of this row are adjacent in part_s
-                float sums[S];
-#pragma unroll
-                for (int kbl = 0; kbl < S; ++kbl) {
-                    float acc4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-                    for (int j = 0; j < CPB; ++j)
-                        acc4[j & 3] += ex2(fmaf(__uint_as_float(r[kbl * CPB + j]), p.c2, -m2));
-                    sums[kbl] = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
-                }
-                float *dst = p.part_s + (bh * p.rows + R) * p.nb + ch * S;
-                const int nvalid = min(S, (p.causal ? qb + 1 : p.nb) - ch * S);
-                if (nvalid == S && (p.nb & 3) == 0) {  // 16-byte aligned whole chunk
-#pragma unroll
-                    for (int v = 0; v < S / 4; ++v)
-                        reinterpret_cast<float4 *>(dst)[v] =
-                            make_float4(sums[4 * v], sums[4 * v + 1], sums[4 * v + 2], sums[4 * v + 3]);
-                } else {
-#pragma unroll
-                    for (int kbl = 0; kbl < S; ++kbl)
-                        if (kbl < nvalid) dst[kbl] = sums[kbl];
-                }
-            }
-        }
-    }
-
-    // ---------------------------------------------------------- teardown
-    if (warp == 1) {
-        if (leader && lane == 0) {
-            umma_commit_pair(drain, 0x1);  // every MMA of the pair has completed
-            mbar_wait_drain(drain, 0, p.timeout_ns);
-        }
-        __syncwarp();
-    }
-    tc_fence_before();
-    cluster_sync_all();  // no CTA leaves while the pair's MMAs or arrivals may touch it
-    tc_fence_after();
-    if (warp == 1) tmem_dealloc_pair(tmem, 512);
-}
-
 // ------------------------------------------------------------ selection
 struct XselParams {
     int B, H, nb, rows, nchunk;  // the stride S is the kernel's template argument

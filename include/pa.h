@@ -42,10 +42,6 @@
  *                       (default 2000; read once, at the first launch); a
  *                       wait that runs out records PA_ERR_TIMEOUT and the
  *                       kernel abandons its work.
- *   PA_XATTN_PAIR=1     (read at every call) pa_xattn_mask runs its estimate
- *                       GEMM on SM pairs (two-CTA clusters, 256x256 tiles);
- *                       the results are the same as with the default one-SM
- *                       kernel.
  */
 #ifndef PA_H
 #define PA_H

@@ -44,12 +44,8 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("pair", [False, True], ids=["one_sm", "sm_pair"])
 @pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
-def test_xattn_parity(case, pair, monkeypatch):
-    """Both estimate GEMMs: one SM per 128 x 256 tile, and the SM-pair kernel
-    (PA_XATTN_PAIR=1, 256 x 256 tiles on two SMs)."""
-    monkeypatch.setenv("PA_XATTN_PAIR", "1" if pair else "0")
+def test_xattn_parity(case):
     name, N, H, Hkv, d, S, tau, B = case
     w = synth.small_workload(seqlen=N, heads=H, kv_heads=Hkv, head_dim=d, groups=H, batch=B, needles=8,
                              seed=700 + CASES.index(case))
