@@ -14,7 +14,9 @@
 // softmax warpgroups (setmaxnreg: 2 x 128 x 208 + 128 x 88 = 384 x 168):
 //   warps 0-3  softmax of head 0, warps 4-7 softmax of head 1 (below)
 //   warp 8     TMA producer: the two Q tiles once, then K and V tiles of the
-//              listed blocks into a ring (128-byte swizzle).
+//              listed blocks into rings (128-byte swizzle).  V of tile i and K
+//              of tile i+1 share one barrier and one release, since the MMA
+//              thread needs both at the same point (PV(i), then QK(i+1)).
 //   warp 9     TMEM owner and single-thread tcgen05.mma issuer:
 //                S_t = Q_t K^T   (M=128, N=128, K=16 steps; A, B K-major smem)
 //                O_t += P_t V    (M=128, N=d,   A = P_t read from TMEM,
@@ -32,9 +34,12 @@
 // SKIP = true adds BLASST's running-max block skip (BLASST introduction and
 // 3.1): a visited block after the first whose row maxima all lie below the
 // rows' running maxima (over the blocks visited before, in ascending order)
-// by more than -log2(lambda) is dropped -- no exponentials, no P, no PV.  The
-// four warps of a head take the block-level decision by a bounded vote in
-// shared memory; the MMA warp reads it after the head's p_full barrier.
+// by more than -log2(lambda) is dropped -- no exponentials, no P, no PV, and
+// no V load: K runs ahead on a ring of its own, and the producer loads V of a
+// tile only once a head that visits it has kept it.  The four warps of a head
+// take the block-level decision by a bounded vote in shared memory; the
+// producer reads it from a tagged slot per head, the MMA warp after the
+// head's p_full barrier.
 #pragma once
 #include "sm100.cuh"
 
@@ -149,19 +154,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint8_t *sK = smem + 2 * TB;             // [KS][TB]
     uint8_t *sV = smem + (2 + KS) * TB;      // [KS][TB]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + (2 + 2 * KS) * TB);
+    // Without SKIP, k_full[g % KS] / k_empty[g % KS] carry load group g: K(0)
+    // for g = 0, then V(g-1) with K(g) (the MMA thread needs both at the same
+    // point, PV(g-1) then QK(g)), the last group V alone; v_full / v_empty are
+    // unused.  With SKIP, K and V have rings of their own (below).
     uint64_t *q_full = bars;                 // 1
     uint64_t *s_full = bars + 1;             // 2
     uint64_t *p_full = bars + 3;             // 2
-    uint64_t *o_done = bars + 5;             // 2
-    uint64_t *drain = bars + 7;              // 1
-    uint64_t *k_full = bars + 8;             // KS
-    uint64_t *k_empty = bars + 8 + KS;       // KS
-    uint64_t *v_full = bars + 8 + 2 * KS;    // KS
-    uint64_t *v_empty = bars + 8 + 3 * KS;   // KS
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8 + 4 * KS);
+    uint64_t *drain = bars + 5;              // 1: every MMA of the CTA has completed
+    uint64_t *k_full = bars + 6;             // KS
+    uint64_t *k_empty = bars + 6 + KS;       // KS
+    uint64_t *v_full = bars + 6 + 2 * KS;    // KS
+    uint64_t *v_empty = bars + 6 + 3 * KS;   // KS
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6 + 4 * KS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile uint32_t *vote = tmem_slot + 4;        // SKIP: [2 heads][4 warps] tagged votes
     volatile uint32_t *skip_flag = tmem_slot + 12;  // SKIP: [2 heads][2 tile parities]
+    volatile uint32_t *dec = tmem_slot + 16;        // SKIP: [2 heads][2 tile parities] (block << 1 | skipped)
     uint32_t *bm = reinterpret_cast<uint32_t *>(smem + (2 + 2 * KS) * TB + 512);  // [2][128] block bitmaps
 
     // ------------------------------------------------------------ work item
@@ -242,7 +251,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int t = 0; t < 2; ++t) {
             mbar_init(&s_full[t], 1);
             mbar_init(&p_full[t], 128);
-            mbar_init(&o_done[t], 1);
         }
         mbar_init(drain, 1);
         for (int s = 0; s < KS; ++s) {
@@ -254,6 +262,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         *abort_flag = 0;
         for (int x = 0; x < 8; ++x) vote[x] = 0xFFFFFFFFu;  // a tag no tile carries
         for (int x = 0; x < 4; ++x) skip_flag[x] = 0u;
+        for (int x = 0; x < 4; ++x) dec[x] = 0xFFFFFFFFu;  // a tag no block carries
         fence_mbar_init();
     }
     if (warp == kProducerWarp && lane == 0) {
@@ -284,33 +293,103 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 tma_load_4d(sQ + cc * 16384, &tmQ, q_full, cc * 64, pair[0], qb * 128, b);
                 if (pair[1] >= 0) tma_load_4d(sQ + TB + cc * 16384, &tmQ, q_full, cc * 64, pair[1], qb * 128, b);
             }
-            int issued = 0;
-            int i = 0;
-            for (int kb = next_block(bm, bm + 128, 0, words); kb >= 0;
-                 kb = next_block(bm, bm + 128, kb + 1, words), ++i) {
-                const int s = i % KS;
-                const uint32_t ph = ((i / KS) - 1) & 1;
-                if (i >= KS && !mbar_wait(&k_empty[s], ph, wc)) break;
-                mbar_arrive_expect_tx(&k_full[s], TB);
+          if constexpr (SKIP) {
+            // K runs KS tiles ahead.  V of a tile is loaded only once a head that
+            // visits it has kept it (its decision slot carries the block's tag with
+            // the skip bit clear); a tile every visiting head skips loads no V.  A
+            // head decides at most one tile ahead of this loop (its next S needs a
+            // K this loop loads after the decision), so two slots per head suffice.
+            int nk = 0, nvl = 0;  // K and V copies issued
+            int kbk = next_block(bm, bm + 128, 0, words);
+            for (; kbk >= 0 && nk < KS; kbk = next_block(bm, bm + 128, kbk + 1, words), ++nk) {
+                mbar_arrive_expect_tx(&k_full[nk], TB);
 #pragma unroll
                 for (int cc = 0; cc < D / 64; ++cc)
-                    tma_load_4d(sK + s * TB + cc * 16384, &tmK, &k_full[s], cc * 64, kvh, kb * 128, b);
-                if (i >= KS && !mbar_wait(&v_empty[s], ph, wc)) {
-                    issued = -(i + 1);  // K of tile i issued, V not
-                    break;
+                    tma_load_4d(sK + nk * TB + cc * 16384, &tmK, &k_full[nk], cc * 64, kvh, kbk * 128, b);
+            }
+            int seen_t[2] = {0, 0};  // tiles of each head passed so far
+            for (int kb = next_block(bm, bm + 128, 0, words); kb >= 0; kb = next_block(bm, bm + 128, kb + 1, words)) {
+                const bool f0 = ((bm[kb >> 5] >> (kb & 31)) & 1u) != 0u;
+                const bool f1 = ((bm[128 + (kb >> 5)] >> (kb & 31)) & 1u) != 0u;
+                bool d0 = !f0, d1 = !f1, keep = false, good = true;
+                const uint64_t t0 = globaltimer();
+                for (uint32_t it = 0; !keep && !(d0 && d1); ++it) {
+                    if (!d0) {
+                        const uint32_t v = dec[seen_t[0] & 1];
+                        if ((v >> 1) == static_cast<uint32_t>(kb)) { d0 = true; keep = keep || (v & 1u) == 0u; }
+                    }
+                    if (!d1) {
+                        const uint32_t v = dec[2 + (seen_t[1] & 1)];
+                        if ((v >> 1) == static_cast<uint32_t>(kb)) { d1 = true; keep = keep || (v & 1u) == 0u; }
+                    }
+                    if ((it & 31u) == 31u) {
+                        if (*wc.abort) { good = false; break; }
+                        if (globaltimer() - t0 > wc.timeout_ns || it > (1u << 30)) {
+                            *wc.abort = 1;
+                            flag_status(kStTimeout);
+                            good = false;
+                            break;
+                        }
+                    }
                 }
-                mbar_arrive_expect_tx(&v_full[s], TB);
+                if (!good) break;
+                seen_t[0] += f0 ? 1 : 0;
+                seen_t[1] += f1 ? 1 : 0;
+                if (keep) {
+                    const int sv = nvl % KS;
+                    if (nvl >= KS && !mbar_wait(&v_empty[sv], ((nvl / KS) - 1) & 1, wc)) break;
+                    mbar_arrive_expect_tx(&v_full[sv], TB);
 #pragma unroll
-                for (int cc = 0; cc < D / 64; ++cc)
-                    tma_load_4d(sV + s * TB + cc * 16384, &tmV, &v_full[s], cc * 64, kvh, kb * 128, b);
-                issued = i + 1;
+                    for (int cc = 0; cc < D / 64; ++cc)
+                        tma_load_4d(sV + sv * TB + cc * 16384, &tmV, &v_full[sv], cc * 64, kvh, kb * 128, b);
+                    ++nvl;
+                }
+                if (kbk >= 0) {
+                    const int sk = nk % KS;
+                    if (!mbar_wait(&k_empty[sk], ((nk / KS) - 1) & 1, wc)) break;
+                    mbar_arrive_expect_tx(&k_full[sk], TB);
+#pragma unroll
+                    for (int cc = 0; cc < D / 64; ++cc)
+                        tma_load_4d(sK + sk * TB + cc * 16384, &tmK, &k_full[sk], cc * 64, kvh, kbk * 128, b);
+                    ++nk;
+                    kbk = next_block(bm, bm + 128, kbk + 1, words);
+                }
             }
             // teardown: let every copy in flight land before the CTA exits
             mbar_wait_drain(q_full, 0, p.timeout_ns);
-            const int nk = issued >= 0 ? issued : -issued;
-            const int nv = issued >= 0 ? issued : -issued - 1;
-            for (int i = max(nk - KS, 0); i < nk; ++i) mbar_wait_drain(&k_full[i % KS], (i / KS) & 1, p.timeout_ns);
-            for (int i = max(nv - KS, 0); i < nv; ++i) mbar_wait_drain(&v_full[i % KS], (i / KS) & 1, p.timeout_ns);
+            for (int x = max(nk - KS, 0); x < nk; ++x) mbar_wait_drain(&k_full[x % KS], (x / KS) & 1, p.timeout_ns);
+            for (int x = max(nvl - KS, 0); x < nvl; ++x) mbar_wait_drain(&v_full[x % KS], (x / KS) & 1, p.timeout_ns);
+          } else {
+            // group 0 = K(0); group g >= 1 = V(g-1) and K(g); the last group V(n-1) alone.
+            // Group g uses barrier slot g % KS, K slot g % KS and V slot (g-1) % KS, which
+            // group g - KS released.
+            int kb = next_block(bm, bm + 128, 0, words);
+            int kb_v = -1;
+            int issued = 0;
+            for (int g = 0; kb >= 0 || kb_v >= 0; ++g) {
+                const int s = g % KS;
+                if (g >= KS && !mbar_wait(&k_empty[s], ((g / KS) - 1) & 1, wc)) break;
+                mbar_arrive_expect_tx(&k_full[s], (kb >= 0 ? TB : 0) + (kb_v >= 0 ? TB : 0));
+                if (kb_v >= 0) {
+                    const int sv = (g + KS - 1) % KS;
+#pragma unroll
+                    for (int cc = 0; cc < D / 64; ++cc)
+                        tma_load_4d(sV + sv * TB + cc * 16384, &tmV, &k_full[s], cc * 64, kvh, kb_v * 128, b);
+                }
+                if (kb >= 0) {
+#pragma unroll
+                    for (int cc = 0; cc < D / 64; ++cc)
+                        tma_load_4d(sK + s * TB + cc * 16384, &tmK, &k_full[s], cc * 64, kvh, kb * 128, b);
+                }
+                issued = g + 1;
+                kb_v = kb;
+                if (kb >= 0) kb = next_block(bm, bm + 128, kb + 1, words);
+            }
+            // teardown: let every copy in flight land before the CTA exits
+            mbar_wait_drain(q_full, 0, p.timeout_ns);
+            for (int g = max(issued - KS, 0); g < issued; ++g)
+                mbar_wait_drain(&k_full[g % KS], (g / KS) & 1, p.timeout_ns);
+          }
         }
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------- MMA issuer
@@ -339,7 +418,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 for (int kk = 0; kk < 8; ++kk)  // 128 keys, 16 per step
                     umma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, bv + static_cast<uint64_t>(kk * 128),
                             IDESC_PV, kk > 0 ? 1u : acc0);
-                umma_commit(&o_done[t]);
             };
             // Visit cursor: the bitmap word holding the current block, of both
             // heads, stays in registers, so shared memory is read once per 32
@@ -373,14 +451,52 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 umma_commit(&k_empty[0]);
             }
             int i = 0;
+            int nvl = 0;  // SKIP: V tiles loaded (tiles some head kept), the V ring's counter
             for (int kb = kb_first; kb >= 0 && ok; ++i) {
-                const int s = i % KS;
                 const int s1 = (i + 1) % KS;
                 uint32_t n0 = 0u, n1 = 0u;  // heads active at kb_next
                 const int kb_next = next_visit(kb, n0, n1);
                 const bool has_next = kb_next >= 0;
-                if (!mbar_wait(&v_full[s], (i / KS) & 1, wc)) break;
-                if (has_next && !mbar_wait(&k_full[s1], ((i + 1) / KS) & 1, wc)) break;
+                if constexpr (SKIP) {
+                    // K(i+1) now; V(i) only once a head has kept tile i
+                    if (has_next && !mbar_wait(&k_full[s1], ((i + 1) / KS) & 1, wc)) break;
+                    tc_fence_after();
+                    const int sv = nvl % KS;
+                    bool v_in = false;
+                    for (int t = 0; t < 2; ++t) {
+                        if (t ? c1 : c0) {
+                            int &seen = t ? seen1 : seen0;
+                            int &pv = t ? pv1 : pv0;
+                            if (!mbar_wait(&p_full[t], seen & 1, wc)) { ok = false; break; }
+                            tc_fence_after();
+                            const bool skipped = skip_flag[t * 2 + (seen & 1)] != 0u;
+                            ++seen;
+                            if (!skipped) {
+                                if (!v_in) {
+                                    if (!mbar_wait(&v_full[sv], (nvl / KS) & 1, wc)) { ok = false; break; }
+                                    tc_fence_after();
+                                    v_in = true;
+                                }
+                                issue_pv(t, sv, pv > 0);
+                                ++pv;
+                            }
+                        }
+                        if (has_next && (t ? n1 : n0)) issue_qk(t, s1);
+                    }
+                    if (!ok) break;
+                    if (v_in) {
+                        umma_commit(&v_empty[sv]);
+                        ++nvl;
+                    }
+                    if (has_next) umma_commit(&k_empty[s1]);
+                    kb = kb_next;
+                    c0 = n0;
+                    c1 = n1;
+                    continue;
+                }
+                const int s = i % KS;
+                // load group i+1: V(i) and, with a next tile, K(i+1)
+                if (!mbar_wait(&k_full[s1], ((i + 1) / KS) & 1, wc)) break;
                 tc_fence_after();
                 for (int t = 0; t < 2; ++t) {
                     if (t ? c1 : c0) {
@@ -388,23 +504,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         int &pv = t ? pv1 : pv0;
                         if (!mbar_wait(&p_full[t], seen & 1, wc)) { ok = false; break; }
                         tc_fence_after();
-                        if constexpr (SKIP) {
-                            const bool skipped = skip_flag[t * 2 + (seen & 1)] != 0u;
-                            ++seen;
-                            if (!skipped) {
-                                issue_pv(t, s, pv > 0);
-                                ++pv;
-                            }
-                        } else {
-                            issue_pv(t, s, seen > 0);  // without skipping every tile has its PV
-                            ++seen;
-                        }
+                        issue_pv(t, s, seen > 0);  // without skipping every tile has its PV
+                        ++seen;
+                        (void)pv;
                     }
                     if (has_next && (t ? n1 : n0)) issue_qk(t, s1);
                 }
                 if (!ok) break;
-                umma_commit(&v_empty[s]);
-                if (has_next) umma_commit(&k_empty[s1]);
+                umma_commit(&k_empty[s1]);  // load group i+1 consumed
                 kb = kb_next;
                 c0 = n0;
                 c1 = n1;
@@ -433,7 +540,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         bool ok = true;
         uint32_t s[128];
         int i = 0;    // tiles of this head so far
-        int npv = 0;  // of them, tiles whose PV product was issued (o_done phases)
+        int npv = 0;  // of them, tiles whose PV product was issued
         for (int kb = next_block(bmt, bmt, 0, words); kb >= 0; kb = next_block(bmt, bmt, kb + 1, words), ++i) {
             if (!warp_wait(&s_full[t], i & 1, wc)) { ok = false; break; }
             tc_fence_after();
@@ -465,7 +572,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     if (!vote_ok) { ok = false; break; }
                 }
                 mtrue = fmaxf(mtrue, mt);
-                if (row == 0) skip_flag[t * 2 + (i & 1)] = skip ? 1u : 0u;
+                if (row == 0) {
+                    skip_flag[t * 2 + (i & 1)] = skip ? 1u : 0u;
+                    dec[t * 2 + (i & 1)] = (static_cast<uint32_t>(kb) << 1) | (skip ? 1u : 0u);
+                }
                 if (skip) {
                     // nothing of this tile enters O or l; S is free for the next QK
                     if (row == 0 && p.skipped) p.skipped[skip_base + kb] = 1;
@@ -480,7 +590,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (__any_sync(0xffffffffu, need)) {
                     // raise the running max: O (in TMEM) and l scale by 2^(m - m_new)
                     const float alpha = (m == -INFINITY) ? 0.0f : ex2(m - m_new);
-                    if (!warp_wait(&o_done[t], ((SKIP ? npv : i) - 1) & 1, wc)) { ok = false; break; }
+                    // (this tile's S was committed after the head's last PV was issued,
+                    // and a commit covers every earlier MMA, so that PV is complete)
                     tc_fence_after();
 #pragma unroll
                     for (int ch = 0; ch < D / 32; ++ch) {
@@ -542,7 +653,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         // epilogue: O / l -> bf16 -> global; LSE
         const int ct = SKIP ? npv : i;
-        if (ct > 0 && ok && warp_wait(&o_done[t], (ct - 1) & 1, wc)) {
+        if (ct > 0 && ok && warp_wait(drain, 0, wc)) {
             tc_fence_after();
             const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
             __nv_bfloat16 *orow = p.o + b * p.osb + static_cast<int64_t>(qb * 128 + row) * p.oss + h * p.osh;
