@@ -25,7 +25,6 @@
 //                       shortest prefix whose estimates reach tau in 2^-40
 //                       fixed point (find_blocks).
 #pragma once
-#include <cub/block/block_radix_sort.cuh>
 
 #include "sm100.cuh"
 
@@ -359,28 +358,42 @@ __device__ __forceinline__ void bitonic_sort_256(unsigned long long *keys) {
     __syncthreads();
 }
 
-// The sort of 1024 or 2048 keys: a stable LSD radix sort (CUB's
-// BlockRadixSort, 4-bit digits) of the upper 32 bits, the descending-estimate
-// code, with the lower 32 bits, the block index, carried along as values.
-// Thread t hands in entries t*E .. t*E+E-1, i.e. the keys in block-index
-// order, and gets back the same positions of the sorted sequence.  A stable
-// sort leaves equal estimates in index order, so the result is the ascending
-// order of the whole 64-bit keys, as the bitonic network produces.  Shorter
-// rows keep the bitonic network, which is faster there (eight radix passes
-// with block-wide scans cost more than the shuffle stages for 256 keys).
-template <int E>
-using XselRadixSort = cub::BlockRadixSort<uint32_t, 256, E, uint32_t>;
+// The sort of 1024 or 2048 keys: a stable LSD radix sort of the upper 32
+// bits, the descending-estimate code, four bits per pass, with the lower 32
+// bits, the block index, carried along.  Thread t holds entries t*E ..
+// t*E+E-1 (the keys start in block-index order).  A pass:
+//   1. each thread counts its keys per digit in two packed words (4 bits per
+//      digit, E <= 8 keys) and writes the 16 counts to cnt[digit][thread];
+//   2. one exclusive scan over cnt in (digit, thread) order gives each
+//      thread the first output position of its keys of each digit;
+//   3. each thread scatters its keys, in its own order, to those positions.
+// Positions follow (digit, thread, key) order, so the pass is stable, and a
+// stable LSD sort leaves equal estimates in index order: the result is the
+// ascending order of the whole 64-bit keys, as the bitonic network produces.
+// A pass whose digit is the same for every key would not move any and is
+// skipped.  Shorter rows keep the bitonic network, which is faster there.
+constexpr int kXselRadixBits = 4;
+constexpr int kXselDigits = 1 << kXselRadixBits;
 
-// Shared memory the selection kernel needs beyond its P keys for the sort.
+// Shared memory the selection kernel needs beyond its P keys for the sort:
+// the per-(digit, thread) counts and the eight warps' scan totals.
 __host__ __device__ constexpr size_t xsel_sort_temp_bytes(int P) {
-    return P == 1024   ? sizeof(typename XselRadixSort<4>::TempStorage)
-           : P == 2048 ? sizeof(typename XselRadixSort<8>::TempStorage)
-                       : 0;
+    return (P == 1024 || P == 2048) ? (kXselDigits * 256 + 8) * sizeof(uint32_t) : 0;
+}
+
+// count field of digit d in the packed pair (lo: digits 0-7, hi: 8-15)
+__device__ __forceinline__ uint32_t xsel_field(uint32_t lo, uint32_t hi, uint32_t d) {
+    return ((d < 8 ? lo : hi) >> (4 * (d & 7))) & 15u;
 }
 
 template <int E>
 __device__ __forceinline__ void radix_sort_keys(unsigned long long *keys, void *temp) {
+    static_assert(E <= 8, "4-bit packed counts hold at most 15 keys per digit");
+    constexpr int P = 256 * E;
+    uint32_t *cnt = reinterpret_cast<uint32_t *>(temp);  // [kXselDigits][256]
+    uint32_t *wsum = cnt + kXselDigits * 256;           // [8]
     const int tid = static_cast<int>(threadIdx.x);
+    const int lane = tid & 31, warp = tid >> 5;
     uint32_t k[E], v[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) {
@@ -388,11 +401,65 @@ __device__ __forceinline__ void radix_sort_keys(unsigned long long *keys, void *
         k[e] = static_cast<uint32_t>(x >> 32);
         v[e] = static_cast<uint32_t>(x);
     }
-    XselRadixSort<E>(*reinterpret_cast<typename XselRadixSort<E>::TempStorage *>(temp)).Sort(k, v);
-    __syncthreads();  // every thread's reads of the keys are done
+    for (int shift = 0; shift < 32; shift += kXselRadixBits) {
+        // a pass that would not move any key is skipped (the whole CTA agrees)
+        const uint32_t ref = static_cast<uint32_t>(keys[0] >> (32 + shift)) & (kXselDigits - 1);
+        bool same = true;
 #pragma unroll
-    for (int e = 0; e < E; ++e) keys[tid * E + e] = (static_cast<unsigned long long>(k[e]) << 32) | v[e];
-    __syncthreads();
+        for (int e = 0; e < E; ++e) same = same && ((k[e] >> shift) & (kXselDigits - 1)) == ref;
+        if (__syncthreads_and(same)) continue;
+        // 1. this thread's counts per digit
+        uint32_t lo = 0, hi = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const uint32_t d = (k[e] >> shift) & (kXselDigits - 1);
+            if (d < 8) lo += 1u << (4 * d); else hi += 1u << (4 * (d - 8));
+        }
+#pragma unroll
+        for (int d = 0; d < kXselDigits; ++d) cnt[d * 256 + tid] = xsel_field(lo, hi, d);
+        __syncthreads();
+        // 2. exclusive scan of the 4096 counts in (digit, thread) order: thread
+        // t scans the 16 consecutive counts at 16t, the warps' totals are
+        // scanned through shared memory
+        uint32_t c[kXselDigits];
+        uint32_t run = 0;
+#pragma unroll
+        for (int x = 0; x < kXselDigits; ++x) {
+            c[x] = run;
+            run += cnt[tid * kXselDigits + x];
+        }
+        uint32_t incl = run;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        uint32_t base = incl - run;
+        for (int w = 0; w < warp; ++w) base += wsum[w];
+#pragma unroll
+        for (int x = 0; x < kXselDigits; ++x) cnt[tid * kXselDigits + x] = base + c[x];
+        __syncthreads();
+        // 3. scatter: the first free position of each digit of this thread
+        uint32_t seen_lo = 0, seen_hi = 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const uint32_t d = (k[e] >> shift) & (kXselDigits - 1);
+            const uint32_t pos = cnt[d * 256 + tid] + xsel_field(seen_lo, seen_hi, d);
+            if (d < 8) seen_lo += 1u << (4 * d); else seen_hi += 1u << (4 * (d - 8));
+            keys[pos] = (static_cast<unsigned long long>(k[e]) << 32) | v[e];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const unsigned long long x = keys[tid * E + e];
+            k[e] = static_cast<uint32_t>(x >> 32);
+            v[e] = static_cast<uint32_t>(x);
+        }
+        __syncthreads();  // every thread has read its keys before the next pass writes
+    }
+    (void)P;
 }
 
 // One CTA of 256 threads per (b, h, qb), long rows first; dynamic shared
