@@ -103,17 +103,28 @@ __global__ void __launch_bounds__(256, 2) pool_heads_kernel(PoolParams p) {
         for (int t = 0; t < 8; ++t)
             if (t < nv) kvv[t] = __ldg(reinterpret_cast<const uint4 *>(krow + (v0 + t) * p.ksh));
         if (!q_done) {
-            // q heads in blocks of 6: all 16-byte loads of a block in flight
-            // before the first add, the adds in ascending head order
-            for (int t0 = 0; t0 < hpg; t0 += 6) {
-                const int n = min(6, hpg - t0);
-                uint4 qv[6];
+            // q heads in blocks of 4, software-pipelined: the next block's
+            // 16-byte loads are in flight while this block is added (adds in
+            // ascending head order)
+            constexpr int QB = 4;
+            uint4 qa[QB], qb2[QB];
+            auto load_blk = [&](uint4 (&dst)[QB], int t0) {
 #pragma unroll
-                for (int t = 0; t < 6; ++t)
-                    if (t < n) qv[t] = __ldg(reinterpret_cast<const uint4 *>(qrow + (h0 + t0 + t) * p.qsh));
+                for (int t = 0; t < QB; ++t)
+                    if (t0 + t < hpg) dst[t] = __ldg(reinterpret_cast<const uint4 *>(qrow + (h0 + t0 + t) * p.qsh));
+            };
+            auto add_blk = [&](const uint4 (&src)[QB], int t0) {
 #pragma unroll
-                for (int t = 0; t < 6; ++t)
-                    if (t < n) add_bf16x8(aq, qv[t]);
+                for (int t = 0; t < QB; ++t)
+                    if (t0 + t < hpg) add_bf16x8(aq, src[t]);
+            };
+            load_blk(qa, 0);
+            for (int t0 = 0; t0 < hpg; t0 += 2 * QB) {
+                if (t0 + QB < hpg) load_blk(qb2, t0 + QB);
+                add_blk(qa, t0);
+                if (t0 + QB >= hpg) break;
+                if (t0 + 2 * QB < hpg) load_blk(qa, t0 + 2 * QB);
+                add_blk(qb2, t0 + QB);
             }
             q_done = true;
         }
