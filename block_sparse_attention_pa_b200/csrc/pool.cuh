@@ -86,48 +86,44 @@ __global__ void __launch_bounds__(256, 2) pool_heads_kernel(PoolParams p) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) aq[j] = ak[j] = 0.0;
 
-    // The k proxy adds, for every q head h of the group in ascending order, the
-    // row of its KV head v(h) = h * Hkv / H; v(h) does not decrease with h, so
-    // each KV row is converted to fp64 once and added once per q head reading
-    // it, which is the same sequence of additions.  The distinct KV rows of
-    // the group are loaded first (up to 8 per pass) and the q heads are summed
-    // while those loads are in flight.
+    // The q heads first, in blocks of 8, software-pipelined: the next block's
+    // 16-byte loads are in flight while this block is added (adds in ascending
+    // head order).  Then the k proxy: for every q head h of the group in
+    // ascending order it adds the row of its KV head v(h) = h * Hkv / H; v(h)
+    // does not decrease with h, so each KV row is converted to fp64 once and
+    // added once per q head reading it, which is the same sequence of
+    // additions.  The group's distinct KV rows are loaded up to 8 per pass.
     const int hend = h0 + hpg;
     const int v_lo = static_cast<int>(static_cast<int64_t>(h0) * p.Hkv / p.H);
     const int v_hi = static_cast<int>(static_cast<int64_t>(hend - 1) * p.Hkv / p.H);
-    bool q_done = !doq;
+    if (doq) {
+        constexpr int QB = 8;
+        uint4 qa[QB], qb2[QB];
+        auto load_blk = [&](uint4 (&dst)[QB], int t0) {
+#pragma unroll
+            for (int t = 0; t < QB; ++t)
+                if (t0 + t < hpg) dst[t] = __ldg(reinterpret_cast<const uint4 *>(qrow + (h0 + t0 + t) * p.qsh));
+        };
+        auto add_blk = [&](const uint4 (&src)[QB], int t0) {
+#pragma unroll
+            for (int t = 0; t < QB; ++t)
+                if (t0 + t < hpg) add_bf16x8(aq, src[t]);
+        };
+        load_blk(qa, 0);
+        for (int t0 = 0; t0 < hpg; t0 += 2 * QB) {
+            if (t0 + QB < hpg) load_blk(qb2, t0 + QB);
+            add_blk(qa, t0);
+            if (t0 + QB >= hpg) break;
+            if (t0 + 2 * QB < hpg) load_blk(qa, t0 + 2 * QB);
+            add_blk(qb2, t0 + QB);
+        }
+    }
     for (int v0 = v_lo; v0 <= v_hi; v0 += 8) {
         const int nv = min(8, v_hi - v0 + 1);
         uint4 kvv[8];
 #pragma unroll
         for (int t = 0; t < 8; ++t)
             if (t < nv) kvv[t] = __ldg(reinterpret_cast<const uint4 *>(krow + (v0 + t) * p.ksh));
-        if (!q_done) {
-            // q heads in blocks of 4, software-pipelined: the next block's
-            // 16-byte loads are in flight while this block is added (adds in
-            // ascending head order)
-            constexpr int QB = 4;
-            uint4 qa[QB], qb2[QB];
-            auto load_blk = [&](uint4 (&dst)[QB], int t0) {
-#pragma unroll
-                for (int t = 0; t < QB; ++t)
-                    if (t0 + t < hpg) dst[t] = __ldg(reinterpret_cast<const uint4 *>(qrow + (h0 + t0 + t) * p.qsh));
-            };
-            auto add_blk = [&](const uint4 (&src)[QB], int t0) {
-#pragma unroll
-                for (int t = 0; t < QB; ++t)
-                    if (t0 + t < hpg) add_bf16x8(aq, src[t]);
-            };
-            load_blk(qa, 0);
-            for (int t0 = 0; t0 < hpg; t0 += 2 * QB) {
-                if (t0 + QB < hpg) load_blk(qb2, t0 + QB);
-                add_blk(qa, t0);
-                if (t0 + QB >= hpg) break;
-                if (t0 + 2 * QB < hpg) load_blk(qa, t0 + 2 * QB);
-                add_blk(qb2, t0 + QB);
-            }
-            q_done = true;
-        }
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
             if (t < nv) {
