@@ -194,19 +194,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int kvh = kv_of_cta;
     const int hk = static_cast<int>((static_cast<long long>(kvh) * p.H + p.Hkv - 1) / p.Hkv);
     const int nh = static_cast<int>((static_cast<long long>(kvh + 1) * p.H + p.Hkv - 1) / p.Hkv) - hk;
+    // An odd head count leaves the last unit of a query block one head.  Such
+    // lone units of two consecutive query blocks share one CTA, slot 0 taking
+    // query block qb and slot 1 qb - 1 (their lists overlap as much as two rows
+    // of one ranking do), so that two chains keep the tensor core busy: the
+    // unit at qb with nb-1-qb even takes both, the one at the other parity has
+    // no work.  qbt[t] is slot t's query block.
+    const bool lone = (nh & 1) != 0 && j == (nh >> 1);
+    if (lone && ((p.nb - 1 - qb) & 1) != 0) return;  // taken by the CTA of qb + 1 (whole CTA, before any sync)
+    const bool lone_pair = lone && qb > 0;
     __shared__ int pair_heads[2];
-    if (static_cast<int>(threadIdx.x) < nh) {
-        const int32_t *cq = p.cnt + (static_cast<long long>(b) * p.H + hk) * p.nb + qb;
-        const int me = static_cast<int>(threadIdx.x);
-        const int32_t c_me = cq[static_cast<long long>(me) * p.nb];
-        int r = 0;
-        for (int y = 0; y < nh; ++y) {
-            const int32_t c_y = cq[static_cast<long long>(y) * p.nb];
-            r += (c_y < c_me || (c_y == c_me && y < me)) ? 1 : 0;
+    for (int t = 0; t < (lone_pair ? 2 : 1); ++t) {
+        const int qx = qb - t;
+        if (static_cast<int>(threadIdx.x) < nh) {
+            const int32_t *cq = p.cnt + (static_cast<long long>(b) * p.H + hk) * p.nb + qx;
+            const int me = static_cast<int>(threadIdx.x);
+            const int32_t c_me = cq[static_cast<long long>(me) * p.nb];
+            int r = 0;
+            for (int y = 0; y < nh; ++y) {
+                const int32_t c_y = cq[static_cast<long long>(y) * p.nb];
+                r += (c_y < c_me || (c_y == c_me && y < me)) ? 1 : 0;
+            }
+            if (lone) {
+                if (r == nh - 1) pair_heads[t] = hk + me;  // the lone head of query block qx
+            } else if ((r >> 1) == j) {
+                pair_heads[r & 1] = hk + me;
+            }
         }
-        if ((r >> 1) == j) pair_heads[r & 1] = hk + me;
     }
-    if (threadIdx.x == 0 && 2 * j + 1 >= nh) pair_heads[1] = -1;  // an odd head count leaves the last unit one head
+    if (threadIdx.x == 0 && 2 * j + 1 >= nh && !lone_pair) pair_heads[1] = -1;  // one head, one slot
     // The selected blocks of each head as a bitmap over 0..qb: head t takes the
     // first c[t] entries of its list.  Every role then visits them in
     // ascending block order (the result does not depend on the order), so the
@@ -218,26 +234,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const volatile int *pair = pair_heads;
     const int h0 = pair[0];
     const int h1 = pair[1];
+    const int qbt[2] = {qb, lone_pair ? qb - 1 : qb};
     const long long T = p.causal ? static_cast<long long>(p.nb) * (p.nb + 1) / 2 : static_cast<long long>(p.nb) * p.nb;
-    const long long row_off = p.causal ? static_cast<long long>(qb) * (qb + 1) / 2 : static_cast<long long>(qb) * p.nb;
-    const int row_len = p.causal ? qb + 1 : p.nb;  // blocks in this query block's list
+    auto row_off_of = [&](int x) -> long long {
+        return p.causal ? static_cast<long long>(x) * (x + 1) / 2 : static_cast<long long>(x) * p.nb;
+    };
+    const int row_len = p.causal ? qb + 1 : p.nb;  // blocks in slot 0's list (slot 1's is no longer)
+    const int row_len1 = p.causal ? qbt[1] + 1 : p.nb;
     const int32_t *list0 =
-        p.rank + (static_cast<long long>(b) * p.G + static_cast<long long>(h0) * p.G / p.H) * T + row_off;
+        p.rank + (static_cast<long long>(b) * p.G + static_cast<long long>(h0) * p.G / p.H) * T + row_off_of(qbt[0]);
     const int32_t *list1 =
         p.rank + (static_cast<long long>(b) * p.G + static_cast<long long>(h1 >= 0 ? h1 : h0) * p.G / p.H) * T +
-        row_off;
+        row_off_of(qbt[1]);
     int craw[2];
-    craw[0] = p.cnt[(static_cast<long long>(b) * p.H + h0) * p.nb + qb];
-    craw[1] = (h1 >= 0) ? p.cnt[(static_cast<long long>(b) * p.H + h1) * p.nb + qb] : 0;
+    craw[0] = p.cnt[(static_cast<long long>(b) * p.H + h0) * p.nb + qbt[0]];
+    craw[1] = (h1 >= 0) ? p.cnt[(static_cast<long long>(b) * p.H + h1) * p.nb + qbt[1]] : 0;
     int c[2];
-    for (int t = 0; t < 2; ++t) c[t] = min(max(craw[t], 0), row_len);
+    c[0] = min(max(craw[0], 0), row_len);
+    c[1] = min(max(craw[1], 0), row_len1);
     const int ntiles = (h1 >= 0) ? 2 : 1;
-    const int words = (row_len + 31) >> 5;  // bitmap words covering the row's blocks
+    const int words = (row_len + 31) >> 5;  // bitmap words covering both slots' blocks
 
     for (int x = threadIdx.x; x < c[0] + c[1]; x += blockDim.x) {
         const int t = (x < c[0]) ? 0 : 1;
         const int kb = t ? list1[x - c[0]] : list0[x];
-        if (kb < 0 || kb >= row_len) {
+        if (kb < 0 || kb >= (t ? row_len1 : row_len)) {
             flag_status(kStBounds);
             continue;
         }
@@ -290,8 +311,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_arrive_expect_tx(q_full, ntiles * TB);
 #pragma unroll
             for (int cc = 0; cc < D / 64; ++cc) {
-                tma_load_4d(sQ + cc * 16384, &tmQ, q_full, cc * 64, pair[0], qb * 128, b);
-                if (pair[1] >= 0) tma_load_4d(sQ + TB + cc * 16384, &tmQ, q_full, cc * 64, pair[1], qb * 128, b);
+                tma_load_4d(sQ + cc * 16384, &tmQ, q_full, cc * 64, pair[0], qbt[0] * 128, b);
+                if (pair[1] >= 0) tma_load_4d(sQ + TB + cc * 16384, &tmQ, q_full, cc * 64, pair[1], qbt[1] * 128, b);
             }
           if constexpr (SKIP) {
             // K runs KS tiles ahead.  V of a tile is loaded only once a head that
@@ -528,7 +549,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // ---------------------------------------------------------- softmax
         const int t = static_cast<int>(warp >> 2);
         const int h = (t && pair[1] >= 0) ? pair[1] : pair[0];  // an unpaired unit's second warpgroup has no blocks
-        const long long skip_base = (static_cast<long long>(b) * p.H + h) * T + row_off;
+        const int qbs = qbt[t];  // this slot's query block
+        const long long skip_base = (static_cast<long long>(b) * p.H + h) * T + row_off_of(qbs);
         const uint32_t *bmt = bm + t * 128;
         const int q4 = static_cast<int>(warp & 3);
         const int row = q4 * 32 + static_cast<int>(lane);
@@ -544,7 +566,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int kb = next_block(bmt, bmt, 0, words); kb >= 0; kb = next_block(bmt, bmt, kb + 1, words), ++i) {
             if (!warp_wait(&s_full[t], i & 1, wc)) { ok = false; break; }
             tc_fence_after();
-            const bool masked = p.causal && kb == qb;  // the causal diagonal tile: same for the whole CTA
+            const bool masked = p.causal && kb == qbs;  // the causal diagonal tile: same for the whole warpgroup
             tmem_ld128(s_addr, s);
             if (masked) {
 #pragma unroll
@@ -656,7 +678,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (ct > 0 && ok && warp_wait(drain, 0, wc)) {
             tc_fence_after();
             const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
-            __nv_bfloat16 *orow = p.o + b * p.osb + static_cast<int64_t>(qb * 128 + row) * p.oss + h * p.osh;
+            __nv_bfloat16 *orow = p.o + b * p.osb + static_cast<int64_t>(qbs * 128 + row) * p.oss + h * p.osh;
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
                 uint32_t r[32];
@@ -672,7 +694,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 dst[3] = make_uint4(w[12], w[13], w[14], w[15]);
             }
             if (p.lse)
-                p.lse[(static_cast<long long>(b) * p.H + h) * p.N + qb * 128 + row] =
+                p.lse[(static_cast<long long>(b) * p.H + h) * p.N + qbs * 128 + row] =
                     (m + log2f(l)) * 0.69314718055994531f;
         }
     }
