@@ -79,7 +79,8 @@ def parse_args():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
-                    help="skip the extra configurations of the 128K layer (G = 4, fixed 10 %%, logit units)")
+                    help="skip the extra configurations (the 128K layer at G = 4, fixed 10 %%, logit units; "
+                         "the 32K, Qwen 64K and 256K workloads)")
     return ap.parse_args()
 
 
@@ -823,7 +824,9 @@ def run_extras(w, x, gamma, dense_ms, peak, dist_on, local, rank):
                     attention speed-up over dense;
       logit_units   the labelled logit-unit input, where per-head dynamic
                     budgets differ (two heads of a CTA keep different prefixes
-                    of their list)."""
+                    of their list);
+      configs       the method's other workloads on their own inputs
+                    (run_other_configs)."""
     out = {}
     q, k, v = x["q"], x["k"], x["v"]
     H = w.num_q_heads
@@ -858,6 +861,54 @@ def run_extras(w, x, gamma, dense_ms, peak, dist_on, local, rank):
     out["logit_units"]["workload"] = wl.name
     del xl
     torch.cuda.empty_cache()
+    out["configs"] = run_other_configs(gamma, peak, dist_on, local, rank)
+    return out
+
+
+# The other workloads of the method's configs, timed in the default run: the
+# 32K Llama layer, the Qwen 64K layer at G = 4, and the 256K sweep's ends.
+OTHER_CONFIGS = [
+    ("llama8b_n32k", None, 0, 0),
+    ("qwen7b_n64k", None, 0, 0),
+    ("llama8b_n256k", 0.8, 0, 0),
+    ("llama8b_n256k", None, 1, 50),
+]
+
+
+def run_other_configs(gamma_default, peak, dist_on, local, rank):
+    """Each workload on its own inputs: 3 timed steps of the whole path and 2 of
+    the dense (every causal block) attention of the same kernel."""
+    out = {}
+    for name, gamma, mode, frac in OTHER_CONFIGS:
+        w = synth.WORKLOADS[name]
+        g = w.gamma if gamma is None else gamma
+        x = synth.make_inputs(w, device=f"cuda:{local}", seed=w.seed + rank)
+        pipe = Pipeline(x["q"], x["k"], x["v"], w.num_groups, mode, g, frac)
+        sampler = ClockSampler(local) if rank == 0 else None
+        _, stages, clocks = time_pipeline(pipe, 3, 2, dist_on, sampler)
+        vis, flops, _ = pipe.visited()
+        est, attn = float(stages[:3].sum()), float(stages[3])
+        del pipe
+        dense = Pipeline(x["q"], x["k"], x["v"], w.num_groups, 2, g, frac)
+        _, dstages, _ = time_pipeline(dense, 2, 1, dist_on)
+        dense_ms = float(dstages[3])
+        nb = w.nb
+        tf = flops / (attn * 1e-3) / 1e12
+        key = f"{name}_" + (f"gamma{g}" if mode == 0 else f"fixed{frac / 10:g}pct")
+        r = {"groups": w.num_groups,
+             "budget": f"dynamic gamma={g}" if mode == 0 else f"fixed {frac / 10:.1f}% of causal blocks",
+             "layer_ms": est + attn, "est_ms": est, "attn_ms": attn, "attn_tflops": tf,
+             "attn_frac_of_sustained": tf / peak, "density": vis / (w.batch * w.num_q_heads * nb * (nb + 1) // 2),
+             "dense_attn_ms": dense_ms, "speedup_vs_dense": dense_ms / attn, "estimate_frac_of_dense": est / dense_ms,
+             "steps": 3}
+        busy = tensor_busy(flops, attn, clocks, x["q"].device)
+        if busy is not None:
+            r["tensor_busy"] = busy
+            r["sm_mhz"] = clocks["sm_mhz"]
+            r["clock_reasons"] = clocks["reasons"]
+        out[key] = r
+        del dense, x
+        torch.cuda.empty_cache()
     return out
 
 
