@@ -410,20 +410,24 @@ def tensor_busy(flops: float, ms: float, clocks, device):
     return flops / (TENSOR_FLOP_PER_CLK_SM * sms * ms * 1e-3 * clocks["sm_mhz"] * 1e6)
 
 
-def counters_for(kernel_key: str, source_files):
+def sources_sha256(source_files) -> str:
+    h = hashlib.sha256()
+    for s in source_files:
+        with open(os.path.join(ROOT, s), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def counters_for(kernel_key: str, source_files, path=None):
     """DRAM bytes of a kernel from a committed ncu summary, if the kernel's
     sources still hash to what was profiled; else None."""
-    p = os.path.join(ROOT, "profiles", "counters.json")
+    p = path or os.path.join(ROOT, "profiles", "counters.json")
     try:
         with open(p) as f:
             c = json.load(f)[kernel_key]
     except Exception:
         return None
-    h = hashlib.sha256()
-    for s in source_files:
-        with open(os.path.join(ROOT, s), "rb") as f:
-            h.update(f.read())
-    if h.hexdigest() != c.get("source_sha256"):
+    if sources_sha256(source_files) != c.get("source_sha256"):
         return None
     return c
 
