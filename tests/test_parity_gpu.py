@@ -78,6 +78,11 @@ CASES = [
     # paired heads (one KV head) that follow different lists: G = H under GQA
     ("gqa_g_eq_h_pairs",  768,  8, 2,  64, 8, pa.DYNAMIC,   0.9,  0,   1),
     ("gqa_g4_pairs_d128", 640,  8, 2, 128, 4, pa.FIXED_FRACTION, 0, 400, 1),
+    # odd head counts per KV head: the lone units of query blocks qb and qb-1
+    # share a CTA (odd and even nb, a single block, MHA where every unit is lone)
+    ("lone_single_block", 128,  3, 1,  64, 1, pa.DYNAMIC,   0.9,  0,   1),
+    ("lone_mha_nb3",      384,  2, 2, 128, 2, pa.DYNAMIC,   0.9,  0,   1),
+    ("lone_g5_nb6_b2",    768, 10, 2,  64, 2, pa.FIXED_FRACTION, 0, 500, 2),
 ]
 
 
