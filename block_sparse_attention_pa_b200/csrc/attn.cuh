@@ -522,12 +522,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 for (int t = 0; t < 2; ++t) {
                     if (t ? c1 : c0) {
                         int &seen = t ? seen1 : seen0;
-                        int &pv = t ? pv1 : pv0;
                         if (!mbar_wait(&p_full[t], seen & 1, wc)) { ok = false; break; }
                         tc_fence_after();
                         issue_pv(t, s, seen > 0);  // without skipping every tile has its PV
                         ++seen;
-                        (void)pv;
                     }
                     if (has_next && (t ? n1 : n0)) issue_qk(t, s1);
                 }
