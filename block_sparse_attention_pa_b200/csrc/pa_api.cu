@@ -14,6 +14,8 @@
 #include <mutex>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "pa.h"
 #include "attn.cuh"
 #include "mask.cuh"
@@ -49,6 +51,29 @@ pa_status ok() {
 constexpr int kBlk = 128;
 constexpr int kMaxNb = 4096;
 constexpr int kScoreChunk = 16;  // tiles per score/mass work unit
+
+// NVTX ranges around every launch (and around pa_prefill and
+// pa_prefill_varlen as a whole) when PA_NVTX=1, for profilers that group
+// kernels by range; off by default (read once, at the first call).
+bool nvtx_on() {
+    static const bool v = [] {
+        const char *e = getenv("PA_NVTX");
+        return e && e[0] == '1';
+    }();
+    return v;
+}
+
+struct Trace {
+    bool on;
+    explicit Trace(const char *name) : on(nvtx_on()) {
+        if (on) nvtxRangePushA(name);
+    }
+    ~Trace() {
+        if (on) nvtxRangePop();
+    }
+    Trace(const Trace &) = delete;
+    Trace &operator=(const Trace &) = delete;
+};
 
 uint64_t wait_timeout_ns() {
     static uint64_t v = [] {
@@ -261,6 +286,7 @@ pa_status check_xstride(int S) {
 // ------------------------------------------------------------- launches
 pa_status launch_pool(const pa_shape *s, int stride, const void *q, pa_strides qs, const void *k, pa_strides ks,
                       void *qp, void *kp, cudaStream_t st) {
+    Trace tr_("pa.pool_heads");
     pa::PoolParams p;
     p.q = static_cast<const __nv_bfloat16 *>(q);
     p.k = static_cast<const __nv_bfloat16 *>(k);
@@ -293,6 +319,7 @@ pa_status launch_tile_gemm_t(const CUtensorMap &a, const CUtensorMap &b, const p
 
 pa_status launch_scores(const pa_shape *s, int stride, const void *qp, const void *kp, float *scores,
                         cudaStream_t st) {
+    Trace tr_("pa.block_scores");
     const int B = s->batch, G = s->num_groups, N = s->seqlen, d = s->head_dim, nb = N / kBlk;
     CUtensorMap ma, mb;
     pa_status r = map_proxy(&ma, qp, B, G, N / stride, d, "q_proxy");
@@ -324,6 +351,7 @@ pa_status launch_scores(const pa_shape *s, int stride, const void *qp, const voi
 
 pa_status launch_mass(const pa_shape *s, const void *q, pa_strides qs, const void *k, pa_strides ks, float2 *partial,
                       float *mass, cudaStream_t st) {
+    Trace tr_("pa.head_mass");
     const int B = s->batch, H = s->num_q_heads, Hkv = s->num_kv_heads, N = s->seqlen, d = s->head_dim;
     const int nb = N / kBlk;
     CUtensorMap ma, mb;
@@ -350,6 +378,7 @@ pa_status launch_mass(const pa_shape *s, const void *q, pa_strides qs, const voi
 }
 
 pa_status launch_rank(const pa_shape *s, const float *scores, int32_t *rank, cudaStream_t st) {
+    Trace tr_("pa.rank");
     const int nb = s->seqlen / kBlk;
     int P = 1;
     while (P < nb - 1) P <<= 1;
@@ -363,6 +392,7 @@ pa_status launch_rank(const pa_shape *s, const float *scores, int32_t *rank, cud
 
 pa_status launch_budget(const pa_shape *s, const pa_budget *bu, const int32_t *rank, const float *mass, int32_t *cnt,
                         int32_t *budget, cudaStream_t st) {
+    Trace tr_("pa.budget");
     pa::BudgetParams p;
     p.B = s->batch; p.H = s->num_q_heads; p.G = s->num_groups; p.nb = s->seqlen / kBlk;
     p.mode = bu->mode; p.gamma = bu->gamma; p.frac_permille = bu->frac_permille;
@@ -396,6 +426,7 @@ pa_status launch_xattn_gemm_d(int S, const CUtensorMap &mq, const CUtensorMap &m
 
 pa_status launch_xattn(const pa_shape *s, int S, float tau, const void *q, pa_strides qs, const void *k,
                        pa_strides ks, int32_t *rank, int32_t *cnt, float *mass, void *ws, cudaStream_t st) {
+    Trace tr_("pa.xattn_mask");
     const int B = s->batch, H = s->num_q_heads, Hkv = s->num_kv_heads, N = s->seqlen, d = s->head_dim;
     const int nb = N / kBlk, rows = N / S;
     CUtensorMap mq, mk;
@@ -485,6 +516,7 @@ pa_status launch_attn_t(const CUtensorMap &mq, const CUtensorMap &mk, const CUte
 pa_status launch_attn(const pa_shape *s, const void *q, pa_strides qs, const void *k, pa_strides ks, const void *v,
                       pa_strides vs, const int32_t *rank, const int32_t *cnt, float scale, void *o, pa_strides os,
                       float *lse, float skip_threshold, uint8_t *skipped, cudaStream_t st) {
+    Trace tr_("pa.block_sparse_attn");
     const int B = s->batch, H = s->num_q_heads, Hkv = s->num_kv_heads, N = s->seqlen, d = s->head_dim;
     CUtensorMap mq, mk, mv;
     pa_status r = map_bnhd(&mq, q, B, N, H, d, qs, "q");
@@ -712,6 +744,7 @@ pa_status pa_prefill(const pa_shape *shape, const pa_budget *budget, const void 
     if (!ws || ws_bytes < w.total)
         return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, w.total);
     if ((r = check_ptr(ws, "workspace", 256))) return r;
+    Trace tr_("pa.prefill");
     if ((r = run_prefill(shape, budget, q, qs, k, ks, v, vs, o, os, mask_out, ws,
                          reinterpret_cast<cudaStream_t>(stream))))
         return r;
@@ -746,6 +779,7 @@ pa_status pa_prefill_varlen(const pa_shape *shape, const pa_budget *budget, int3
     if ((r = check_ptr(ws, "workspace", 256))) return r;
     const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int G = shape->num_groups, H = shape->num_q_heads;
+    Trace tr_("pa.prefill_varlen");
     int64_t rows_off = 0, blk_off = 0;  // sums of T_s and nb_s over the sequences before
     for (int s = 0; s < num_seqs; ++s) {
         pa_shape one = *shape;

@@ -42,6 +42,13 @@
  *                       (default 2000; read once, at the first launch); a
  *                       wait that runs out records PA_ERR_TIMEOUT and the
  *                       kernel abandons its work.
+ *   PA_NVTX=1           (read once) every launch, and pa_prefill /
+ *                       pa_prefill_varlen as a whole, is wrapped in an NVTX
+ *                       range named after its stage ("pa.pool_heads",
+ *                       "pa.block_scores", "pa.head_mass", "pa.rank",
+ *                       "pa.budget", "pa.block_sparse_attn", "pa.xattn_mask",
+ *                       "pa.prefill", "pa.prefill_varlen") for profilers that
+ *                       group kernels by range.  Off by default.
  */
 #ifndef PA_H
 #define PA_H
