@@ -200,11 +200,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // of one ranking do), so that two chains keep the tensor core busy: the
     // unit at qb with nb-1-qb even takes both, the one at the other parity has
     // no work.  qbt[t] is slot t's query block.
-    const bool lone = (nh & 1) != 0 && j == (nh >> 1);
+    //
+    // With the block skip, every unit is one head at query blocks qb and qb - 1
+    // (one unit per head, units_per_kv = the heads of a KV head): a tile saves
+    // time only when both slots skip it, and one head's decisions on the blocks
+    // of two adjacent rows agree far more often than two heads' decisions do.
+    const bool lone = SKIP || ((nh & 1) != 0 && j == (nh >> 1));
     if (lone && ((p.nb - 1 - qb) & 1) != 0) return;  // taken by the CTA of qb + 1 (whole CTA, before any sync)
     const bool lone_pair = lone && qb > 0;
     __shared__ int pair_heads[2];
-    for (int t = 0; t < (lone_pair ? 2 : 1); ++t) {
+    if constexpr (SKIP) {
+        if (threadIdx.x == 0) {
+            pair_heads[0] = hk + j;
+            pair_heads[1] = lone_pair ? hk + j : -1;
+        }
+    }
+    for (int t = 0; t < (SKIP ? 0 : (lone_pair ? 2 : 1)); ++t) {
         const int qx = qb - t;
         if (static_cast<int>(threadIdx.x) < nh) {
             const int32_t *cq = p.cnt + (static_cast<long long>(b) * p.H + hk) * p.nb + qx;
@@ -222,7 +233,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
         }
     }
-    if (threadIdx.x == 0 && 2 * j + 1 >= nh && !lone_pair) pair_heads[1] = -1;  // one head, one slot
+    if (!SKIP && threadIdx.x == 0 && 2 * j + 1 >= nh && !lone_pair) pair_heads[1] = -1;  // one head, one slot
     // The selected blocks of each head as a bitmap over 0..qb: head t takes the
     // first c[t] entries of its list.  Every role then visits them in
     // ascending block order (the result does not depend on the order), so the

@@ -475,18 +475,18 @@ pa_status launch_xattn(const pa_shape *s, int S, float tau, const void *q, pa_st
     return PA_OK;
 }
 
-// Head units of the attention kernel: pairs of consecutive q heads that share
-// their KV head (so they share one K/V stream; each follows its own group's
-// ranked list); a head left over forms a unit alone.
-// Head units of every KV head: its q heads h with h * Hkv / H == kv, two per
-// unit (the kernel pairs them by row count); returns the largest count.
-int build_units(const pa_shape *s, int16_t *kv_units) {
+// Head units of every KV head: its q heads h with h * Hkv / H == kv share one
+// K/V stream.  Without the block skip two heads per unit (the kernel pairs them
+// by row count; a head left over forms a unit whose CTA takes two query
+// blocks); with the skip one head per unit (its CTA takes two query blocks).
+// Returns the largest count.
+int build_units(const pa_shape *s, int16_t *kv_units, bool one_head_per_unit) {
     const int H = s->num_q_heads, Hkv = s->num_kv_heads;
     int most = 0;
     for (int kv = 0; kv < Hkv; ++kv) {
         const long long first = (static_cast<long long>(kv) * H + Hkv - 1) / Hkv;
         const long long next = (static_cast<long long>(kv + 1) * H + Hkv - 1) / Hkv;
-        const int units = static_cast<int>((next - first + 1) / 2);
+        const int units = static_cast<int>(one_head_per_unit ? next - first : (next - first + 1) / 2);
         kv_units[kv] = static_cast<int16_t>(units);
         most = std::max(most, units);
     }
@@ -525,7 +525,8 @@ pa_status launch_attn(const pa_shape *s, const void *q, pa_strides qs, const voi
     if ((r = map_bnhd(&mv, v, B, N, Hkv, d, vs, "v"))) return r;
     pa::AttnParams p{};
     p.B = B; p.N = N; p.H = H; p.Hkv = Hkv; p.G = s->num_groups; p.nb = N / kBlk;
-    p.units_per_kv = build_units(s, p.kv_units);
+    const bool skip = skip_threshold > 0.0f;
+    p.units_per_kv = build_units(s, p.kv_units, skip);
     p.rank = rank; p.cnt = cnt;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.o = static_cast<__nv_bfloat16 *>(o);
@@ -533,7 +534,6 @@ pa_status launch_attn(const pa_shape *s, const void *q, pa_strides qs, const voi
     p.lse = lse;
     p.causal = causal_of(s) ? 1 : 0;
     p.timeout_ns = wait_timeout_ns();
-    const bool skip = skip_threshold > 0.0f;
     p.skip_log2 = skip ? static_cast<float>(std::log2(static_cast<double>(skip_threshold))) : -INFINITY;
     p.skipped = skip ? skipped : nullptr;
     if (skip)
