@@ -72,3 +72,58 @@ def test_noalloc_matches_workspace_entry_point_twice():
         assert torch.equal(got.budget, ref.budget), f"call {call}: budget"
         mg, mr = got.mass.cpu().numpy(), ref.mass.cpu().numpy()
         assert np.all(np.abs(mg - mr) <= 2e-5 + 2e-3 * np.abs(mr)), f"call {call}: mass"
+
+
+@pytest.mark.gpu
+def test_noalloc_under_cuda_graph_capture():
+    """After one eager call on the device (which looks up the scratch address),
+    the entry point records into a CUDA graph: capture it on a side stream,
+    replay the graph on new inputs copied into the captured buffers, and
+    compare with an eager call on the same inputs bit for bit."""
+    f = _noalloc()
+    G, gamma = 2, 0.9
+    w = synth.small_workload(seqlen=1536, heads=8, kv_heads=2, head_dim=128, groups=G, gamma=gamma, seed=21)
+    x = synth.make_inputs(w, device="cuda")
+    q, k = x["q"].clone(), x["k"].clone()
+    shape = pa.make_shape(q, k, G)
+    budget = pa.make_budget(pa.DYNAMIC, gamma)
+
+    def call(scores, out, stream):
+        bufs = out.bufs()
+        r = f(ctypes.byref(shape), ctypes.byref(budget), scores.data_ptr(), q.data_ptr(), pa._strides(q),
+              k.data_ptr(), pa._strides(k), ctypes.byref(bufs), stream)
+        assert r == 0, pa.lib().pa_last_error()
+
+    qp, kp = pa.pool_heads(q, k, G)
+    scores = pa.block_scores(qp, kp, 8, 2)
+    warm = pa.Mask.empty(shape, q.device, True)
+    call(scores, warm, pa._stream(q.device))
+    torch.cuda.synchronize()
+
+    captured = pa.Mask.empty(shape, q.device, True)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            call(scores, captured, side.cuda_stream)
+    torch.cuda.synchronize()
+
+    # new inputs into the captured buffers, then replay
+    x2 = synth.make_inputs(synth.small_workload(seqlen=1536, heads=8, kv_heads=2, head_dim=128, groups=G,
+                                                gamma=gamma, seed=22), device="cuda")
+    q.copy_(x2["q"])
+    k.copy_(x2["k"])
+    qp2, kp2 = pa.pool_heads(q, k, G)
+    scores.copy_(pa.block_scores(qp2, kp2, 8, 2))
+    g.replay()
+    torch.cuda.synchronize()
+    eager = pa.Mask.empty(shape, q.device, True)
+    call(scores, eager, pa._stream(q.device))
+    torch.cuda.synchronize()
+    assert pa.device_status() == 0
+    assert torch.equal(captured.rank, eager.rank)
+    assert torch.equal(captured.cnt, eager.cnt)
+    assert torch.equal(captured.budget, eager.budget)
+    assert torch.equal(captured.mass, eager.mass)
+    del g
