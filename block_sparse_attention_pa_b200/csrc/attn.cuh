@@ -180,60 +180,107 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int U = p.units_per_kv;
     const int j = static_cast<int>(blockIdx.x % U);
     long long rest = blockIdx.x / U;
-    const int qb = p.nb - 1 - static_cast<int>(rest % p.nb);
+    const int qb_grid = p.nb - 1 - static_cast<int>(rest % p.nb);
     rest /= p.nb;
     const int kv_of_cta = static_cast<int>(rest % p.Hkv);
     const int b = static_cast<int>(rest / p.Hkv);
     if (j >= p.kv_units[kv_of_cta]) return;  // this KV head has fewer units (whole CTA, before any sync)
-    // The q heads of this KV head, [hk, hk + nh), are paired by their row counts
-    // for this query block: ranked by (cnt, head) and unit j takes ranks 2j and
-    // 2j+1.  Heads of one proxy group visit prefixes of the same list, so a pair
-    // with close counts shares most of its K/V tiles and both heads are busy on
-    // them.  Every CTA of (b, kv, qb) ranks the same counts the same way, so the
-    // units cover each head once.
     const int kvh = kv_of_cta;
     const int hk = static_cast<int>((static_cast<long long>(kvh) * p.H + p.Hkv - 1) / p.Hkv);
     const int nh = static_cast<int>((static_cast<long long>(kvh + 1) * p.H + p.Hkv - 1) / p.Hkv) - hk;
-    // An odd head count leaves the last unit of a query block one head.  Such
-    // lone units of two consecutive query blocks share one CTA, slot 0 taking
-    // query block qb and slot 1 qb - 1 (their lists overlap as much as two rows
-    // of one ranking do), so that two chains keep the tensor core busy: the
-    // unit at qb with nb-1-qb even takes both, the one at the other parity has
-    // no work.  qbt[t] is slot t's query block.
+    // The CTAs of query blocks qtop and qtop - 1 (qtop at an even distance from
+    // the last block) sit next to each other in the grid and split the 2 * nh
+    // (head, query block) items of this KV head between them in one of two ways:
     //
-    // With the block skip, every unit is one head at query blocks qb and qb - 1
-    // (one unit per head, units_per_kv = the heads of a KV head): a tile saves
-    // time only when both slots skip it, and one head's decisions on the blocks
-    // of two adjacent rows agree far more often than two heads' decisions do.
-    const bool lone = SKIP || ((nh & 1) != 0 && j == (nh >> 1));
-    if (lone && ((p.nb - 1 - qb) & 1) != 0) return;  // taken by the CTA of qb + 1 (whole CTA, before any sync)
-    const bool lone_pair = lone && qb > 0;
+    // by count: per query block, the heads ranked by (cnt, head), unit j taking
+    //   ranks 2j and 2j+1.  Heads of one proxy group visit prefixes of the same
+    //   list, so a pair with close counts shares most of its K/V tiles and both
+    //   heads are busy on them.  An odd head count leaves the last unit of a
+    //   query block one head; such lone units of the two query blocks share the
+    //   CTA of qtop (slot 0 at qtop, slot 1 at qtop - 1), and the lone unit at
+    //   qtop - 1 has no work.
+    // by head: each CTA takes one head at qtop (slot 0) and qtop - 1 (slot 1):
+    //   two rows of one ranking with nearly equal budgets, whose lists overlap
+    //   in most blocks even when the heads of the KV head have very different
+    //   budgets (where pairs by count leave many tiles to one slot alone).
+    //
+    // Both CTAs choose the same way from the counts of both query blocks: by
+    // head when the sum over heads of the larger of a head's two counts, plus
+    // 2 % for the blocks only one of the two rows keeps, is below the tiles of
+    // the pairs by count (the larger count of each pair, and the larger of the
+    // two lone heads' counts).  With the block skip every unit is one head at
+    // qtop and qtop - 1 (one unit per head, units_per_kv = the heads of a KV
+    // head): a tile saves time only when both slots skip it, and one head's
+    // decisions on the blocks of two adjacent rows agree far more often than
+    // two heads' decisions do.  qbt[t] is slot t's query block.
+    const bool upper = ((p.nb - 1 - qb_grid) & 1) == 0;
+    const int qtop = upper ? qb_grid : qb_grid + 1;
     __shared__ int pair_heads[2];
-    if constexpr (SKIP) {
+    __shared__ int pair_cost[3];  // by count (pairs), by head, by count (the lone heads)
+    bool by_head = SKIP;
+    if constexpr (!SKIP) {
+        if (qtop > 0) {  // uniform over the CTA
+            if (threadIdx.x < 3) pair_cost[threadIdx.x] = 0;
+            __syncthreads();
+            if (static_cast<int>(threadIdx.x) < nh) {
+                const int me = static_cast<int>(threadIdx.x);
+                int c_me[2];
+                for (int t = 0; t < 2; ++t) {
+                    const int qx = qtop - t;
+                    const int len = p.causal ? qx + 1 : p.nb;
+                    const int32_t *cq = p.cnt + (static_cast<long long>(b) * p.H + hk) * p.nb + qx;
+                    c_me[t] = min(max(static_cast<int>(cq[static_cast<long long>(me) * p.nb]), 0), len);
+                    int r = 0;
+                    for (int y = 0; y < nh; ++y) {
+                        const int c_y = min(max(static_cast<int>(cq[static_cast<long long>(y) * p.nb]), 0), len);
+                        r += (c_y < c_me[t] || (c_y == c_me[t] && y < me)) ? 1 : 0;
+                    }
+                    if ((nh & 1) != 0 && r == nh - 1)
+                        atomicMax(&pair_cost[2], c_me[t]);
+                    else if ((r & 1) != 0)
+                        atomicAdd(&pair_cost[0], c_me[t]);
+                }
+                atomicAdd(&pair_cost[1], max(c_me[0], c_me[1]));
+            }
+            __syncthreads();
+            by_head = 50LL * pair_cost[1] < 49LL * (static_cast<long long>(pair_cost[0]) + pair_cost[2]);
+        }
+    }
+    int qb = qb_grid;  // slot 0's query block
+    bool lone_pair;    // slot 1 takes query block qb - 1
+    if (by_head) {
+        const int x = SKIP ? (upper ? j : nh) : (upper ? 0 : static_cast<int>(p.kv_units[kvh])) + j;
+        if (x >= nh) return;  // no head left for this CTA (the whole CTA returns)
+        qb = qtop;
+        lone_pair = qtop > 0;
         if (threadIdx.x == 0) {
-            pair_heads[0] = hk + j;
-            pair_heads[1] = lone_pair ? hk + j : -1;
+            pair_heads[0] = hk + x;
+            pair_heads[1] = lone_pair ? hk + x : -1;
         }
-    }
-    for (int t = 0; t < (SKIP ? 0 : (lone_pair ? 2 : 1)); ++t) {
-        const int qx = qb - t;
-        if (static_cast<int>(threadIdx.x) < nh) {
-            const int32_t *cq = p.cnt + (static_cast<long long>(b) * p.H + hk) * p.nb + qx;
-            const int me = static_cast<int>(threadIdx.x);
-            const int32_t c_me = cq[static_cast<long long>(me) * p.nb];
-            int r = 0;
-            for (int y = 0; y < nh; ++y) {
-                const int32_t c_y = cq[static_cast<long long>(y) * p.nb];
-                r += (c_y < c_me || (c_y == c_me && y < me)) ? 1 : 0;
-            }
-            if (lone) {
-                if (r == nh - 1) pair_heads[t] = hk + me;  // the lone head of query block qx
-            } else if ((r >> 1) == j) {
-                pair_heads[r & 1] = hk + me;
+    } else {
+        const bool lone = (nh & 1) != 0 && j == (nh >> 1);
+        if (lone && !upper) return;  // taken by the CTA of qtop (the whole CTA returns)
+        lone_pair = lone && qb > 0;
+        for (int t = 0; t < (lone_pair ? 2 : 1); ++t) {
+            const int qx = qb - t;
+            if (static_cast<int>(threadIdx.x) < nh) {
+                const int32_t *cq = p.cnt + (static_cast<long long>(b) * p.H + hk) * p.nb + qx;
+                const int me = static_cast<int>(threadIdx.x);
+                const int32_t c_me = cq[static_cast<long long>(me) * p.nb];
+                int r = 0;
+                for (int y = 0; y < nh; ++y) {
+                    const int32_t c_y = cq[static_cast<long long>(y) * p.nb];
+                    r += (c_y < c_me || (c_y == c_me && y < me)) ? 1 : 0;
+                }
+                if (lone) {
+                    if (r == nh - 1) pair_heads[t] = hk + me;  // the lone head of query block qx
+                } else if ((r >> 1) == j) {
+                    pair_heads[r & 1] = hk + me;
+                }
             }
         }
+        if (threadIdx.x == 0 && 2 * j + 1 >= nh && !lone_pair) pair_heads[1] = -1;  // one head, one slot
     }
-    if (!SKIP && threadIdx.x == 0 && 2 * j + 1 >= nh && !lone_pair) pair_heads[1] = -1;  // one head, one slot
     // The selected blocks of each head as a bitmap over 0..qb: head t takes the
     // first c[t] entries of its list.  Every role then visits them in
     // ascending block order (the result does not depend on the order), so the
