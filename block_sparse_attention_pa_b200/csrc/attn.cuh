@@ -13,7 +13,8 @@
 // columns).  At the start the third warpgroup hands registers to the two
 // softmax warpgroups (setmaxnreg: 2 x 128 x 208 + 128 x 88 = 384 x 168):
 //   warps 0-3  softmax of head 0, warps 4-7 softmax of head 1 (below)
-//   warp 8     TMA producer: the two Q tiles once, then K and V tiles of the
+//   warp 8     TMA producer: the two Q tiles (issued before the CTA's setup
+//              barrier, so the copy overlaps the setup), then K and V tiles of the
 //              listed blocks into rings (128-byte swizzle).  V of tile i and K
 //              of tile i+1 share one barrier and one release, since the MMA
 //              thread needs both at the same point (PV(i), then QK(i+1)).
@@ -313,19 +314,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int ntiles = (h1 >= 0) ? 2 : 1;
     const int words = (row_len + 31) >> 5;  // bitmap words covering both slots' blocks
 
-    for (int x = threadIdx.x; x < c[0] + c[1]; x += blockDim.x) {
-        const int t = (x < c[0]) ? 0 : 1;
-        const int kb = t ? list1[x - c[0]] : list0[x];
-        if (kb < 0 || kb >= (t ? row_len1 : row_len)) {
-            flag_status(kStBounds);
-            continue;
-        }
-        atomicOr(&bm[t * 128 + (kb >> 5)], 1u << (kb & 31));
-    }
-
     const uint32_t warp = warp_id(), lane = lane_id();
-    if (threadIdx.x == 0) {
-        if (c[0] != craw[0] || (h1 >= 0 && c[1] != craw[1])) flag_status(kStBounds);
+    if (warp == kProducerWarp && lane == 0) {
+        // The barriers, then the two Q tiles at once: their copy overlaps the
+        // bitmap build, the TMEM allocation and the CTA barrier below.  No other
+        // thread touches a barrier before that CTA barrier.
         mbar_init(q_full, 1);
         for (int t = 0; t < 2; ++t) {
             mbar_init(&s_full[t], 1);
@@ -343,12 +336,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int x = 0; x < 4; ++x) skip_flag[x] = 0u;
         for (int x = 0; x < 4; ++x) dec[x] = 0xFFFFFFFFu;  // a tag no block carries
         fence_mbar_init();
-    }
-    if (warp == kProducerWarp && lane == 0) {
         tma_prefetch_desc(&tmQ);
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
+        mbar_arrive_expect_tx(q_full, ntiles * TB);
+#pragma unroll
+        for (int cc = 0; cc < D / 64; ++cc) {
+            tma_load_4d(sQ + cc * 16384, &tmQ, q_full, cc * 64, h0, qbt[0] * 128, b);
+            if (h1 >= 0) tma_load_4d(sQ + TB + cc * 16384, &tmQ, q_full, cc * 64, h1, qbt[1] * 128, b);
+        }
     }
+
+    for (int x = threadIdx.x; x < c[0] + c[1]; x += blockDim.x) {
+        const int t = (x < c[0]) ? 0 : 1;
+        const int kb = t ? list1[x - c[0]] : list0[x];
+        if (kb < 0 || kb >= (t ? row_len1 : row_len)) {
+            flag_status(kStBounds);
+            continue;
+        }
+        atomicOr(&bm[t * 128 + (kb >> 5)], 1u << (kb & 31));
+    }
+
+    if (threadIdx.x == 0 && (c[0] != craw[0] || (h1 >= 0 && c[1] != craw[1]))) flag_status(kStBounds);
     if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
@@ -365,13 +374,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       reg_release<kRegsAux>();
       if (warp == kProducerWarp) {
         // ---------------------------------------------------------- producer
-        if (lane == 0) {
-            mbar_arrive_expect_tx(q_full, ntiles * TB);
-#pragma unroll
-            for (int cc = 0; cc < D / 64; ++cc) {
-                tma_load_4d(sQ + cc * 16384, &tmQ, q_full, cc * 64, pair[0], qbt[0] * 128, b);
-                if (pair[1] >= 0) tma_load_4d(sQ + TB + cc * 16384, &tmQ, q_full, cc * 64, pair[1], qbt[1] * 128, b);
-            }
+        if (lane == 0) {  // (the Q tiles are already on their way)
           if constexpr (SKIP) {
             // K runs KS tiles ahead.  V of a tile is loaded only once a head that
             // visits it has kept it (its decision slot carries the block's tag with
