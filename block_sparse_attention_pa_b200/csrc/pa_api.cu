@@ -297,10 +297,23 @@ pa_status launch_pool(const pa_shape *s, int stride, const void *q, pa_strides q
     p.B = s->batch; p.N = s->seqlen; p.H = s->num_q_heads; p.Hkv = s->num_kv_heads;
     p.G = s->num_groups; p.d = s->head_dim;
     p.stride = stride;
-    const long long threads = static_cast<long long>(p.B) * p.N * p.G * (p.d / 8);
-    const unsigned grid = static_cast<unsigned>((threads + 255) / 256);
-    if (p.d == 128) pa::pool_heads_kernel<128><<<grid, 256, 0, st>>>(p);
-    else pa::pool_heads_kernel<64><<<grid, 256, 0, st>>>(p);
+    // one thread per 8 head-dim elements of one (batch, token, group): x over
+    // tokens, y over groups, z over the batch (in launches of at most 65535
+    // sequences, the grid's z limit)
+    const int B = p.B;
+    constexpr int kMaxZ = 65535;
+    for (int b0 = 0; b0 < B; b0 += kMaxZ) {
+        pa::PoolParams pc = p;
+        pc.B = std::min(kMaxZ, B - b0);
+        pc.q = p.q + static_cast<int64_t>(b0) * p.qsb;
+        pc.k = p.k + static_cast<int64_t>(b0) * p.ksb;
+        pc.qp = p.qp + static_cast<int64_t>(b0) * p.G * (p.N / stride) * p.d;
+        pc.kp = p.kp + static_cast<int64_t>(b0) * p.G * p.N * p.d;
+        const dim3 grid(static_cast<unsigned>((static_cast<long long>(p.N) * (p.d / 8) + 255) / 256),
+                        static_cast<unsigned>(p.G), static_cast<unsigned>(pc.B));
+        if (p.d == 128) pa::pool_heads_kernel<128><<<grid, 256, 0, st>>>(pc);
+        else pa::pool_heads_kernel<64><<<grid, 256, 0, st>>>(pc);
+    }
     PA_CUDA(cudaGetLastError());
     return PA_OK;
 }

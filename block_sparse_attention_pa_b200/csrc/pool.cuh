@@ -66,15 +66,13 @@ __device__ __forceinline__ uint4 mean_to_bf16x8(const double (&acc)[8], int n) {
 template <int D>
 __global__ void __launch_bounds__(256, 2) pool_heads_kernel(PoolParams p) {
     constexpr int TPR = D / 8;  // threads per (token, group) row
-    const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const int64_t rows = static_cast<int64_t>(p.B) * p.N * p.G;
-    const int64_t row = gid / TPR;
-    if (row >= rows) return;
-    const int c = static_cast<int>(gid % TPR) * 8;
-    const int g = static_cast<int>(row % p.G);
-    const int64_t bi = row / p.G;  // b * N + i
-    const int i = static_cast<int>(bi % p.N);
-    const int b = static_cast<int>(bi / p.N);
+    // grid (tokens * TPR / 256, G, B): no runtime division in the index math
+    const uint32_t t = blockIdx.x * blockDim.x + threadIdx.x;
+    const int i = static_cast<int>(t / TPR);
+    if (i >= p.N) return;
+    const int c = static_cast<int>(t % TPR) * 8;
+    const int g = static_cast<int>(blockIdx.y);
+    const int b = static_cast<int>(blockIdx.z);
 
     const int hpg = p.H / p.G;
     const int h0 = g * hpg;

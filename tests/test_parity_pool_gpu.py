@@ -83,3 +83,22 @@ def test_pool_strided_bit_exact_wide_range(r):
     _, _, qpb, kpb = oracle.pool(q, k, 2)
     assert same_bits(qp, qpb[:, :, r - 1::r])
     assert same_bits(kp, kpb)
+
+
+def test_pool_batch_beyond_one_launch():
+    """More sequences than one launch's grid holds along the batch axis
+    (65535): the rest go to a second launch with offset pointers.  With one q
+    head per group the q proxy of a row is that head's row and the k proxy the
+    row of the KV head it reads, so the whole output is known exactly."""
+    B, N, H, Hkv, d = 65537, 128, 2, 1, 64
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(5)
+    q = torch.randn(B, N, H, d, device="cuda", dtype=torch.bfloat16, generator=gen)
+    k = torch.randn(B, N, Hkv, d, device="cuda", dtype=torch.bfloat16, generator=gen)
+    qp, kp = pa.pool_heads(q, k, H)
+    torch.cuda.synchronize()
+    assert pa.device_status(clear=True) == 0
+    assert torch.equal(qp, q.permute(0, 2, 1, 3))
+    assert torch.equal(kp, k.permute(0, 2, 1, 3).expand(B, H, N, d))
+    del q, k, qp, kp
+    torch.cuda.empty_cache()
