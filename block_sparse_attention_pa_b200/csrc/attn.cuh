@@ -2,12 +2,12 @@
 // the block-sparse mask "fed to FlashAttention", end of "4. ProxyAttn
 // method"; the attention formula of "2. Background").
 //
-// One CTA computes one query block (128 rows) of one or two heads that share
-// a KV head.  Head t visits the first cnt_t entries of its proxy group's
-// ranked list (two heads of one group share the list); a K/V tile is loaded
-// once for both heads whenever either needs it.  The heads of a KV head are
-// paired per query block by their row counts (ranked by (cnt, head)), so the
-// two heads of a CTA share most of their tiles even when budgets differ.
+// One CTA computes two (q head, query block) items of one KV head, one per
+// slot: two heads at one query block, or one head at two adjacent query
+// blocks (the work decode below chooses from the counts).  The item of slot t
+// visits the first cnt entries of its row of its proxy group's ranked list;
+// a K/V tile is loaded once for both slots whenever either needs it, so the
+// pairing aims at two items that share most of their tiles.
 //
 // Warp roles (384 threads = three warpgroups, one CTA per SM, all 512 TMEM
 // columns).  At the start the third warpgroup hands registers to the two

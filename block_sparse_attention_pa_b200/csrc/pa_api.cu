@@ -489,10 +489,11 @@ pa_status launch_xattn(const pa_shape *s, int S, float tau, const void *q, pa_st
 }
 
 // Head units of every KV head: its q heads h with h * Hkv / H == kv share one
-// K/V stream.  Without the block skip two heads per unit (the kernel pairs them
-// by row count; a head left over forms a unit whose CTA takes two query
-// blocks); with the skip one head per unit (its CTA takes two query blocks).
-// Returns the largest count.
+// K/V stream.  Without the block skip ceil(heads / 2) units per query block: the
+// kernel's CTAs of two adjacent query blocks pair the heads by row count per
+// query block (a head left over at both forms one unit of two query blocks) or
+// take one head at both query blocks each; with the skip one head per unit
+// (its CTA takes two query blocks).  Returns the largest count.
 int build_units(const pa_shape *s, int16_t *kv_units, bool one_head_per_unit) {
     const int H = s->num_q_heads, Hkv = s->num_kv_heads;
     int most = 0;
