@@ -64,7 +64,7 @@ __device__ __forceinline__ uint4 mean_to_bf16x8(const double (&acc)[8], int n) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(256, 2) pool_heads_kernel(PoolParams p) {
+__global__ void __launch_bounds__(256, 3) pool_heads_kernel(PoolParams p) {
     constexpr int TPR = D / 8;  // threads per (token, group) row
     // grid (tokens * TPR / 256, G, B): no runtime division in the index math
     const uint32_t t = blockIdx.x * blockDim.x + threadIdx.x;
@@ -84,18 +84,20 @@ __global__ void __launch_bounds__(256, 2) pool_heads_kernel(PoolParams p) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) aq[j] = ak[j] = 0.0;
 
-    // The q heads first, in blocks of 8, software-pipelined: the next block's
+    // The q heads first, in blocks of 4, software-pipelined: the next block's
     // 16-byte loads are in flight while this block is added (adds in ascending
     // head order).  Then the k proxy: for every q head h of the group in
     // ascending order it adds the row of its KV head v(h) = h * Hkv / H; v(h)
     // does not decrease with h, so each KV row is converted to fp64 once and
     // added once per q head reading it, which is the same sequence of
-    // additions.  The group's distinct KV rows are loaded up to 8 per pass.
+    // additions.  The group's distinct KV rows are loaded up to 4 per pass
+    // (small blocks keep the kernel at 80 registers, three CTAs per SM).
+    constexpr int KB = 4;  // KV rows loaded per pass
     const int hend = h0 + hpg;
     const int v_lo = static_cast<int>(static_cast<int64_t>(h0) * p.Hkv / p.H);
     const int v_hi = static_cast<int>(static_cast<int64_t>(hend - 1) * p.Hkv / p.H);
     if (doq) {
-        constexpr int QB = 8;
+        constexpr int QB = 4;
         uint4 qa[QB], qb2[QB];
         auto load_blk = [&](uint4 (&dst)[QB], int t0) {
 #pragma unroll
@@ -116,14 +118,14 @@ __global__ void __launch_bounds__(256, 2) pool_heads_kernel(PoolParams p) {
             add_blk(qb2, t0 + QB);
         }
     }
-    for (int v0 = v_lo; v0 <= v_hi; v0 += 8) {
-        const int nv = min(8, v_hi - v0 + 1);
-        uint4 kvv[8];
+    for (int v0 = v_lo; v0 <= v_hi; v0 += KB) {
+        const int nv = min(KB, v_hi - v0 + 1);
+        uint4 kvv[KB];
 #pragma unroll
-        for (int t = 0; t < 8; ++t)
+        for (int t = 0; t < KB; ++t)
             if (t < nv) kvv[t] = __ldg(reinterpret_cast<const uint4 *>(krow + (v0 + t) * p.ksh));
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
+        for (int t = 0; t < KB; ++t) {
             if (t < nv) {
                 const int v = v0 + t;
                 // q heads reading KV head v: [ceil(v H / Hkv), ceil((v+1) H / Hkv)) within the group
