@@ -199,7 +199,7 @@ def test_strided_packed_qkv():
     assert o_buf[:, :, :2].abs().max().item() == 0 and o_buf[:, :, 6:].abs().max().item() == 0
 
 
-def pairs_by_head(cnt, b, hk, nh, qtop, nb):
+def pairs_by_head(cnt, b, hk, nh, qtop, nb, causal=True):
     """The kernel's choice for the CTAs of query blocks qtop and qtop - 1 of
     one KV head (a scheduling model, not method arithmetic): True when each
     CTA takes one head at both query blocks, False when heads are paired by
@@ -208,24 +208,28 @@ def pairs_by_head(cnt, b, hk, nh, qtop, nb):
         return False
     pairs = lone = 0
     for qx in (qtop, qtop - 1):
-        c = np.clip(cnt[b, hk:hk + nh, qx], 0, qx + 1)
+        c = np.clip(cnt[b, hk:hk + nh, qx], 0, qx + 1 if causal else nb)
         order = sorted(range(nh), key=lambda y: (c[y], y))
         for r, y in enumerate(order):
             if nh % 2 and r == nh - 1:
                 lone = max(lone, int(c[y]))
             elif r % 2:
                 pairs += int(c[y])
-    top = np.clip(cnt[b, hk:hk + nh, qtop], 0, qtop + 1)
-    low = np.clip(cnt[b, hk:hk + nh, qtop - 1], 0, qtop)
+    top = np.clip(cnt[b, hk:hk + nh, qtop], 0, qtop + 1 if causal else nb)
+    low = np.clip(cnt[b, hk:hk + nh, qtop - 1], 0, qtop if causal else nb)
     by_head = int(np.maximum(top, low).sum())
     return 50 * by_head < 49 * (pairs + lone)
 
 
 PAIRING_CASES = [
-    # name,          N,    H, Hkv, d,  B
-    ("nh4_nb10",     1280, 8, 2, 128, 1),
-    ("nh3_nb9_odd",  1152, 6, 2,  64, 1),
-    ("nh5_nb8_b2",   1024, 10, 2, 64, 2),
+    # name,               N,    H, Hkv, d,  B, G, causal
+    ("nh4_nb10",          1280, 8, 2, 128, 1, 1, True),
+    ("nh3_nb9_odd",       1152, 6, 2,  64, 1, 1, True),
+    ("nh5_nb8_b2",        1024, 10, 2, 64, 2, 1, True),
+    # the heads of a KV head in two proxy groups (two lists per KV head)
+    ("nh4_g4_two_lists",  1280, 8, 2, 128, 1, 4, True),
+    # non-causal rows: every block of the row can be listed
+    ("nh4_noncausal",     1152, 8, 2,  64, 1, 1, False),
 ]
 
 
@@ -236,22 +240,21 @@ def test_attention_under_both_head_pairings(case):
     head at both query blocks) and others equal budgets (heads paired by
     count): O and LSE of every (batch, head, query block) against the oracle
     with the same lists."""
-    name, N, H, Hkv, d, B = case
-    G = 1
+    name, N, H, Hkv, d, B, G, causal = case
     w = synth.small_workload(seqlen=N, heads=H, kv_heads=Hkv, head_dim=d, groups=G, gamma=0.9, batch=B,
                              needles=8, seed=500 + PAIRING_CASES.index(case))
     x = synth.make_inputs(w)
     qc, kc, vc = x["q"], x["k"], x["v"]
     q, k, v = qc.cuda(), kc.cuda(), vc.cuda()
     qp, kp = pa.pool_heads(q, k, G)
-    mask = pa.build_mask(pa.block_scores(qp, kp, H, Hkv), q, k, G, pa.ALL)
+    mask = pa.build_mask(pa.block_scores(qp, kp, H, Hkv, causal=causal), q, k, G, pa.ALL, causal=causal)
     rank = mask.rank.cpu().numpy()
     nb = N // 128
     rng = np.random.default_rng(7)
     cnt = np.zeros((B, H, nb), np.int32)
     for b in range(B):
         for qb in range(nb):
-            n = qb + 1
+            n = qb + 1 if causal else nb
             pair_index = (nb - 1 - qb) // 2
             if pair_index % 2 == 0:   # budgets spread evenly from n/nh to n over the heads of a KV head
                 nh = H // Hkv
@@ -263,14 +266,14 @@ def test_attention_under_both_head_pairings(case):
         for kv in range(Hkv):
             hk, nh = kv * (H // Hkv), H // Hkv
             for qtop in range(nb - 1, 0, -2):
-                modes.add(pairs_by_head(cnt, b, hk, nh, qtop, nb))
+                modes.add(pairs_by_head(cnt, b, hk, nh, qtop, nb, causal))
     assert modes == {True, False}, modes
     cnt_t = torch.from_numpy(cnt).cuda()
-    o, lse = pa.block_sparse_attn(q, k, v, mask.rank, cnt_t, G, return_lse=True)
+    o, lse = pa.block_sparse_attn(q, k, v, mask.rank, cnt_t, G, return_lse=True, causal=causal)
     torch.cuda.synchronize()
     check_status()
     items = [(b, h, qb) for b in range(B) for h in range(H) for qb in range(nb)]
-    oref, lref = oracle.sparse_attn(qc, kc, vc, rank, cnt, G, items)
+    oref, lref = oracle.sparse_attn(qc, kc, vc, rank, cnt, G, items, causal=causal)
     og = o.float().cpu().numpy()
     lg = lse.cpu().numpy()
     ogi = np.stack([og[b, qb * 128:(qb + 1) * 128, h] for (b, h, qb) in items])
