@@ -58,13 +58,6 @@ constexpr int kRegsAux = 88;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsAux <= kAttnThreads * kRegsLaunch,
               "setmaxnreg split exceeds the registers the CTA is launched with");
 
-// Of every 8 column pairs of a non-diagonal S tile, this many take their
-// exponentials from the FMA-pipe polynomial instead of the MUFU unit.
-#ifndef PA_POLY_PAIRS_PER8
-#define PA_POLY_PAIRS_PER8 0
-#endif
-constexpr int kPolyPairsPer8 = PA_POLY_PAIRS_PER8;
-
 struct AttnParams {
     int B, N, H, Hkv, G, nb;
     int units_per_kv;          // max head units (CTAs) of one KV head per (b, qb): the grid stride
@@ -691,9 +684,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             // P = 2^(x - m) as bf16 pairs written over the first 64 columns of S.
             // Each column pair takes one packed FMA for x = s * scale - m and
-            // one packed add into four partial row sums; a share of the pairs
-            // of a non-diagonal tile takes its exponentials from the FMA-pipe
-            // polynomial instead of the MUFU unit.
+            // one packed add into four partial row sums.
             const float negm = (m == -INFINITY) ? 0.0f : -m;
             const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
             const float2 nm = make_float2(negm, negm);
@@ -703,26 +694,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t pk[32];
-                if (masked) {
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const int j = half * 32 + jj;
-                        const float2 x =
-                            __ffma2_rn(make_float2(__uint_as_float(s[2 * j]), __uint_as_float(s[2 * j + 1])), c2, nm);
-                        const float2 e = make_float2(ex2(x.x), ex2(x.y));
-                        acc[j & 3] = __fadd2_rn(acc[j & 3], e);
-                        pk[jj] = pack_bf16x2(e.x, e.y);
-                    }
-                } else {
-#pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        const int j = half * 32 + jj;
-                        const float2 x =
-                            __ffma2_rn(make_float2(__uint_as_float(s[2 * j]), __uint_as_float(s[2 * j + 1])), c2, nm);
-                        const float2 e = ((j & 7) < kPolyPairsPer8) ? ex2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
-                        acc[j & 3] = __fadd2_rn(acc[j & 3], e);
-                        pk[jj] = pack_bf16x2(e.x, e.y);
-                    }
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int j = half * 32 + jj;
+                    const float2 x =
+                        __ffma2_rn(make_float2(__uint_as_float(s[2 * j]), __uint_as_float(s[2 * j + 1])), c2, nm);
+                    const float2 e = make_float2(ex2(x.x), ex2(x.y));
+                    acc[j & 3] = __fadd2_rn(acc[j & 3], e);
+                    pk[jj] = pack_bf16x2(e.x, e.y);
                 }
                 tmem_st32(s_addr + half * 32, pk);
             }

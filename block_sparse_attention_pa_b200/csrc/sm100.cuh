@@ -310,31 +310,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
-// 2^x on the FMA pipe for a pair of values, x <= 64 (Cody & Waite range
-// reduction plus a degree-3 minimax polynomial for 2^f on [-1/2, 1/2],
-// relative error <= 7.5e-5; coefficients from csrc/exp2_poly.py), using the
-// packed two-lane fp32 add and FMA of sm_100 (one instruction per operation
-// for both values).  x = n + f with n the nearest integer (added into the
-// exponent field); inputs below -125 clamp there (the result is then below
-// 2^-124, zero for every use here).  f = x - n is formed as n * (-1) + x,
-// which is exact like the subtraction.
-constexpr float kEx2C3 = 5.517166853e-02f, kEx2C2 = 2.426111251e-01f, kEx2C1 = 6.932609677e-01f,
-                kEx2C0 = 9.999280572e-01f;
-constexpr float kEx2Round = 12582912.0f;  // 1.5 * 2^23: x + this holds round(x) in the low mantissa bits
-
-__device__ __forceinline__ float2 ex2_poly2(float2 x) {
-    x.x = fmaxf(x.x, -125.0f);
-    x.y = fmaxf(x.y, -125.0f);
-    const float2 j = __fadd2_rn(x, make_float2(kEx2Round, kEx2Round));
-    const float2 n = __fadd2_rn(j, make_float2(-kEx2Round, -kEx2Round));
-    const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), x);
-    float2 p = __ffma2_rn(make_float2(kEx2C3, kEx2C3), f, make_float2(kEx2C2, kEx2C2));
-    p = __ffma2_rn(p, f, make_float2(kEx2C1, kEx2C1));
-    p = __ffma2_rn(p, f, make_float2(kEx2C0, kEx2C0));
-    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(j.x) << 23)),
-                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(j.y) << 23)));
-}
-
 // Two fp32 values -> packed bf16x2 (round to nearest even); `lo` in bits 0..15.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
