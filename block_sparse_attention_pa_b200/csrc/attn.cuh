@@ -658,25 +658,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     continue;
                 }
             }
+            // The running max is raised only when it grows by more than 2^8; then O
+            // (in TMEM) and l scale by alpha = 2^(m - m_new).  O is scaled after this
+            // tile's P is stored, when the S registers are dead, and before P is
+            // handed over, so before this tile's PV adds into O.
             const float m_new = fmaxf(m, mt);
+            bool rescale = false;
+            float alpha = 1.0f;
             if (i > 0) {
                 const bool need = m_new > m + 8.0f;
                 if (__any_sync(0xffffffffu, need)) {
-                    // raise the running max: O (in TMEM) and l scale by 2^(m - m_new)
-                    const float alpha = (m == -INFINITY) ? 0.0f : ex2(m - m_new);
-                    // (this tile's S was committed after the head's last PV was issued,
-                    // and a commit covers every earlier MMA, so that PV is complete)
-                    tc_fence_after();
-#pragma unroll
-                    for (int ch = 0; ch < D / 32; ++ch) {
-                        uint32_t o[32];
-                        tmem_ld32(o_addr + ch * 32, o);
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                        tmem_st32(o_addr + ch * 32, o);
-                    }
-                    tmem_st_wait();
-                    l *= alpha;
+                    rescale = true;
+                    alpha = (m == -INFINITY) ? 0.0f : ex2(m - m_new);
                     m = m_new;
                 }
             } else {
@@ -705,7 +698,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
                 tmem_st32(s_addr + half * 32, pk);
             }
-            l += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+            l = l * alpha + (((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                             ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y)));
+            if (rescale) {
+                // (this tile's S was committed after the head's last PV was issued,
+                // and a commit covers every earlier MMA, so that PV is complete)
+                tc_fence_after();
+#pragma unroll
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    uint32_t o[32];
+                    tmem_ld32(o_addr + ch * 32, o);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                    tmem_st32(o_addr + ch * 32, o);
+                }
+            }
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&p_full[t]);
