@@ -12,7 +12,7 @@
 // Warp roles (384 threads = three warpgroups, one CTA per SM, all 512 TMEM
 // columns).  At the start the third warpgroup hands registers to the two
 // softmax warpgroups (setmaxnreg: 2 x 128 x 208 + 128 x 88 = 384 x 168):
-//   warps 0-3  softmax of head 0, warps 4-7 softmax of head 1 (below)
+//   warps 0-3  softmax of slot 0, warps 4-7 softmax of slot 1 (below)
 //   warp 8     TMA producer: the two Q tiles (issued before the CTA's setup
 //              barrier, so the copy overlaps the setup), then K and V tiles of the
 //              listed blocks into rings (128-byte swizzle).  V of tile i and K
@@ -23,12 +23,13 @@
 //                O_t += P_t V    (M=128, N=d,   A = P_t read from TMEM,
 //                                 B = V, MN-major smem)
 //              in ping-pong order  PV_0(i), QK_0(i+1), PV_1(i), QK_1(i+1), so
-//              the tensor core computes one head's products while the other
-//              head's softmax runs.
+//              the tensor core computes one slot's products while the other
+//              slot's softmax runs.
 //   softmax    one thread per query row (TMEM lane).  S is read from TMEM once; row max,
 //              then exp2/row sum/bf16 pack of P, written back over S; online
 //              softmax with the running max raised only when it grows by more
-//              than 2^8 (then O is rescaled in TMEM), final O/l and LSE.
+//              than 2^8 (then O is rescaled in TMEM, after the tile's P is
+//              stored and before it is handed over), final O/l and LSE.
 // TMEM columns: S_0 [0,128)  S_1 [128,256)  O_0 [256,384)  O_1 [384,512);
 // P_t (bf16 pairs) overwrites the first 64 columns of S_t.
 //
