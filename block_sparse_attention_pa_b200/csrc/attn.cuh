@@ -483,17 +483,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-                    umma_ss(tmem + t * 128, a + off, bk + off, IDESC_QK, kk > 0 ? 1u : 0u);
+                    if (kk == 0)
+                        umma_ss_c<false>(tmem + t * 128, a + off, bk + off, IDESC_QK);
+                    else
+                        umma_ss_c<true>(tmem + t * 128, a + off, bk + off, IDESC_QK);
                 }
                 umma_commit(&s_full[t]);
             };
             auto issue_pv = [&](int t, int s, bool accumulate) {
                 const uint64_t bv = dv0 + static_cast<uint64_t>((s * TB) >> 4);
                 const uint32_t acc0 = accumulate ? 1u : 0u;
+                umma_ts(tmem + 256 + t * 128, tmem + t * 128, bv, IDESC_PV, acc0);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)  // 128 keys, 16 per step
-                    umma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, bv + static_cast<uint64_t>(kk * 128),
-                            IDESC_PV, kk > 0 ? 1u : acc0);
+                for (int kk = 1; kk < 8; ++kk)  // 128 keys, 16 per step
+                    umma_ts_c<true>(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, bv + static_cast<uint64_t>(kk * 128),
+                                    IDESC_PV);
             };
             // Visit cursor: the bitmap word holding the current block, of both
             // heads, stays in registers, so shared memory is read once per 32
